@@ -1,0 +1,373 @@
+"""Benchmark of the gated delta-rule forward pass on B200.
+
+One step = one pass of the whole hot path over one batch: the chunkwise
+prefill (cumulative gate, UT transform, state pass, output) of the Gated
+DeltaNet workload (B=4, H=16, T=4096, dk=dv=128, chunk 64, bf16 q/k/v, fp32
+state), then one recurrent decode step that continues every (b, h) from the
+prefill's final state (prefill -> decode handoff).  The memory-bound decode
+workload (B=256, H=32, 512 MiB fp32 state, chained in-place steps) is timed in
+the same run and reported under "decode".
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+With N > 1 launch under torch.distributed.run: every rank runs its own batch
+(heads are independent: weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+
+from synth import CONFIGS, DECODE, decode_inputs, make_inputs, problem
+
+METRIC = "delta-rule fwd Mtokens·heads/s (prefill) & decode GB/s; % of roofline"
+WORKLOAD = "gdn_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- work model
+def flops_per_token_head(dk, dv, C):
+    """Algorithmic FLOPs of the chunkwise form per token and head (triangular masks exploited)."""
+    return C * (3 * dk + 2 * dv) + 6 * dk * dv + C * C / 3.0
+
+
+def prefill_bytes(p, with_S0):
+    """Algorithmic HBM bytes of one prefill: inputs read once, outputs written once."""
+    io = 2 if p.io == "bf16" else 4
+    per = io * (2 * p.dk + 2 * p.dv)
+    per += {"none": 0, "scalar": 4, "channel": 4 * p.dk}[p.alpha]
+    per += {"scalar": 4, "channel": 4 * p.dk}[p.beta_k]
+    per += {"none": 0, "scalar": 4, "channel": 4 * p.dv}[p.beta_v]
+    state = p.B * p.H * p.dk * p.dv * 4 * (2 if with_S0 else 1)
+    return p.token_heads * per + state
+
+
+def decode_bytes(B, H, dk, dv, io=2, alpha_ch=True, beta_ch=True):
+    """Per decode step: state read + write, q, k, v, o, gates."""
+    heads = B * H
+    per = 2 * dk * dv * 4 + io * (2 * dk + 2 * dv) + (4 * dk if alpha_ch else 4) + (4 * dk if beta_ch else 4)
+    return heads * per
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index, period=0.002):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self._stop = period, threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv is not None:
+            self.t.join()
+
+    def summary(self):
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- helpers
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(x, ws, device):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def to_dev(x, dev):
+    return {k: (None if t is None else t.to(dev)) for k, t in x.items()}
+
+
+def cpu_oracle_sample(p, seconds=12.0):
+    """Time the float64 oracle on a bounded sample of the prefill workload (whole heads, all T)."""
+    import oracle
+
+    threads = oracle.max_threads()
+    x = make_inputs(p.replace(B=max(1, min(p.B, threads // p.H))))
+    t0 = time.perf_counter()
+    oracle.delta_rule_sequential(x["q"], x["k"], x["v"], x["beta_k"], alpha=x["alpha"], beta_v=x["beta_v"],
+                                 S0=x["S0"], threads=threads)
+    dt = time.perf_counter() - t0
+    th = x["q"].shape[0] * x["q"].shape[1] * x["q"].shape[2]
+    return {"value": th / dt / 1e6, "unit": "Mtokens·heads/s", "cores": threads, "kind": "oracle",
+            "sample": f"{x['q'].shape[0] * x['q'].shape[2]} whole heads x T={p.T} of the {p.name} workload, float64, "
+                      f"{threads} OpenMP threads, {dt:.2f} s"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return 0
+    import oracle
+
+    p = CONFIGS[WORKLOAD]
+    threads = oracle.max_threads()
+    # each step: the oracle over a bounded sample of the workload (whole heads, full T)
+    sub = p.replace(B=max(1, min(p.B, threads // p.H)))
+    sample_heads = sub.B * sub.H
+    xs = make_inputs(sub)
+    run = lambda: oracle.delta_rule_sequential(xs["q"], xs["k"], xs["v"], xs["beta_k"], alpha=xs["alpha"],
+                                               beta_v=xs["beta_v"], S0=xs["S0"], threads=threads)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = (time.perf_counter() - t0) / args.steps
+    th = sample_heads * p.T
+    v = th / dt / 1e6
+    sample = f"{sample_heads} whole heads x T={p.T} of {p.name} per step, float64 oracle, {threads} threads"
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "Mtokens·heads/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": p.name, "B": p.B, "H": p.H, "T": p.T, "dk": p.dk, "dv": p.dv, "chunk": p.chunk},
+            "cpu_baseline": {"value": v, "unit": "Mtokens·heads/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": "Mtokens·heads/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    ws, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, ws, rank)
+    args.warmup = max(args.warmup, 3)
+
+    import weight_recurrence_chunkwise_b200 as dr
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    peaks, peaks_src = load_peaks()
+    st = torch.cuda.current_stream()
+
+    # ---------------- prefill -> decode step workload (every rank its own seeded batch)
+    p = CONFIGS[WORKLOAD].replace(seed=CONFIGS[WORKLOAD].seed + 1000 * rank)
+    x = to_dev(make_inputs(p), dev)
+    nxt = to_dev(make_inputs(p.replace(T=1, seed=p.seed + 500)), dev)  # the token after the prompt
+    o = torch.empty_like(x["v"])
+    S = torch.empty((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=dev)
+    o1 = torch.empty_like(nxt["v"])
+    ws_buf = torch.zeros(max(dr.workspace_bytes(dr.make_problem(x["q"], x["v"], x["alpha"], x["beta_k"],
+                                                                 x["beta_v"], p.chunk)), 256),
+                         dtype=torch.uint8, device=dev)
+
+    def step():
+        dr.dr_chunk_fwd(x["q"], x["k"], x["v"], x["beta_k"], alpha=x["alpha"], beta_v=x["beta_v"], S0=None,
+                        chunk=p.chunk, o=o, S_T=S, workspace=ws_buf, stream=st)
+        dr.dr_decode_step(nxt["q"], nxt["k"], nxt["v"], nxt["beta_k"], S, alpha=nxt["alpha"], o=o1, stream=st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert dr.dr_workspace_status(ws_buf) == dr.DR_OK
+
+    n = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(st)
+        for i in range(n):
+            ev[i][0].record(st)
+            dr.dr_chunk_fwd(x["q"], x["k"], x["v"], x["beta_k"], alpha=x["alpha"], beta_v=x["beta_v"], S0=None,
+                            chunk=p.chunk, o=o, S_T=S, workspace=ws_buf, stream=st)
+            ev[i][1].record(st)
+            dr.dr_decode_step(nxt["q"], nxt["k"], nxt["v"], nxt["beta_k"], S, alpha=nxt["alpha"], o=o1, stream=st)
+            ev[i][2].record(st)
+        t_end.record(st)
+        torch.cuda.synchronize()
+    barrier(ws)
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), ws, dev)
+    ms_step = ms_total / n
+    prefill_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    handoff_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    tok_heads = p.B * p.H * (p.T + 1)
+    value = tok_heads * ws / (ms_step / 1e3) / 1e6
+
+    # roofline of the dominant kernel (the fused chunk kernel), HBM-bound on algorithmic counts
+    byts = prefill_bytes(p, with_S0=False)
+    flops = p.token_heads * flops_per_token_head(p.dk, p.dv, p.chunk)
+    achieved_gbs = byts / (prefill_ms / 1e3) / 1e9
+    t_roof_ms = max(byts / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops_sustained"] * 1e12)) * 1e3
+    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks_src,
+                "kernel": "chunk_fwd_tc_kernel", "algorithmic_bytes_per_launch": byts,
+                "algorithmic_flops_per_launch": flops,
+                "tensor_tflops_achieved": flops / (prefill_ms / 1e3) / 1e12,
+                "roofline_time_ms": t_roof_ms, "frac_of_max_roofline": t_roof_ms / prefill_ms}
+
+    # ---------------- decode workload (B=256, H=32, 512 MiB state, chained in-place steps)
+    d = decode_inputs()
+    S_dec = d["S"].to(dev)
+    pool = {k: (None if d[k] is None else d[k].to(dev)) for k in ("q", "k", "v", "alpha", "beta_k")}
+    o_dec = torch.empty((DECODE.B, 1, DECODE.H, DECODE.dv), dtype=torch.bfloat16, device=dev)
+    del d
+
+    def dstep(i):
+        j = i % DECODE.pool
+        dr.dr_decode_step(pool["q"][j], pool["k"][j], pool["v"][j], pool["beta_k"][j], S_dec, alpha=pool["alpha"][j],
+                          o=o_dec, stream=st)
+
+    for i in range(3):
+        dstep(i)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for i in range(args.decode_steps):
+        dstep(i)
+    e1.record(st)
+    torch.cuda.synchronize()
+    dms = max_over_ranks(e0.elapsed_time(e1), ws, dev) / args.decode_steps
+    dbytes = decode_bytes(DECODE.B, DECODE.H, DECODE.dk, DECODE.dv)
+    dgbs = dbytes / (dms / 1e3) / 1e9
+    decode = {"value": dgbs * ws, "unit": "GB/s", "ms_per_step": dms, "steps": args.decode_steps,
+              "config": {"workload": DECODE.name, "B": DECODE.B, "H": DECODE.H, "dk": DECODE.dk, "dv": DECODE.dv,
+                         "state_MiB": DECODE.B * DECODE.H * DECODE.dk * DECODE.dv * 4 / 2 ** 20},
+              "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": dgbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks_src,
+                           "kernel": "decode_step_kernel", "algorithmic_bytes_per_launch": dbytes}}
+    del S_dec, pool
+
+    # ---------------- end to end through the public API with host buffers (pinned), copies timed
+    host = {k: (None if t is None else t.cpu().pin_memory()) for k, t in x.items()}
+    host_n = {k: (None if t is None else t.cpu().pin_memory()) for k, t in nxt.items()}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    S_h = torch.empty(S.shape, dtype=S.dtype).pin_memory()
+    o1_h = torch.empty(o1.shape, dtype=o1.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in list(host.values()) + list(host_n.values()) if t is not None)
+    d2h = o_h.numel() * o_h.element_size() + S_h.numel() * 4 + o1_h.numel() * o1_h.element_size()
+    e2e_steps = max(3, min(10, n))
+
+    def e2e_step():
+        g = {k: (None if t is None else t.to(dev, non_blocking=True)) for k, t in host.items()}
+        gn = {k: (None if t is None else t.to(dev, non_blocking=True)) for k, t in host_n.items()}
+        og, Sg = dr.dr_chunk_fwd(g["q"], g["k"], g["v"], g["beta_k"], alpha=g["alpha"], beta_v=g["beta_v"],
+                                 chunk=p.chunk, workspace=ws_buf, stream=st)
+        og1 = dr.dr_decode_step(gn["q"], gn["k"], gn["v"], gn["beta_k"], Sg, alpha=gn["alpha"], stream=st)
+        o_h.copy_(og, non_blocking=True)
+        S_h.copy_(Sg, non_blocking=True)
+        o1_h.copy_(og1, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0.record(st)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws, dev) / e2e_steps
+    e2e = {"value": tok_heads * ws / (e2e_ms / 1e3) / 1e6, "unit": "Mtokens·heads/s", "ms_per_step": e2e_ms,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(p)
+
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "Mtokens·heads/s", "n_gpus": ws, "steps": n,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": p.name, "B": p.B, "H": p.H, "T": p.T, "dk": p.dk, "dv": p.dv, "chunk": p.chunk,
+                   "step": "chunkwise prefill of T tokens + one decode step per (b,h)", "parallelism": f"dp{ws}",
+                   "l2": "inputs (275 MB per rank) larger than the 126 MB L2; no flush between steps"},
+        "prefill_ms": prefill_ms, "handoff_decode_ms": handoff_ms,
+        "roofline": roofline, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
+        "gpu_launches": 2 * n, "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,146 @@
+/*
+ * deltarule.h -- C ABI of the gated delta-rule forward pass on NVIDIA B200 (sm_100a).
+ *
+ * The operation (one independent recurrence per batch row b and head h):
+ *
+ *   b_t = sqrt(beta_k_t) (.) k_t                              erase key
+ *   w_t = beta_v_t (.) v_t   if beta_v is given,
+ *         sqrt(beta_k_t) (.) v_t   otherwise                  write vector
+ *   S_t = (I - b_t b_t^T) Diag(alpha_t) S_{t-1} + b_t w_t^T   S_t in R^{dk x dv}, fp32
+ *   o_t = S_t^T q_t                                           output (no 1/sqrt(d) scale)
+ *
+ * Sources of each part:
+ *   - DeltaNet page (robocikowo.com "DeltaNet"), numbered steps 1-6: per-token
+ *     q, k, v and a learning rate beta in (0, 1]; read the state with the key,
+ *     error beta (v - read), rank-1 write, output read from the updated
+ *     state.  That page writes the state transposed (dv x dk); here S is
+ *     dk x dv and reads are S^T x.
+ *   - FG2-GDN page (gist.science), section 1: Gated DeltaNet's scalar forget
+ *     factor alpha_t and KDA's channel-wise alpha_t in R^{dk}.
+ *   - FG2-GDN page, section 2 "Kerninnovation": channel-wise beta_t in R^{dk},
+ *     k~ = sqrt(beta) (.) k, v~ = sqrt(beta) (.) v and the update
+ *     S_t = (I - k~ k~^T) Diag(alpha_t) S_{t-1} + k~ v~^T.
+ *   - FG2-GDN page, section 2 "Erweiterung: FG2-GDN+": decoupled erase
+ *     strength beta^k and write strength beta^v (write vector beta^v (.) v).
+ *   - DeltaNet page, step 7 and the remarks on Householder-product
+ *     representations: training/prefill runs chunkwise over the sequence with
+ *     the WY/UT form on tensor cores; inference uses the recurrent form.
+ *
+ * Layouts (row-major, contiguous, caller-owned device memory):
+ *   q, k : [B, T, H, dk]  in io_dtype       v : [B, T, H, dv]  in io_dtype
+ *   o    : [B, T, H, dv]  in io_dtype
+ *   alpha  : NULL (alpha = 1), [B, T, H] (DR_SCALAR) or [B, T, H, dk] (DR_CHANNEL), fp32
+ *   beta_k : [B, T, H] (DR_SCALAR) or [B, T, H, dk] (DR_CHANNEL), fp32
+ *   beta_v : NULL (symmetric write, sqrt(beta_k) (.) v), [B, T, H] or [B, T, H, dv], fp32
+ *   S0, S_T, S : [B, H, dk, dv] fp32.  S0 == NULL means a zero initial state.
+ * The symmetric channel-wise form (beta_v == NULL, beta_k channel-wise) needs dk == dv.
+ * Every pointer must be 16-byte aligned.
+ *
+ * Supported sizes: dk, dv in {64, 128}; chunk in {16, 32, 64}; T >= 0 (a
+ * partial last chunk is handled); B, H >= 1.
+ *
+ * Ownership and threading: the caller owns every buffer; the library
+ * allocates no device memory and keeps no state between calls.  All work is
+ * enqueued on the caller's stream (a cudaStream_t passed as void*, NULL = the
+ * legacy default stream); no call synchronises.  S_T may alias S0.
+ *
+ * Errors: argument checks run on the host before anything is enqueued and
+ * return DR_ERR_INVALID_ARG / DR_ERR_UNSUPPORTED / DR_ERR_ALIGNMENT /
+ * DR_ERR_WORKSPACE; a failed launch returns DR_ERR_CUDA.  Conditions found on
+ * the device (a chunk whose cumulative decay leaves the representable range,
+ * or a bounded wait that expired) are recorded in the workspace status word
+ * and read back with dr_workspace_status() after the caller's stream has
+ * been synchronised.
+ */
+#ifndef DELTARULE_H
+#define DELTARULE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifndef DR_API
+#if defined(__GNUC__)
+#define DR_API __attribute__((visibility("default")))
+#else
+#define DR_API
+#endif
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DR_OK = 0,
+  DR_ERR_INVALID_ARG = 1,   /* NULL required pointer, negative size, mode/shape mismatch */
+  DR_ERR_UNSUPPORTED = 2,   /* valid but not implemented: dk/dv/chunk outside the lists above */
+  DR_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
+  DR_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than dr_chunk_fwd_workspace() */
+  DR_ERR_RANGE = 5,         /* device: cumulative decay inside a chunk below the factorised range */
+  DR_ERR_TIMEOUT = 6,       /* device: a bounded wait expired; outputs are invalid */
+  DR_ERR_CUDA = 7           /* a CUDA runtime call or kernel launch failed */
+} dr_status;
+
+typedef enum { DR_F32 = 0, DR_BF16 = 1 } dr_dtype;
+
+typedef enum { DR_ABSENT = 0, DR_SCALAR = 1, DR_CHANNEL = 2 } dr_mode;
+
+typedef struct {
+  int B, T, H;          /* batch, sequence length (tokens), heads */
+  int dk, dv;           /* key and value head dimensions */
+  int chunk;            /* chunk length C of the WY/UT form (prefill only) */
+  dr_dtype io_dtype;    /* dtype of q, k, v, o */
+  dr_mode alpha_mode;   /* DR_ABSENT, DR_SCALAR or DR_CHANNEL (per key channel) */
+  dr_mode beta_k_mode;  /* DR_SCALAR or DR_CHANNEL (per key channel) */
+  dr_mode beta_v_mode;  /* DR_ABSENT, DR_SCALAR or DR_CHANNEL (per value channel) */
+} dr_problem;
+
+/* Bytes of device workspace dr_chunk_fwd needs for problem p (status word).  0 if p is invalid. */
+DR_API size_t dr_chunk_fwd_workspace(const dr_problem *p);
+
+/*
+ * Chunkwise prefill: all T tokens of every (b, h), starting from S0, writing
+ * o_t for every token and the final state S_T.  Computed with the chunkwise
+ * WY/UT (Householder-product) form: per chunk of C tokens the cumulative
+ * gate, the UT transform T = (I + strictly-lower(B^ A^T))^-1, the serial
+ * inter-chunk state pass in fp32 and the intra-chunk output (DeltaNet page,
+ * step 7; FG2-GDN page, section 2, DPLR/WY remark).
+ * workspace: device memory of at least dr_chunk_fwd_workspace(p) bytes,
+ * reused across calls on the same stream; its status word is reset at the
+ * start of every call.
+ */
+DR_API dr_status dr_chunk_fwd(const dr_problem *p,
+                       const void *q, const void *k, const void *v,
+                       const float *alpha, const float *beta_k, const float *beta_v,
+                       const float *S0, void *o, float *S_T,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One recurrent decode step for every (b, h) (DeltaNet page, steps 3-6 and
+ * "inference uses the recurrent form"): reads S, writes the updated state
+ * back into S in place and the output o.  p->T must be 1; p->chunk is
+ * ignored.  q, k, v, o use the [B, 1, H, d] layouts above.
+ */
+DR_API dr_status dr_decode_step(const dr_problem *p,
+                         const void *q, const void *k, const void *v,
+                         const float *alpha, const float *beta_k, const float *beta_v,
+                         float *S, void *o, void *stream);
+
+/*
+ * Synchronises `stream`, then reads the status word a previous dr_chunk_fwd
+ * left in `workspace` (DR_OK, DR_ERR_RANGE or DR_ERR_TIMEOUT).  Returns
+ * DR_ERR_CUDA if the copy fails.
+ */
+DR_API dr_status dr_workspace_status(const void *workspace, void *stream);
+
+/* Static, human-readable name of a status code. */
+DR_API const char *dr_status_string(dr_status s);
+
+/* Library ABI version (major * 100 + minor). */
+DR_API int dr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DELTARULE_H */

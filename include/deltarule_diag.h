@@ -1,0 +1,41 @@
+/*
+ * deltarule_diag.h -- diagnostic entry points of libdeltarule (not part of the
+ * operation itself; the pages have no counterpart).  They exercise the
+ * tensor-core building blocks of the prefill kernel in isolation so that a
+ * layout or descriptor fault is found before it hides inside the full kernel.
+ */
+#ifndef DELTARULE_DIAG_H
+#define DELTARULE_DIAG_H
+
+#include <stddef.h>
+
+#ifndef DR_API
+#if defined(__GNUC__)
+#define DR_API __attribute__((visibility("default")))
+#else
+#define DR_API
+#endif
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * D[128 x N] = A[128 x K] * B[K x N] on one CTA through tcgen05.mma (16-bit
+ * inputs: bf16 if bf16 != 0, else fp16; fp32 accumulate), with A staged
+ * K-major (a_mn = 0) or MN-major (a_mn = 1)
+ * and B staged K-major (b_mn = 0) or MN-major (b_mn = 1) in 128-byte-swizzled
+ * shared memory, the result read back from tensor memory.
+ * A, B: row-major 16-bit device buffers; D: row-major fp32 device buffer;
+ * workspace: >= 256 bytes of device memory (status word, same meaning as in
+ * dr_workspace_status).  N, K in {64, 128}.  Returns a dr_status code.
+ */
+DR_API int dr_diag_umma_selftest(int N, int K, int a_mn, int b_mn, int bf16, const void *A, const void *B,
+                                 float *D, void *workspace, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DELTARULE_DIAG_H */

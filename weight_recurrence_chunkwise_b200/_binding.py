@@ -1,0 +1,169 @@
+"""ctypes binding of ``libdeltarule.so`` (include/deltarule.h).
+
+Argument marshalling only: shapes become a ``dr_problem``, tensors become
+device pointers, status codes become exceptions.  Every step of the operation
+runs inside the library's CUDA kernels; there is no host or PyTorch fallback,
+and a missing library is an error.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdeltarule.so")
+
+DR_OK, DR_ERR_INVALID_ARG, DR_ERR_UNSUPPORTED, DR_ERR_ALIGNMENT = 0, 1, 2, 3
+DR_ERR_WORKSPACE, DR_ERR_RANGE, DR_ERR_TIMEOUT, DR_ERR_CUDA = 4, 5, 6, 7
+DR_F32, DR_BF16 = 0, 1
+DR_ABSENT, DR_SCALAR, DR_CHANNEL = 0, 1, 2
+
+_DTYPE = {torch.float32: DR_F32, torch.bfloat16: DR_BF16}
+
+
+class dr_problem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("chunk", ctypes.c_int),
+                ("io_dtype", ctypes.c_int), ("alpha_mode", ctypes.c_int),
+                ("beta_k_mode", ctypes.c_int), ("beta_v_mode", ctypes.c_int)]
+
+
+class DeltaRuleError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)}")
+
+
+_lib = None
+
+EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_decode_step", "dr_workspace_status",
+           "dr_status_string", "dr_version", "dr_diag_umma_selftest")
+
+
+def lib():
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with weight_recurrence_chunkwise_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, P = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(dr_problem)
+        L.dr_chunk_fwd_workspace.argtypes = [P]
+        L.dr_chunk_fwd_workspace.restype = sz
+        L.dr_chunk_fwd.argtypes = [P] + [vp] * 9 + [vp, sz, vp]
+        L.dr_chunk_fwd.restype = ctypes.c_int
+        L.dr_decode_step.argtypes = [P] + [vp] * 8 + [vp]
+        L.dr_decode_step.restype = ctypes.c_int
+        L.dr_workspace_status.argtypes = [vp, vp]
+        L.dr_workspace_status.restype = ctypes.c_int
+        L.dr_status_string.argtypes = [ctypes.c_int]
+        L.dr_status_string.restype = ctypes.c_char_p
+        L.dr_version.argtypes = []
+        L.dr_version.restype = ctypes.c_int
+        L.dr_diag_umma_selftest.argtypes = [ctypes.c_int] * 5 + [vp, vp, vp, vp, vp]
+        L.dr_diag_umma_selftest.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().dr_status_string(int(code)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _mode(x, scalar_ndim):
+    if x is None:
+        return DR_ABSENT
+    return DR_SCALAR if x.dim() == scalar_ndim else DR_CHANNEL
+
+
+def make_problem(q, v, alpha, beta_k, beta_v, chunk=64) -> dr_problem:
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype not in _DTYPE:
+        raise TypeError(f"unsupported I/O dtype {q.dtype}")
+    return dr_problem(B, T, H, dk, dv, int(chunk), _DTYPE[q.dtype], _mode(alpha, 3),
+                      _mode(beta_k, 3), _mode(beta_v, 3))
+
+
+def _check_tensors(io_dtype, named):
+    for name, t in named:
+        if t is None:
+            continue
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+        want = io_dtype if name in ("q", "k", "v", "o") else torch.float32
+        if t.dtype != want:
+            raise TypeError(f"{name} must be {want}, got {t.dtype}")
+
+
+def workspace_bytes(problem: dr_problem) -> int:
+    return int(lib().dr_chunk_fwd_workspace(ctypes.byref(problem)))
+
+
+def dr_chunk_fwd(q, k, v, beta_k, alpha=None, beta_v=None, S0=None, chunk=64, o=None, S_T=None,
+                 workspace=None, stream=None, final_state=True):
+    """Chunkwise prefill.  Returns ``(o, S_T)``; S_T is None when ``final_state`` is False."""
+    p = make_problem(q, v, alpha, beta_k, beta_v, chunk)
+    dev = q.device
+    if o is None:
+        o = torch.empty(q.shape[:3] + (p.dv,), dtype=q.dtype, device=dev)
+    if S_T is None and final_state:
+        S_T = torch.empty((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=dev)
+    _check_tensors(q.dtype, [("q", q), ("k", k), ("v", v), ("o", o), ("alpha", alpha),
+                             ("beta_k", beta_k), ("beta_v", beta_v), ("S0", S0), ("S_T", S_T)])
+    need = workspace_bytes(p)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    rc = lib().dr_chunk_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
+                            _ptr(beta_v), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+                            ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if rc != DR_OK:
+        raise DeltaRuleError(rc, "dr_chunk_fwd")
+    return o, S_T
+
+
+def dr_decode_step(q, k, v, beta_k, S, alpha=None, beta_v=None, o=None, stream=None):
+    """One recurrent step for every (b, h); updates ``S`` in place and returns ``o``.
+
+    q, k: [B, 1, H, dk]; v: [B, 1, H, dv]; gates [B, 1, H] or [B, 1, H, d]; S [B, H, dk, dv].
+    """
+    p = make_problem(q, v, alpha, beta_k, beta_v, 0)
+    if o is None:
+        o = torch.empty(q.shape[:3] + (p.dv,), dtype=q.dtype, device=q.device)
+    _check_tensors(q.dtype, [("q", q), ("k", k), ("v", v), ("o", o), ("alpha", alpha),
+                             ("beta_k", beta_k), ("beta_v", beta_v), ("S", S)])
+    rc = lib().dr_decode_step(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
+                              _ptr(beta_v), _ptr(S), _ptr(o), _stream(stream))
+    if rc != DR_OK:
+        raise DeltaRuleError(rc, "dr_decode_step")
+    return o
+
+
+def dr_workspace_status(workspace, stream=None) -> int:
+    return int(lib().dr_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def dr_diag_umma_selftest(A, B, a_mn: bool, b_mn: bool, stream=None):
+    """128 x N product of bf16 or fp16 A, B through the tcgen05 building blocks; returns (D, status)."""
+    K, N = B.shape
+    if A.dtype != B.dtype or A.dtype not in (torch.bfloat16, torch.float16):
+        raise TypeError("A and B must both be bf16 or both fp16")
+    D = torch.empty((A.shape[0], N), dtype=torch.float32, device=A.device)
+    ws = torch.zeros(256, dtype=torch.uint8, device=A.device)
+    rc = lib().dr_diag_umma_selftest(N, K, int(a_mn), int(b_mn), int(A.dtype == torch.bfloat16), _ptr(A), _ptr(B), _ptr(D), _ptr(ws),
+                                     _stream(stream))
+    if rc != DR_OK:
+        raise DeltaRuleError(rc, "dr_diag_umma_selftest")
+    return D, dr_workspace_status(ws, stream)

@@ -1,0 +1,237 @@
+// deltarule_api.cu -- the C ABI declared in include/deltarule.h: argument
+// checks, workspace status word, and dispatch to the sm_100a kernels.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/deltarule.h"
+#include "../../include/deltarule_diag.h"
+#include "chunk_simt.cuh"
+#include "chunk_tc.cuh"
+#include "common.cuh"
+#include "decode.cuh"
+#include "umma_selftest.cuh"
+
+namespace {
+
+constexpr size_t kWorkspaceBytes = 256;  // status word, padded to an allocation granule
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dr_status check_common(const dr_problem *p, bool decode) {
+  if (!p) return DR_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->T < 0 || p->dk <= 0 || p->dv <= 0) return DR_ERR_INVALID_ARG;
+  if (decode && p->T != 1) return DR_ERR_INVALID_ARG;
+  if (!decode && p->chunk <= 0) return DR_ERR_INVALID_ARG;
+  if (p->io_dtype != DR_F32 && p->io_dtype != DR_BF16) return DR_ERR_INVALID_ARG;
+  if (p->alpha_mode < DR_ABSENT || p->alpha_mode > DR_CHANNEL) return DR_ERR_INVALID_ARG;
+  if (p->beta_k_mode != DR_SCALAR && p->beta_k_mode != DR_CHANNEL) return DR_ERR_INVALID_ARG;
+  if (p->beta_v_mode < DR_ABSENT || p->beta_v_mode > DR_CHANNEL) return DR_ERR_INVALID_ARG;
+  // sqrt(beta) (.) v with beta in R^{dk} only type-checks when dk == dv
+  if (p->beta_v_mode == DR_ABSENT && p->beta_k_mode == DR_CHANNEL && p->dk != p->dv) return DR_ERR_INVALID_ARG;
+  if ((p->dk != 64 && p->dk != 128) || (p->dv != 64 && p->dv != 128)) return DR_ERR_UNSUPPORTED;
+  if (!decode && p->chunk != 16 && p->chunk != 32 && p->chunk != 64) return DR_ERR_UNSUPPORTED;
+  const double elems = double(p->B) * p->T * p->H * (p->dk > p->dv ? p->dk : p->dv);
+  if (elems > 9.0e15) return DR_ERR_INVALID_ARG;
+  return DR_OK;
+}
+
+dr_status check_pointers(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                         const float *beta_k, const float *beta_v, const void *o) {
+  const bool need_tokens = p->T > 0;
+  if (need_tokens && (!q || !k || !v || !o || !beta_k)) return DR_ERR_INVALID_ARG;
+  if (need_tokens && ((alpha == nullptr) != (p->alpha_mode == DR_ABSENT))) return DR_ERR_INVALID_ARG;
+  if (need_tokens && ((beta_v == nullptr) != (p->beta_v_mode == DR_ABSENT))) return DR_ERR_INVALID_ARG;
+  const void *ptrs[] = {q, k, v, alpha, beta_k, beta_v, o};
+  for (const void *x : ptrs)
+    if (x && !aligned16(x)) return DR_ERR_ALIGNMENT;
+  return DR_OK;
+}
+
+dr_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------- prefill, CUDA-core path
+template <typename IO, int DK, int DV, int C>
+dr_status simt_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                      const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
+                      uint32_t *status, cudaStream_t st) {
+  constexpr int VS = 32;
+  auto kern = dr::chunk_fwd_simt_kernel<IO, DK, DV, VS, C>;
+  constexpr size_t smem = dr::SimtSmem<DK, VS, C>::bytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return DR_ERR_CUDA;
+  dim3 grid(DV / VS, p->H, p->B);
+  kern<<<grid, 256, smem, st>>>(p->T, p->H, static_cast<const IO *>(q), static_cast<const IO *>(k),
+                                static_cast<const IO *>(v), alpha, p->alpha_mode, beta_k, p->beta_k_mode,
+                                beta_v, p->beta_v_mode, S0, static_cast<IO *>(o), S_T, status);
+  return launch_status();
+}
+
+template <typename IO, int DK, int DV>
+dr_status simt_by_chunk(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                        const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
+                        uint32_t *status, cudaStream_t st) {
+  switch (p->chunk) {
+    case 16: return simt_launch<IO, DK, DV, 16>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+    case 32: return simt_launch<IO, DK, DV, 32>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+    default: return simt_launch<IO, DK, DV, 64>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+  }
+}
+
+template <typename IO>
+dr_status simt_dispatch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                        const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
+                        uint32_t *status, cudaStream_t st) {
+  if (p->dk == 128 && p->dv == 128)
+    return simt_by_chunk<IO, 128, 128>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+  if (p->dk == 128 && p->dv == 64)
+    return simt_by_chunk<IO, 128, 64>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+  if (p->dk == 64 && p->dv == 128)
+    return simt_by_chunk<IO, 64, 128>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+  return simt_by_chunk<IO, 64, 64>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+}
+
+// ----------------------------------------------------------------- prefill, tensor-core path (bf16 I/O)
+dr_status tc_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                    const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
+                    uint32_t *status, cudaStream_t st) {
+  using IO = __nv_bfloat16;
+  auto kern = dr::tc::chunk_fwd_tc_kernel<IO>;
+  constexpr size_t smem = dr::tc::SMEM_BYTES;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return DR_ERR_CUDA;
+  dim3 grid(p->dv / dr::tc::VS, p->H, p->B);
+  kern<<<grid, dr::tc::NT, smem, st>>>(p->T, p->H, p->dv, static_cast<const IO *>(q), static_cast<const IO *>(k),
+                                       static_cast<const IO *>(v), alpha, p->alpha_mode, beta_k, p->beta_k_mode,
+                                       beta_v, p->beta_v_mode, S0, static_cast<IO *>(o), S_T, status);
+  return launch_status();
+}
+
+// ----------------------------------------------------------------- decode
+template <typename IO, int DK, int DV>
+dr_status decode_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                        const float *beta_k, const float *beta_v, float *S, void *o, cudaStream_t st) {
+  const long long heads = static_cast<long long>(p->B) * p->H;
+  if (heads > 0x7fffffffLL) return DR_ERR_INVALID_ARG;
+  dr::decode_step_kernel<IO, DK, DV><<<static_cast<unsigned>(heads), 256, 0, st>>>(
+      static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v), alpha, p->alpha_mode,
+      beta_k, p->beta_k_mode, beta_v, p->beta_v_mode, S, static_cast<IO *>(o));
+  return launch_status();
+}
+
+template <typename IO>
+dr_status decode_dispatch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                          const float *beta_k, const float *beta_v, float *S, void *o, cudaStream_t st) {
+  if (p->dk == 128 && p->dv == 128) return decode_launch<IO, 128, 128>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
+  if (p->dk == 128 && p->dv == 64) return decode_launch<IO, 128, 64>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
+  if (p->dk == 64 && p->dv == 128) return decode_launch<IO, 64, 128>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
+  return decode_launch<IO, 64, 64>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int dr_version(void) { return 100; }
+
+const char *dr_status_string(dr_status s) {
+  switch (s) {
+    case DR_OK: return "DR_OK";
+    case DR_ERR_INVALID_ARG: return "DR_ERR_INVALID_ARG: invalid argument";
+    case DR_ERR_UNSUPPORTED: return "DR_ERR_UNSUPPORTED: size or mode not supported";
+    case DR_ERR_ALIGNMENT: return "DR_ERR_ALIGNMENT: pointer not 16-byte aligned";
+    case DR_ERR_WORKSPACE: return "DR_ERR_WORKSPACE: workspace missing or too small";
+    case DR_ERR_RANGE: return "DR_ERR_RANGE: cumulative decay in a chunk below the supported range";
+    case DR_ERR_TIMEOUT: return "DR_ERR_TIMEOUT: a bounded device wait expired";
+    case DR_ERR_CUDA: return "DR_ERR_CUDA: CUDA call or launch failed";
+  }
+  return "unknown dr_status";
+}
+
+size_t dr_chunk_fwd_workspace(const dr_problem *p) {
+  return check_common(p, false) == DR_OK ? kWorkspaceBytes : 0;
+}
+
+dr_status dr_chunk_fwd(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                       const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+  dr_status s = check_common(p, false);
+  if (s != DR_OK) return s;
+  s = check_pointers(p, q, k, v, alpha, beta_k, beta_v, o);
+  if (s != DR_OK) return s;
+  if ((S0 && !aligned16(S0)) || (S_T && !aligned16(S_T))) return DR_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < kWorkspaceBytes) return DR_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return DR_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *status = static_cast<uint32_t *>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DR_ERR_CUDA;
+  const size_t state_bytes = sizeof(float) * size_t(p->B) * p->H * p->dk * p->dv;
+  if (p->T == 0) {  // nothing to scan: the final state is the initial state
+    if (!S_T) return DR_OK;
+    const cudaError_t e = S0 ? (S0 == S_T ? cudaSuccess
+                                          : cudaMemcpyAsync(S_T, S0, state_bytes, cudaMemcpyDeviceToDevice, st))
+                             : cudaMemsetAsync(S_T, 0, state_bytes, st);
+    return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+  }
+  if (p->io_dtype == DR_F32)
+    return simt_dispatch<float>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+  if (p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv % dr::tc::VS == 0)
+    return tc_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+  return simt_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+}
+
+dr_status dr_decode_step(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                         const float *beta_k, const float *beta_v, float *S, void *o, void *stream) {
+  dr_status s = check_common(p, true);
+  if (s != DR_OK) return s;
+  s = check_pointers(p, q, k, v, alpha, beta_k, beta_v, o);
+  if (s != DR_OK) return s;
+  if (!S) return DR_ERR_INVALID_ARG;
+  if (!aligned16(S)) return DR_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p->io_dtype == DR_F32) return decode_dispatch<float>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
+  return decode_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
+}
+
+dr_status dr_workspace_status(const void *workspace, void *stream) {
+  if (!workspace) return DR_ERR_WORKSPACE;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DR_ERR_CUDA;
+  uint32_t w = 0;
+  if (cudaMemcpy(&w, workspace, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return DR_ERR_CUDA;
+  if (w & dr::STATUS_TIMEOUT) return DR_ERR_TIMEOUT;
+  if (w & dr::STATUS_RANGE) return DR_ERR_RANGE;
+  return DR_OK;
+}
+
+int dr_diag_umma_selftest(int N, int K, int a_mn, int b_mn, int bf16, const void *A, const void *B, float *D,
+                          void *workspace, void *stream) {
+  if (!A || !B || !D || !workspace) return DR_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *status = static_cast<uint32_t *>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DR_ERR_CUDA;
+  const size_t smem = 1024 + size_t(128) * K * 2 + size_t(K) * N * 2;
+  const auto *a = static_cast<const uint16_t *>(A);
+  const auto *b = static_cast<const uint16_t *>(B);
+#define DR_SELFTEST_CASE(NN, KK)                                                                      \
+  if (N == NN && K == KK) {                                                                           \
+    auto kern = dr::umma_selftest_kernel<NN, KK>;                                                     \
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess) \
+      return DR_ERR_CUDA;                                                                             \
+    kern<<<1, 128, smem, st>>>(a, b, D, a_mn, b_mn, bf16, status);                                          \
+    return launch_status();                                                                           \
+  }
+  DR_SELFTEST_CASE(64, 64)
+  DR_SELFTEST_CASE(64, 128)
+  DR_SELFTEST_CASE(128, 64)
+  DR_SELFTEST_CASE(128, 128)
+#undef DR_SELFTEST_CASE
+  return DR_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

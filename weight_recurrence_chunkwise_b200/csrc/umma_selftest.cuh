@@ -1,0 +1,80 @@
+// umma_selftest.cuh -- diagnostic: one 128 x N x K bf16 or fp16 product through the exact
+// tcgen05 building blocks the prefill kernel uses (128-byte swizzled shared
+// tiles written by threads, K-major and MN-major smem descriptors, the kind::f16
+// instruction descriptor, commit to an mbarrier, TMEM allocation and the
+// 32x32b TMEM load).  The tests compare it with a host matmul so that a layout
+// or descriptor mistake shows up in isolation.
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace dr {
+
+// A, Bm: 16-bit elements, bf16 (bf16 != 0) or fp16.
+template <int N, int K>
+__global__ void __launch_bounds__(128)
+umma_selftest_kernel(const uint16_t *__restrict__ A, const uint16_t *__restrict__ Bm,
+                     float *__restrict__ D, int a_mn, int b_mn, int bf16, uint32_t *status) {
+  constexpr int M = 128;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tmem_base;
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = base;
+  uint8_t *sB = base + M * K * 2;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  for (int e = tid; e < M * K; e += blockDim.x) {
+    const int m = e / K, kk = e % K;
+    const uint32_t off = a_mn ? sw128_off(kk, m, K) : sw128_off(m, kk, M);
+    *reinterpret_cast<uint16_t *>(sA + off) = A[e];
+  }
+  for (int e = tid; e < K * N; e += blockDim.x) {
+    const int kk = e / N, n = e % N;
+    const uint32_t off = b_mn ? sw128_off(kk, n, K) : sw128_off(n, kk, N);
+    *reinterpret_cast<uint16_t *>(sB + off) = Bm[e];
+  }
+  fence_async_smem();
+  if (warp == 0) {
+    tmem_alloc(&tmem_base, 128);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tmem_base;
+  if (tid == 0) {
+    const uint32_t idesc = idesc_f16_f32(M, N, a_mn != 0, b_mn != 0, bf16 != 0);
+#pragma unroll
+    for (int kk = 0; kk < K / 16; ++kk) {
+      const uint64_t ad = a_mn ? desc_mnmajor(smem_u32(sA), K, kk) : desc_kmajor(smem_u32(sA), M, kk);
+      const uint64_t bd = b_mn ? desc_mnmajor(smem_u32(sB), K, kk) : desc_kmajor(smem_u32(sB), N, kk);
+      umma_f16(tb, ad, bd, idesc, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&bar);
+  }
+  const bool ok = mbar_wait(&bar, 0, kWaitLimitNs);
+  tc_fence_after();
+  if (!ok) {
+    if (lane == 0) raise_status(status, STATUS_TIMEOUT);
+  } else {
+#pragma unroll
+    for (int c0 = 0; c0 < N; c0 += 16) {
+      float vals[16];
+      tmem_ld16(tmem_addr(tb, 32 * warp, c0), vals);
+      tmem_ld_wait();
+      const int row = 32 * warp + lane;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) D[row * N + c0 + i] = vals[i];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 128);
+}
+
+}  // namespace dr
