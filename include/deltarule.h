@@ -127,6 +127,36 @@ DR_API dr_status dr_decode_step(const dr_problem *p,
                          float *S, void *o, void *stream);
 
 /*
+ * dr_chunk_fwd for callers that cannot allocate device memory.  (The pages
+ * have no counterpart; this is a deployment variant of dr_chunk_fwd.)  Some
+ * hosts pre-plan every byte of device memory and give a kernel no workspace
+ * hook -- plugin interfaces of inference runtimes, memory-budgeted serving
+ * loops -- and some loops cannot afford cudaMalloc/cudaFree at all, since
+ * cudaFree synchronises the device and cudaMalloc may.  This entry point
+ * takes the same inputs and outputs as dr_chunk_fwd but no workspace: the
+ * scratch dr_chunk_fwd would keep in the workspace (its device status word)
+ * lives in a file-scope device array of 4096 bytes inside the library, which
+ * every GPU that loads the library holds until the process exits.  A problem
+ * whose dr_chunk_fwd_workspace() exceeds 4096 bytes is rejected with
+ * DR_ERR_WORKSPACE before anything is enqueued.  The call allocates nothing
+ * (no cudaMalloc, no cudaFree, no allocating library routine).
+ * Device and set-up: the GPU used is the current device, which must be the
+ * device of `stream`.  The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress) and caches it; make that first call
+ * before any stream capture.
+ * Sharing: every call on a device uses the same array, which keeps the last
+ * call's contents; each call clears the status word on its own stream before
+ * its kernel runs.  Calls whose work overlaps on the GPU (several streams, or
+ * several host threads) race on that word, so its device-side status is only
+ * meaningful for calls that do not overlap; the array is not readable
+ * through dr_workspace_status.
+ */
+DR_API dr_status dr_chunk_fwd_noalloc(const dr_problem *p,
+                                      const void *q, const void *k, const void *v,
+                                      const float *alpha, const float *beta_k, const float *beta_v,
+                                      const float *S0, void *o, float *S_T, void *stream);
+
+/*
  * Synchronises `stream`, then reads the status word a previous dr_chunk_fwd
  * left in `workspace` (DR_OK, DR_ERR_RANGE or DR_ERR_TIMEOUT).  Returns
  * DR_ERR_CUDA if the copy fails.

@@ -38,8 +38,8 @@ class DeltaRuleError(RuntimeError):
 
 _lib = None
 
-EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_decode_step", "dr_workspace_status",
-           "dr_status_string", "dr_version", "dr_diag_umma_selftest")
+EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_chunk_fwd_noalloc", "dr_decode_step",
+           "dr_workspace_status", "dr_status_string", "dr_version", "dr_diag_umma_selftest")
 
 
 def lib():
@@ -54,6 +54,8 @@ def lib():
         L.dr_chunk_fwd_workspace.restype = sz
         L.dr_chunk_fwd.argtypes = [P] + [vp] * 9 + [vp, sz, vp]
         L.dr_chunk_fwd.restype = ctypes.c_int
+        L.dr_chunk_fwd_noalloc.argtypes = [P] + [vp] * 9 + [vp]
+        L.dr_chunk_fwd_noalloc.restype = ctypes.c_int
         L.dr_decode_step.argtypes = [P] + [vp] * 8 + [vp]
         L.dr_decode_step.restype = ctypes.c_int
         L.dr_workspace_status.argtypes = [vp, vp]
@@ -131,6 +133,28 @@ def dr_chunk_fwd(q, k, v, beta_k, alpha=None, beta_v=None, S0=None, chunk=64, o=
                             ctypes.c_size_t(workspace.numel()), _stream(stream))
     if rc != DR_OK:
         raise DeltaRuleError(rc, "dr_chunk_fwd")
+    return o, S_T
+
+
+def dr_chunk_fwd_noalloc(q, k, v, beta_k, alpha=None, beta_v=None, S0=None, chunk=64, o=None, S_T=None,
+                         stream=None):
+    """dr_chunk_fwd without a workspace, for callers that cannot allocate device memory.
+
+    The library keeps the scratch in a static device array; ``o`` and ``S_T``
+    must be passed in by such callers (they are only allocated here when
+    omitted, as a convenience for tests).  Returns ``(o, S_T)``.
+    """
+    p = make_problem(q, v, alpha, beta_k, beta_v, chunk)
+    if o is None:
+        o = torch.empty(q.shape[:3] + (p.dv,), dtype=q.dtype, device=q.device)
+    if S_T is None:
+        S_T = torch.empty((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=q.device)
+    _check_tensors(q.dtype, [("q", q), ("k", k), ("v", v), ("o", o), ("alpha", alpha),
+                             ("beta_k", beta_k), ("beta_v", beta_v), ("S0", S0), ("S_T", S_T)])
+    rc = lib().dr_chunk_fwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
+                                    _ptr(beta_v), _ptr(S0), _ptr(o), _ptr(S_T), _stream(stream))
+    if rc != DR_OK:
+        raise DeltaRuleError(rc, "dr_chunk_fwd_noalloc")
     return o, S_T
 
 

@@ -4,6 +4,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/deltarule.h"
 #include "../../include/deltarule_diag.h"
@@ -197,6 +198,44 @@ dr_status dr_decode_step(const dr_problem *p, const void *q, const void *k, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (p->io_dtype == DR_F32) return decode_dispatch<float>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
   return decode_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
+}
+
+// ----------------------------------------------------------------- prefill without allocation
+// Scratch of dr_chunk_fwd_noalloc: a file-scope device array (every GPU that
+// loads this library holds it until the process exits).  Host code must not
+// pass the symbol itself to a kernel -- on the host it is only a stand-in --
+// so its device address is looked up once per device with
+// cudaGetSymbolAddress while that device is current, and cached.
+constexpr size_t kStaticScratchBytes = 4096;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void *g_static_addr[kMaxDevices] = {};
+}  // namespace
+
+dr_status dr_chunk_fwd_noalloc(const dr_problem *p, const void *q, const void *k, const void *v,
+                               const float *alpha, const float *beta_k, const float *beta_v, const float *S0,
+                               void *o, float *S_T, void *stream) {
+  const dr_status s = check_common(p, false);
+  if (s != DR_OK) return s;
+  if (dr_chunk_fwd_workspace(p) > kStaticScratchBytes) return DR_ERR_WORKSPACE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DR_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DR_ERR_UNSUPPORTED;
+  void *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_addr[dev]) {
+      void *addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_static_scratch) != cudaSuccess || !addr) return DR_ERR_CUDA;
+      g_static_addr[dev] = addr;
+    }
+    scratch = g_static_addr[dev];
+  }
+  // dr_chunk_fwd clears the status word at the start of the call, on `stream`.
+  return dr_chunk_fwd(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, scratch, kStaticScratchBytes, stream);
 }
 
 dr_status dr_workspace_status(const void *workspace, void *stream) {
