@@ -195,6 +195,28 @@ def run_reference(args, ws, rank):
     return 0
 
 
+def run_decode_only(args, dr, dev, st, ws):
+    """Profiling aid: the decode workload alone (warm-up, then the timed chained steps)."""
+    d = decode_inputs()
+    S_dec = d["S"].to(dev)
+    pool = {k: (None if d[k] is None else d[k].to(dev)) for k in ("q", "k", "v", "alpha", "beta_k")}
+    o_dec = torch.empty((DECODE.B, 1, DECODE.H, DECODE.dv), dtype=torch.bfloat16, device=dev)
+    n = args.warmup + args.decode_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(n):
+        if i == args.warmup:
+            e0.record(st)
+        j = i % DECODE.pool
+        dr.dr_decode_step(pool["q"][j], pool["k"][j], pool["v"][j], pool["beta_k"][j], S_dec,
+                          alpha=pool["alpha"][j], o=o_dec, stream=st)
+    e1.record(st)
+    torch.cuda.synchronize()
+    dms = e0.elapsed_time(e1) / args.decode_steps
+    dgbs = decode_bytes(DECODE.B, DECODE.H, DECODE.dk, DECODE.dv) / (dms / 1e3) / 1e9
+    print(json.dumps({"only_decode": True, "ms_per_step": dms, "GB/s": dgbs}), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- our arm
 def main():
     ap = argparse.ArgumentParser()
@@ -204,6 +226,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only-prefill", action="store_true",
+                    help="profiling aid: time only the prefill step (no decode workload, e2e or CPU leg)")
+    ap.add_argument("--only-decode", action="store_true",
+                    help="profiling aid: time only the decode workload")
     args = ap.parse_args()
     ws, rank, local = dist_env()
     if args.impl == "reference":
@@ -237,6 +263,8 @@ def main():
                         chunk=p.chunk, o=o, S_T=S, workspace=ws_buf, stream=st)
         dr.dr_decode_step(nxt["q"], nxt["k"], nxt["v"], nxt["beta_k"], S, alpha=nxt["alpha"], o=o1, stream=st)
 
+    if args.only_decode:
+        return run_decode_only(args, dr, dev, st, ws)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -279,6 +307,11 @@ def main():
                 "algorithmic_flops_per_launch": flops,
                 "tensor_tflops_achieved": flops / (prefill_ms / 1e3) / 1e12,
                 "roofline_time_ms": t_roof_ms, "frac_of_max_roofline": t_roof_ms / prefill_ms}
+
+    if args.only_prefill:
+        print(json.dumps({"only_prefill": True, "prefill_ms": prefill_ms, "ms_per_step": ms_step,
+                          "roofline": roofline}), flush=True)
+        return 0
 
     # ---------------- decode workload (B=256, H=32, 512 MiB state, chained in-place steps)
     d = decode_inputs()

@@ -1,6 +1,8 @@
 // deltarule_api.cu -- the C ABI declared in include/deltarule.h: argument
 // checks, workspace status word, and dispatch to the sm_100a kernels.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
 #include <cstring>
@@ -98,19 +100,60 @@ dr_status simt_dispatch(const dr_problem *p, const void *q, const void *k, const
 }
 
 // ----------------------------------------------------------------- prefill, tensor-core path (bf16 I/O)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 4-D map over a [B, T, H, D] row-major tensor (dims innermost first: D, H, T, B) with a box of
+// `box_d` elements x 1 head x `box_t` tokens x 1 batch row; out-of-range rows read as zero.
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, size_t esize, const void *base, int B, int T, int H, int D,
+              int box_d, int box_t) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
+  const cuuint64_t strides[3] = {cuuint64_t(D) * esize, cuuint64_t(D) * H * esize, cuuint64_t(D) * H * T * esize};
+  const cuuint32_t box[4] = {cuuint32_t(box_d), 1u, cuuint32_t(box_t), 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return enc(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 dr_status tc_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
                     const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
                     uint32_t *status, cudaStream_t st) {
   using IO = __nv_bfloat16;
-  auto kern = dr::tc::chunk_fwd_tc_kernel<IO>;
-  constexpr size_t smem = dr::tc::SMEM_BYTES;
+  namespace tc = dr::tc;
+  alignas(64) CUtensorMap mq, mk, mv, mbv;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_map(&mq, bf, 2, q, p->B, p->T, p->H, p->dk, tc::DK, tc::C) ||
+      !make_map(&mk, bf, 2, k, p->B, p->T, p->H, p->dk, tc::DK, tc::C) ||
+      !make_map(&mv, bf, 2, v, p->B, p->T, p->H, p->dv, tc::VS, tc::C))
+    return DR_ERR_CUDA;
+  if (p->beta_v_mode == DR_CHANNEL) {
+    if (!make_map(&mbv, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, beta_v, p->B, p->T, p->H, p->dv, tc::VS, tc::C))
+      return DR_ERR_CUDA;
+  } else {
+    mbv = mv;  // unused by the kernel in this mode
+  }
+  tc::Params prm{p->T, p->H, p->dv, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v, p->beta_v_mode,
+                 S0, o, S_T, status};
+  auto kern = tc::chunk_fwd_tc_kernel<IO>;
+  constexpr size_t smem = tc::SMEM_BYTES;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
     return DR_ERR_CUDA;
-  dim3 grid(p->dv / dr::tc::VS, p->H, p->B);
-  kern<<<grid, dr::tc::NT, smem, st>>>(p->T, p->H, p->dv, static_cast<const IO *>(q), static_cast<const IO *>(k),
-                                       static_cast<const IO *>(v), alpha, p->alpha_mode, beta_k, p->beta_k_mode,
-                                       beta_v, p->beta_v_mode, S0, static_cast<IO *>(o), S_T, status);
+  dim3 grid(p->dv / tc::VS, p->H, p->B);
+  kern<<<grid, tc::NT, smem, st>>>(mq, mk, mv, mbv, prm);
   return launch_status();
 }
 
