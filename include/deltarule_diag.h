@@ -34,6 +34,16 @@ extern "C" {
 DR_API int dr_diag_umma_selftest(int N, int K, int a_mn, int b_mn, int bf16, const void *A, const void *B,
                                  float *D, void *workspace, void *stream);
 
+/*
+ * T = (I + A)^-1 for the strictly lower-triangular part of a 64 x 64 matrix A
+ * (the UT transform of one chunk), computed by the warp-MMA routine of the
+ * prefill kernel (fp16 operands, fp32 accumulation).  A: row-major fp32 device
+ * buffer (its diagonal and upper part are ignored); T: row-major fp32 device
+ * buffer that the caller zeroes first (only the lower blocks are written).
+ * Returns a dr_status code.
+ */
+DR_API int dr_diag_tri_inverse(const float *A, float *T, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

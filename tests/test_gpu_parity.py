@@ -97,6 +97,34 @@ def test_umma_building_blocks(dr, N, K, a_mn, b_mn, dtype):
     np.testing.assert_allclose(D.cpu().double().numpy(), ref.numpy(), rtol=1e-4, atol=1e-3)
 
 
+def _unit_lower_case(seed, scale):
+    g = torch.Generator().manual_seed(seed)
+    return torch.tril(scale * torch.randn(64, 64, generator=g, dtype=torch.float64), -1)
+
+
+@pytest.mark.parametrize("seed,scale", [(0, 0.05), (1, 0.15), (2, 0.3)])
+def test_tri_inverse_building_block(dr, seed, scale):
+    """The warp-MMA UT-transform inverse against a float64 matrix inverse."""
+    A = _unit_lower_case(seed, scale)
+    ref = torch.linalg.inv(torch.eye(64, dtype=torch.float64) + A)
+    T = dr.dr_diag_tri_inverse(A.float().cuda()).double().cpu()
+    assert torch.equal(torch.triu(T, 1), torch.zeros_like(T))          # lower triangular
+    assert torch.allclose(torch.diagonal(T), torch.ones(64, dtype=torch.float64), atol=1e-6)
+    assert float((T - ref).abs().max() / ref.abs().max()) <= 5e-3
+
+
+def test_tri_inverse_on_key_gram_matrix(dr):
+    """A shaped like a real chunk: A_ij = sqrt(b_i b_j) k_i . k_j (unit keys, strengths in (0,1))."""
+    g = torch.Generator().manual_seed(7)
+    k = torch.nn.functional.normalize(torch.randn(64, 128, generator=g, dtype=torch.float64), dim=-1)
+    beta = torch.sigmoid(torch.randn(64, generator=g, dtype=torch.float64))
+    kb = k * beta.sqrt()[:, None]
+    A = torch.tril(kb @ kb.T, -1)
+    ref = torch.linalg.inv(torch.eye(64, dtype=torch.float64) + A)
+    T = dr.dr_diag_tri_inverse(A.float().cuda()).double().cpu()
+    assert float((T - ref).abs().max() / ref.abs().max()) <= 5e-3
+
+
 # ------------------------------------------------------------------------- prefill, small shapes
 SMALL = [
     # (dk, dv, T, chunk, io, alpha, beta_k, beta_v, S0)

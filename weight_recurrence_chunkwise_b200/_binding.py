@@ -39,7 +39,8 @@ class DeltaRuleError(RuntimeError):
 _lib = None
 
 EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_chunk_fwd_noalloc", "dr_decode_step",
-           "dr_workspace_status", "dr_status_string", "dr_version", "dr_diag_umma_selftest")
+           "dr_workspace_status", "dr_status_string", "dr_version", "dr_diag_umma_selftest",
+           "dr_diag_tri_inverse")
 
 
 def lib():
@@ -66,6 +67,8 @@ def lib():
         L.dr_version.restype = ctypes.c_int
         L.dr_diag_umma_selftest.argtypes = [ctypes.c_int] * 5 + [vp, vp, vp, vp, vp]
         L.dr_diag_umma_selftest.restype = ctypes.c_int
+        L.dr_diag_tri_inverse.argtypes = [vp, vp, vp]
+        L.dr_diag_tri_inverse.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -191,3 +194,15 @@ def dr_diag_umma_selftest(A, B, a_mn: bool, b_mn: bool, stream=None):
     if rc != DR_OK:
         raise DeltaRuleError(rc, "dr_diag_umma_selftest")
     return D, dr_workspace_status(ws, stream)
+
+
+def dr_diag_tri_inverse(A, stream=None):
+    """(I + strictly-lower(A))^-1 for a 64 x 64 fp32 CUDA tensor, via the prefill's warp-MMA routine."""
+    if A.shape != (64, 64) or A.dtype != torch.float32 or not A.is_cuda:
+        raise ValueError("A must be a 64 x 64 fp32 CUDA tensor")
+    A = A.contiguous()
+    T = torch.zeros_like(A)
+    rc = lib().dr_diag_tri_inverse(_ptr(A), _ptr(T), _stream(stream))
+    if rc != DR_OK:
+        raise DeltaRuleError(rc, "dr_diag_tri_inverse")
+    return T

@@ -8,9 +8,10 @@
 //
 //  K1  gamma_r = prod_{j<=r} alpha_j per key channel (= exp(g_r)); gamma_C = gamma_{C-1}.
 //  a0  b = sqrt(beta_k) k,  w = beta_v v  or  sqrt(beta_k) v.
-//      Operand tiles:  Qh = gamma q,  Bh = gamma b,  Ac = b / gamma   (= b exp(-g)).
+//      Operand tiles:  Qh = gamma q,  Bh = gamma b,  Ac = b R / gamma_C  (= b exp(-g)),
+//      R_r = prod_{j>r} alpha_j (reverse products: no division per element).
 //  K2  D1 = [Qh; Bh] Ac^T                      (P raw | A raw)           MMA 128x64x128
-//      P = lower(Qh Ac^T),  T = (I + strictly-lower(Bh Ac^T))^-1         (fp32, CUDA cores)
+//      P = lower(Qh Ac^T),  T = (I + strictly-lower(Bh Ac^T))^-1         (warp MMAs, tri_inverse.cuh)
 //      D2 = [T; P] Bh  -> W = T Bh (rows 0..63)                          MMA 128x128x64
 //      D1 = [T; P] Wr  -> U0 = T Wr (rows 0..63)                         MMA 128x64x64
 //  K3  D3 = [-W; Qh] S -> -W S (rows 0..63), Qh S (rows 64..127)         MMA 128x64x128
@@ -31,6 +32,7 @@
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tri_inverse.cuh"
 
 namespace dr {
 namespace tc {
@@ -39,7 +41,7 @@ constexpr int C = 64;     // chunk length
 constexpr int DK = 128;   // key dim
 constexpr int VS = 64;    // value columns per CTA
 constexpr int NT = 512;   // threads
-constexpr int RG = 16;    // rows of a chunk handled by one elementwise thread
+constexpr int RG = 8;     // rows of a chunk handled by one elementwise thread (two columns each)
 
 // shared-memory map (bytes from a 1024-aligned base); fp16 operand tiles use the 128B swizzle
 constexpr uint32_t OFF_QKB = 0;                          // [-W; Qh; Bh] 192 x 128 fp16
@@ -52,12 +54,12 @@ constexpr uint32_t OFF_RQ = OFF_U + 64 * 128;            // raw q, bf16 64 x 128
 constexpr uint32_t OFF_RK = OFF_RQ + 64 * 256;           // raw k
 constexpr uint32_t OFF_RV = OFF_RK + 64 * 256;           // raw v slice, bf16 64 x VS
 constexpr uint32_t OFF_RW = OFF_RV + 64 * VS * 2;        // write scale, fp32 64 x VS (TMA'd beta_v or sqrt(beta_k))
-constexpr uint32_t OFF_AF = OFF_RW + 64 * VS * 4;        // A, fp32 64 x 65
-constexpr uint32_t OFF_TF = OFF_AF + 64 * 65 * 4;        // T, fp32 64 x 65
-constexpr uint32_t OFF_XF = OFF_TF + 64 * 65 * 4;        // block products, fp32 3 x 16 x 17
-constexpr uint32_t OFF_GC = OFF_XF + 3 * 16 * 17 * 4;    // gamma_C, 128 fp32
-constexpr uint32_t OFF_PX = OFF_GC + 128 * 4;            // per-row-group gate products, 4 x 128 fp32
-constexpr uint32_t OFF_END = OFF_PX + 4 * 128 * 4;
+constexpr uint32_t OFF_AH = OFF_RW + 64 * VS * 4;        // A, fp16 64 x LD (inverse input)
+constexpr uint32_t OFF_AHT = OFF_AH + 64 * tri::LD * 2;  // A^T
+constexpr uint32_t OFF_THT = OFF_AHT + 64 * tri::LD * 2; // T^T (inverse scratch)
+constexpr uint32_t OFF_GC = OFF_THT + 64 * tri::LD * 2;  // gamma_C, 128 fp32
+constexpr uint32_t OFF_PX = OFF_GC + 128 * 4;            // per-row-group gate products, 8 x 128 fp32
+constexpr uint32_t OFF_END = OFF_PX + 8 * 128 * 4;
 constexpr size_t SMEM_BYTES = OFF_END + 1024;            // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
@@ -109,6 +111,17 @@ __device__ __forceinline__ float bf16_at(const uint8_t *base, int idx) {
   return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[idx]);
 }
 
+// Gate values of two adjacent key channels (c, c+1) of one token: scalar, channel or absent (= 1).
+__device__ __forceinline__ float2 gate_pair(const float *g, int mode, size_t th, int c) {
+  if (mode == MODE_ABSENT) return make_float2(1.f, 1.f);
+  if (mode == MODE_SCALAR) {
+    const float x = __ldg(g + th);
+    return make_float2(x, x);
+  }
+  return __ldg(reinterpret_cast<const float2 *>(g + th * DK + c));
+}
+__device__ __forceinline__ float sqrt_fast(float x) { return x > 0.f ? x * rsqrtf(x) : 0.f; }
+
 template <typename IO>
 __global__ void __launch_bounds__(NT, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -128,9 +141,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const uint8_t *rK = sm + OFF_RK;
   const uint8_t *rV = sm + OFF_RV;
   float *rW = reinterpret_cast<float *>(sm + OFF_RW);
-  float *sA = reinterpret_cast<float *>(sm + OFF_AF);
-  float *sT = reinterpret_cast<float *>(sm + OFF_TF);
-  float *sX = reinterpret_cast<float *>(sm + OFF_XF);
+  __half *sAh = reinterpret_cast<__half *>(sm + OFF_AH);
+  __half *sAhT = reinterpret_cast<__half *>(sm + OFF_AHT);
+  __half *sThT = reinterpret_cast<__half *>(sm + OFF_THT);
   float *sGC = reinterpret_cast<float *>(sm + OFF_GC);
   float *sPX = reinterpret_cast<float *>(sm + OFF_PX);
 
@@ -157,6 +170,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tma_prefetch_desc(&tm_v);
     if (bv_tma) tma_prefetch_desc(&tm_bv);
   }
+  // rows 0..63 of [T; P] hold the lower-triangular T; its upper blocks stay zero
+  reinterpret_cast<uint4 *>(tTP)[tid] = make_uint4(0u, 0u, 0u, 0u);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -171,42 +186,58 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tma_load_4d(sm + OFF_RV, &tm_v, &raw_bar, v0, h, t0, b);
     if (bv_tma) tma_load_4d(sm + OFF_RW, &tm_bv, &raw_bar, v0, h, t0, b);
   };
-  // Waits are bounded; the decision to stop is made uniformly by the whole CTA.
-  auto wait_bar = [&](uint64_t *bar, uint32_t &ph) -> bool {
-    const bool ok = mbar_wait(bar, ph & 1u, kWaitLimitNs);
-    ph++;
+  // Waits are bounded and the decision to stop is taken by the whole CTA at once.
+  // TMA data: every thread waits on the barrier (each then sees the bytes).
+  auto wait_raw = [&]() -> bool {
+    const bool ok = mbar_wait(&raw_bar, rphase & 1u, kWaitLimitNs);
+    rphase++;
     if (!ok && lane == 0) raise_status(p.status, STATUS_TIMEOUT);
     return __syncthreads_or(!ok) == 0;
   };
+  // MMA completion: one thread waits, the CTA barrier releases the others.
   auto wait_mma = [&]() -> bool {
-    const bool ok = wait_bar(&mma_bar, mphase);
+    bool ok = true;
+    if (tid == 0) ok = mbar_wait(&mma_bar, mphase & 1u, kWaitLimitNs);
+    mphase++;
+    const bool fail = __syncthreads_or(!ok) != 0;
     tc_fence_after();
-    return ok;
+    if (fail && tid == 0) raise_status(p.status, STATUS_TIMEOUT);
+    return !fail;
   };
 
-  // gate prefetch: thread (kc, rg) holds alpha and beta_k of its 16 rows of the next chunk;
-  // threads of the write-vector layout hold the scalar write scale of their row.
-  const int kc = tid & 127, rg = tid >> 7;
-  const int wc = tid >> 3, wj0 = (tid & 7) * 8;  // write-vector element block: row wc, columns wj0..wj0+7
-  float pal[RG], pbe[RG], pws = 0.f;
+  // Elementwise layout: thread (kp, rgp) owns key channels 2kp, 2kp+1 and rows 8rgp .. 8rgp+7.
+  const int kp = tid & 63, rgp = tid >> 6, c0 = 2 * kp;
+  const int wc = tid >> 3, wj0 = (tid & 7) * 8;  // write-vector block: row wc, columns wj0..wj0+7
+  float pal[2 * RG], pbe[2 * RG], pws = 0.f;     // prefetched gates of the next chunk
+#pragma unroll
+  for (int i = 0; i < 2 * RG; ++i) pal[i] = pbe[i] = 1.f;
+  // Loads only, issued one chunk ahead: every value lands directly in its register and is
+  // masked or broadcast only when it is consumed, so nothing here waits for memory.
+  // Rows past the end of the sequence load the last valid row (masked at use).
   auto prefetch_gates = [&](int t0) {
     const int L = min(C, T - t0);
+    const size_t thb = (static_cast<size_t>(b) * T + t0) * H + h;
 #pragma unroll
     for (int j = 0; j < RG; ++j) {
-      const int r = rg * RG + j;
-      pal[j] = 1.f;
-      pbe[j] = 0.f;
-      if (r < L) {
-        const size_t th = (static_cast<size_t>(b) * T + t0 + r) * H + h;
-        pal[j] = gate_at(p.alpha, p.alpha_mode, th, DK, kc);
-        pbe[j] = gate_at(p.beta_k, p.beta_k_mode, th, DK, kc);
+      const size_t th = thb + static_cast<size_t>(min(rgp * RG + j, L - 1)) * H;
+      if (p.alpha_mode == MODE_CHANNEL) {
+        const float2 a = __ldg(reinterpret_cast<const float2 *>(p.alpha + th * DK + c0));
+        pal[2 * j] = a.x;
+        pal[2 * j + 1] = a.y;
+      } else if (p.alpha_mode == MODE_SCALAR) {
+        pal[2 * j] = __ldg(p.alpha + th);
+      }
+      if (p.beta_k_mode == MODE_CHANNEL) {
+        const float2 bt = __ldg(reinterpret_cast<const float2 *>(p.beta_k + th * DK + c0));
+        pbe[2 * j] = bt.x;
+        pbe[2 * j + 1] = bt.y;
+      } else {
+        pbe[2 * j] = __ldg(p.beta_k + th);
       }
     }
-    pws = 0.f;
-    if (wc < L && !bv_tma && !sym_channel) {
-      const size_t th = (static_cast<size_t>(b) * T + t0 + wc) * H + h;
-      pws = (p.beta_v_mode == MODE_SCALAR) ? __ldg(p.beta_v + th) : sqrtf(__ldg(p.beta_k + th));
-    }
+    if (!bv_tma && !sym_channel)  // raw scalar strength of row wc (beta_v, or beta_k for the symmetric write)
+      pws = __ldg((p.beta_v_mode == MODE_SCALAR ? p.beta_v : p.beta_k) + thb +
+                  static_cast<size_t>(min(wc, L - 1)) * H);
   };
 
   // fp32 state slice in registers: row k = trow, columns cq*16 .. cq*16+15 of the slice
@@ -228,85 +259,152 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     prefetch_gates(0);
   }
 
+  // shared-memory descriptors of the operand tiles (K steps are added per MMA)
   const uint32_t a_base = smem_u32(sm);
+  const uint64_t dQB = sdesc_sw128(a_base + OFF_QKB + 64 * 128, 16, 1024);   // [Qh; Bh], K-major, R = 192
+  const uint64_t dWQ = sdesc_sw128(a_base + OFF_QKB, 16, 1024);              // [-W; Qh], K-major, R = 192
+  const uint64_t dBh = sdesc_sw128(a_base + OFF_QKB + 128 * 128, 192 * 128, 1024);  // Bh as MN-major B
+  const uint64_t dAcK = sdesc_sw128(a_base + OFF_AC, 16, 1024);              // Ac, K-major B (N = 64)
+  const uint64_t dAcM = sdesc_sw128(a_base + OFF_AC, 64 * 128, 1024);        // Ac^T as MN-major A (M = 128)
+  const uint64_t dTP = sdesc_sw128(a_base + OFF_TP, 16, 1024);               // [T; P], K-major (K = 64)
+  const uint64_t dWr = sdesc_sw128(a_base + OFF_WR, 64 * 128, 1024);         // Wr, MN-major B
+  const uint64_t dS = sdesc_sw128(a_base + OFF_S, 128 * 128, 1024);          // S, MN-major B
+  const uint64_t dU = sdesc_sw128(a_base + OFF_U, 64 * 128, 1024);           // U, MN-major B
+  // K step kk of a K-major tile with R rows: +32 B inside a 64-column block, +R*128 B per block
+  auto kstep = [](uint64_t d, int R, int kk) -> uint64_t {
+    return d + static_cast<uint64_t>(((kk >> 2) * R * 128 + (kk & 3) * 32) >> 4);
+  };
+  // K step kk of an MN-major tile: 16 rows of 128 B
+  auto mstep = [](uint64_t d, int kk) -> uint64_t { return d + static_cast<uint64_t>(kk * 128); };
+
   for (int t0 = 0; t0 < T; t0 += C) {
     const int L = min(C, T - t0);
-    if (!wait_bar(&raw_bar, rphase)) { aborted = true; break; }
+    if (!wait_raw()) { aborted = true; break; }
 
     // ------------------------------------------------------------ K1 + a0 (operand tiles)
     {
-      float pre[RG];
-      float pr = 1.f;
+      // gates of this chunk: mask rows past the end (alpha = 1, beta = 0), broadcast scalars
 #pragma unroll
       for (int j = 0; j < RG; ++j) {
-        pr *= pal[j];
-        pre[j] = pr;
+        const bool valid = rgp * RG + j < L;
+        if (p.alpha_mode != MODE_CHANNEL) pal[2 * j + 1] = pal[2 * j];
+        if (p.alpha_mode == MODE_ABSENT || !valid) pal[2 * j] = pal[2 * j + 1] = 1.f;
+        if (p.beta_k_mode != MODE_CHANNEL) pbe[2 * j + 1] = pbe[2 * j];
+        if (!valid) pbe[2 * j] = pbe[2 * j + 1] = 0.f;
       }
-      sPX[rg * 128 + kc] = pr;
-      __syncthreads();
-      float head = 1.f, gC = 1.f;
+      float pre[2 * RG];
+      float p0 = 1.f, p1 = 1.f;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const float x = sPX[g * 128 + kc];
-        if (g < rg) head *= x;
-        gC *= x;
+      for (int j = 0; j < RG; ++j) {
+        p0 *= pal[2 * j];
+        p1 *= pal[2 * j + 1];
+        pre[2 * j] = p0;
+        pre[2 * j + 1] = p1;
       }
-      if (rg == 0) {
-        sGC[kc] = gC;
-        if (!(gC >= kMinChunkDecayF16)) raise_status(p.status, STATUS_RANGE);
+      *reinterpret_cast<float2 *>(sPX + rgp * 128 + c0) = make_float2(p0, p1);
+      __syncthreads();
+      // head: product of the row groups before mine; tail: after mine; gamma_C: all
+      float h0 = 1.f, h1 = 1.f, t0a = 1.f, t1a = 1.f;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const float2 x = *reinterpret_cast<const float2 *>(sPX + g * 128 + c0);
+        if (g < rgp) {
+          h0 *= x.x;
+          h1 *= x.y;
+        } else if (g > rgp) {
+          t0a *= x.x;
+          t1a *= x.y;
+        }
       }
-      const bool own_w = sym_channel && kc >= v0 && kc < v0 + VS;
+      const float g0 = h0 * p0 * t0a, g1 = h1 * p1 * t1a;
+      if (rgp == 0) {
+        *reinterpret_cast<float2 *>(sGC + c0) = make_float2(g0, g1);
+        if (!(fminf(g0, g1) >= kMinChunkDecayF16)) raise_status(p.status, STATUS_RANGE);
+      }
+      const bool own_w = sym_channel && c0 >= v0 && c0 < v0 + VS;
+      // swizzled byte offsets of (row, c0) inside the K-major tiles: row & 7 == j for row = 8 rgp + j (+64, +128)
+      const uint32_t blk = static_cast<uint32_t>(kp >> 5), ch = static_cast<uint32_t>((kp & 31) >> 2);
+      const uint32_t inb = static_cast<uint32_t>((kp & 3) * 4);
+      uint8_t *pQ = tQKB + blk * 192 * 128 + (64 + rgp * RG) * 128 + inb;
+      uint8_t *pB = tQKB + blk * 192 * 128 + (128 + rgp * RG) * 128 + inb;
+      uint8_t *pA = tAC + blk * 64 * 128 + (rgp * RG) * 128 + inb;
+      // exp(-g_r) = R_r / gamma_C with R_r = product of the gates after row r (no division per element)
+      const float ig0 = __fdividef(1.f, g0), ig1 = __fdividef(1.f, g1);
+      float suf0 = t0a * ig0, suf1 = t1a * ig1;  // R_r / gamma_C for the last row of my group
+      const bool beta_scalar = p.beta_k_mode == MODE_SCALAR;
       float amax = 0.f;
 #pragma unroll
-      for (int j = 0; j < RG; ++j) {
-        const int r = rg * RG + j;
-        const float sb = sqrtf(pbe[j]);
-        const float bk = sb * bf16_at(rK, r * DK + kc);  // rows >= L: k = 0 (TMA fill), beta = 0
-        const float qv = bf16_at(rQ, r * DK + kc);
-        const float g = head * pre[j];
-        const float ac = bk * __frcp_rn(g);
-        amax = fmaxf(amax, fabsf(ac));
-        st_h16(tQKB, 64 + r, kc, 192, g * qv);   // Qh
-        st_h16(tQKB, 128 + r, kc, 192, g * bk);  // Bh
-        st_h16(tAC, r, kc, 64, ac);              // Ac = b exp(-g)
-        if (own_w) rW[r * VS + (kc - v0)] = sb;  // write scale sqrt(beta_k) of this value column
+      for (int j = RG - 1; j >= 0; --j) {
+        const int r = rgp * RG + j;
+        const uint32_t sw = ((ch ^ static_cast<uint32_t>(j)) << 4) + j * 128;
+        const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(rK + (r * DK + c0) * 2);
+        const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(rQ + (r * DK + c0) * 2);
+        const float2 kf = __bfloat1622float2(k2), qf = __bfloat1622float2(q2);
+        float s0, s1;
+        if (beta_scalar) {  // one square root per row
+          s0 = s1 = sqrt_fast(pbe[2 * j]);
+        } else {
+          s0 = sqrt_fast(pbe[2 * j]);
+          s1 = sqrt_fast(pbe[2 * j + 1]);
+        }
+        const float b0 = s0 * kf.x, b1 = s1 * kf.y;  // rows >= L: k = 0 (TMA fill), beta = 0
+        const float ga = h0 * pre[2 * j], gb = h1 * pre[2 * j + 1];
+        const float a0 = b0 * suf0, a1 = b1 * suf1;
+        suf0 *= pal[2 * j];
+        suf1 *= pal[2 * j + 1];
+        amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
+        *reinterpret_cast<uint32_t *>(pQ + sw) = pack_f16x2(ga * qf.x, gb * qf.y);  // Qh
+        *reinterpret_cast<uint32_t *>(pB + sw) = pack_f16x2(ga * b0, gb * b1);      // Bh
+        *reinterpret_cast<uint32_t *>(pA + sw) = pack_f16x2(a0, a1);                // Ac = b exp(-g)
+        if (own_w) *reinterpret_cast<float2 *>(rW + r * VS + (c0 - v0)) = make_float2(s0, s1);
       }
       if (!(amax < kF16Max)) raise_status(p.status, STATUS_RANGE);
       if (sym_channel) __syncthreads();
       // write vectors w (rows c, value columns of this slice)
       {
-        float w8[8];
-        const bool valid = wc < L;
+        const uint4 vraw = *reinterpret_cast<const uint4 *>(rV + (wc * VS + wj0) * 2);
+        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vraw);
+        float sc[8];
+        if (bv_tma || sym_channel) {
+          const float4 s_lo = *reinterpret_cast<const float4 *>(rW + wc * VS + wj0);
+          const float4 s_hi = *reinterpret_cast<const float4 *>(rW + wc * VS + wj0 + 4);
+          sc[0] = s_lo.x; sc[1] = s_lo.y; sc[2] = s_lo.z; sc[3] = s_lo.w;
+          sc[4] = s_hi.x; sc[5] = s_hi.y; sc[6] = s_hi.z; sc[7] = s_hi.w;
+        } else {
+          const float sc0 = (p.beta_v_mode == MODE_SCALAR) ? pws : sqrt_fast(pws);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float vv = bf16_at(rV, wc * VS + wj0 + i);
-          const float sc = (bv_tma || sym_channel) ? rW[wc * VS + wj0 + i] : pws;
-          w8[i] = valid ? sc * vv : 0.f;
+          for (int i = 0; i < 8; ++i) sc[i] = sc0;
+        }
+        const bool valid = wc < L;
+        float w8[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 vf = __bfloat1622float2(v2[i]);
+          w8[2 * i] = valid ? sc[2 * i] * vf.x : 0.f;
+          w8[2 * i + 1] = valid ? sc[2 * i + 1] * vf.y : 0.f;
         }
         st_h16x8(tWR, wc, wj0, 64, w8);
       }
     }
     fence_async_smem();
     __syncthreads();
-    // the raw staging area and the gate registers are free: fetch chunk c+1 now
-    if (t0 + C < T) {
-      if (tid == 0) issue_raw(t0 + C);
-      prefetch_gates(t0 + C);
-    }
-
     // ------------------------------------------------------------ m1: D1 = [Qh; Bh] Ac^T
     if (tid == 0) {
       tc_fence_after();
       const uint32_t idesc = idesc_f16_f32(128, 64, false, false);
 #pragma unroll
       for (int kk = 0; kk < DK / 16; ++kk)
-        umma_f16(tmem + COL_D1, desc_kmajor(a_base + OFF_QKB + 64 * 128, 192, kk),
-                 desc_kmajor(a_base + OFF_AC, 64, kk), idesc, kk > 0);
+        umma_f16(tmem + COL_D1, kstep(dQB, 192, kk), kstep(dAcK, 64, kk), idesc, kk > 0);
       umma_commit(&mma_bar);
+    }
+    // the raw staging area and the gate registers are free: fetch chunk c+1 while m1 runs
+    if (t0 + C < T) {
+      if (tid == 0) issue_raw(t0 + C);
+      prefetch_gates(t0 + C);
     }
     if (!wait_mma()) { aborted = true; break; }
 
-    // ------------------------------------------------------------ E1: P (fp16 tile), A (fp32)
+    // ------------------------------------------------------------ E1: P (fp16 tile), A and A^T (fp16)
     {
       float x[16];
       tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D1 + cq * 16), x);
@@ -319,60 +417,27 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       } else {  // rows 64..127: Bh Ac^T -> strictly lower A
         const int r = trow - 64;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 16; i += 2) {
           const int col = cq * 16 + i;
-          sA[r * 65 + col] = (col < r) ? x[i] : 0.f;
+          const float x0 = (col < r) ? x[i] : 0.f, x1 = (col + 1 < r) ? x[i + 1] : 0.f;
+          *reinterpret_cast<uint32_t *>(sAh + r * tri::LD + col) = pack_f16x2(x0, x1);
+          sAhT[col * tri::LD + r] = __float2half_rn(x0);
+          sAhT[(col + 1) * tri::LD + r] = __float2half_rn(x1);
         }
       }
     }
     tc_fence_before();
     __syncthreads();
 
-    // ------------------------------------------------------------ K2: T = (I + A)^-1, blocked 4 x 16
-    if (tid < 64) {  // diagonal blocks: one column of one block per thread
-      const int bb = tid >> 4, col = tid & 15, o16 = bb * 16;
-      float xcol[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        float acc = (r == col) ? 1.f : 0.f;
-        if (r > col) {
-#pragma unroll
-          for (int m = 0; m < 16; ++m)
-            if (m >= col && m < r) acc -= sA[(o16 + r) * 65 + o16 + m] * xcol[m];
-        }
-        xcol[r] = (r < col) ? 0.f : acc;
-      }
-#pragma unroll
-      for (int r = 0; r < 16; ++r) sT[(o16 + r) * 65 + o16 + col] = xcol[r];
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int d = 1; d < 4; ++d) {
-      const int nblk = 4 - d;
-      // X_ij = sum_{m in [j16, i16)} A[i16 + rr][m] T[m][j16 + cc],  i = j + d
-      for (int e = tid; e < nblk * 256; e += NT) {
-        const int jb = e >> 8, rr = (e >> 4) & 15, cc = e & 15, ib = jb + d;
-        float acc = 0.f;
-        for (int m = jb * 16; m < ib * 16; ++m) acc += sA[(ib * 16 + rr) * 65 + m] * sT[m * 65 + jb * 16 + cc];
-        sX[(jb * 16 + rr) * 17 + cc] = acc;
-      }
-      __syncthreads();
-      // T_ij = - T_ii X_ij
-      for (int e = tid; e < nblk * 256; e += NT) {
-        const int jb = e >> 8, rr = (e >> 4) & 15, cc = e & 15, ib = jb + d;
-        float acc = 0.f;
-        for (int m = 0; m <= rr; ++m) acc += sT[(ib * 16 + rr) * 65 + ib * 16 + m] * sX[(jb * 16 + m) * 17 + cc];
-        sT[(ib * 16 + rr) * 65 + jb * 16 + cc] = -acc;
-      }
-      __syncthreads();
-    }
-    {  // T (lower, fp16) into rows 0..63 of [T; P]
-      const int r = tid >> 3, c0 = (tid & 7) * 8;
-      float t8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) t8[i] = (c0 + i <= r) ? sT[r * 65 + c0 + i] : 0.f;
-      st_h16x8(tTP, r, c0, 128, t8);
-    }
+    // ------------------------------------------------------------ K2: T = (I + A)^-1 (warp MMAs)
+    tri::inverse64(sAh, sAhT, sThT, warp, lane, [&](int bi, int bj, const tri::Frag &F, int ln) {
+      const int r = ln >> 2, qq = ln & 3;
+      const int row = 16 * bi + r, col = 16 * bj + 2 * qq;
+      *reinterpret_cast<uint32_t *>(tTP + sw128_off(row, col, 128)) = pack_f16x2(F.v[0], F.v[1]);
+      *reinterpret_cast<uint32_t *>(tTP + sw128_off(row + 8, col, 128)) = pack_f16x2(F.v[2], F.v[3]);
+      *reinterpret_cast<uint32_t *>(tTP + sw128_off(row, col + 8, 128)) = pack_f16x2(F.v[4], F.v[5]);
+      *reinterpret_cast<uint32_t *>(tTP + sw128_off(row + 8, col + 8, 128)) = pack_f16x2(F.v[6], F.v[7]);
+    });
     fence_async_smem();
     __syncthreads();
 
@@ -382,13 +447,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const uint32_t id2 = idesc_f16_f32(128, 128, false, true);
       const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
 #pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk)
-        umma_f16(tmem + COL_D2, desc_kmajor(a_base + OFF_TP, 128, kk),
-                 desc_mnmajor(a_base + OFF_QKB + 128 * 128, 192, kk), id2, kk > 0);
+      for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_D2, kstep(dTP, 128, kk), mstep(dBh, kk), id2, kk > 0);
 #pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk)
-        umma_f16(tmem + COL_D1, desc_kmajor(a_base + OFF_TP, 128, kk), desc_mnmajor(a_base + OFF_WR, 64, kk),
-                 id3, kk > 0);
+      for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_D1, kstep(dTP, 128, kk), mstep(dWr, kk), id3, kk > 0);
       umma_commit(&mma_bar);
     }
     if (!wait_mma()) { aborted = true; break; }
@@ -414,9 +475,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       tc_fence_after();
       const uint32_t id = idesc_f16_f32(128, VS, false, true);
 #pragma unroll
-      for (int kk = 0; kk < DK / 16; ++kk)
-        umma_f16(tmem + COL_D3, desc_kmajor(a_base + OFF_QKB, 192, kk), desc_mnmajor(a_base + OFF_S, 128, kk), id,
-                 kk > 0);
+      for (int kk = 0; kk < DK / 16; ++kk) umma_f16(tmem + COL_D3, kstep(dWQ, 192, kk), mstep(dS, kk), id, kk > 0);
       umma_commit(&mma_bar);
     }
     if (!wait_mma()) { aborted = true; break; }
@@ -446,13 +505,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const uint32_t id4 = idesc_f16_f32(128, VS, true, true);
       const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
 #pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk)
-        umma_f16(tmem + COL_D4, desc_mnmajor(a_base + OFF_AC, 64, kk), desc_mnmajor(a_base + OFF_U, 64, kk), id4,
-                 kk > 0);
+      for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_D4, mstep(dAcM, kk), mstep(dU, kk), id4, kk > 0);
 #pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk)
-        umma_f16(tmem + COL_D3, desc_kmajor(a_base + OFF_TP, 128, kk), desc_mnmajor(a_base + OFF_U, 64, kk), id3,
-                 1u);
+      for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_D3, kstep(dTP, 128, kk), mstep(dU, kk), id3, 1u);
       umma_commit(&mma_bar);
     }
     if (!wait_mma()) { aborted = true; break; }

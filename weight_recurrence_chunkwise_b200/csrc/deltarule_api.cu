@@ -316,4 +316,10 @@ int dr_diag_umma_selftest(int N, int K, int a_mn, int b_mn, int bf16, const void
   return DR_ERR_UNSUPPORTED;
 }
 
+int dr_diag_tri_inverse(const float *A, float *T, void *stream) {
+  if (!A || !T) return DR_ERR_INVALID_ARG;
+  dr::tri_selftest_kernel<<<1, 128, 0, static_cast<cudaStream_t>(stream)>>>(A, T);
+  return launch_status();
+}
+
 }  // extern "C"

@@ -1,0 +1,163 @@
+// tri_inverse.cuh -- T = (I + A)^-1 for a strictly lower-triangular 64 x 64 A
+// (the UT transform of the chunkwise WY form), on warp-level tensor-core MMAs.
+//
+// The 64 x 64 matrix is split into 4 x 4 blocks of 16 x 16.  Every block
+// product is two m16n8k16 MMAs (fp16 operands, fp32 accumulation), issued by
+// one warp on register fragments, which suits these tiny dependent products
+// far better than a round trip through tensor memory.
+//
+//  * Diagonal blocks (warps 0..3, one block each): for N = A_bb strictly lower
+//    (N^16 = 0),  (I + N)^-1 = (I - N)(I + N^2)(I + N^4)(I + N^8).
+//  * Off-diagonal blocks, by distance d = i - j = 1, 2, 3 (warp i computes
+//    block (i, j)):  T_ij = -T_ii * sum_{m=j}^{i-1} A_im T_mj.
+//
+// Fragment trick: a 16 x 16 matrix X is held as its accumulator fragment
+// F(X) (8 floats per lane).  F(X) repacks directly into the A operand of an
+// MMA; the B operand for "times Y" is the repacked F(Y^T).  Every matrix is
+// therefore carried together with its transpose, and every product X Y is
+// computed with its transpose Y^T X^T, so no lane shuffles are needed.
+#pragma once
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+namespace dr {
+namespace tri {
+
+constexpr int LD = 72;  // row stride (halves) of the padded 64 x 64 fp16 arrays: conflict-free fragment loads
+
+struct Frag {
+  float v[8];  // X[r][2q], X[r][2q+1], X[r+8][2q], X[r+8][2q+1], X[r][2q+8], X[r][2q+9], X[r+8][2q+8], X[r+8][2q+9]
+};
+
+__device__ __forceinline__ uint32_t h2u(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D += X * Y, where Zt = F(Y^T).
+__device__ __forceinline__ void mul_acc(Frag &D, const Frag &X, const Frag &Zt) {
+  const uint32_t a[4] = {h2u(X.v[0], X.v[1]), h2u(X.v[2], X.v[3]), h2u(X.v[4], X.v[5]), h2u(X.v[6], X.v[7])};
+  float dl[4] = {D.v[0], D.v[1], D.v[2], D.v[3]};
+  float dr[4] = {D.v[4], D.v[5], D.v[6], D.v[7]};
+  mma16816(dl, a, h2u(Zt.v[0], Zt.v[1]), h2u(Zt.v[4], Zt.v[5]));  // output columns 0..7
+  mma16816(dr, a, h2u(Zt.v[2], Zt.v[3]), h2u(Zt.v[6], Zt.v[7]));  // output columns 8..15
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    D.v[i] = dl[i];
+    D.v[4 + i] = dr[i];
+  }
+}
+__device__ __forceinline__ Frag mul(const Frag &X, const Frag &Zt) {
+  Frag D;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) D.v[i] = 0.f;
+  mul_acc(D, X, Zt);
+  return D;
+}
+// I + s X (s = +1 or -1)
+__device__ __forceinline__ Frag eye_plus(const Frag &X, float s, int lane) {
+  const int r = lane >> 2, q = lane & 3;
+  Frag D;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) D.v[i] = s * X.v[i];
+  D.v[0] += (r == 2 * q) ? 1.f : 0.f;
+  D.v[1] += (r == 2 * q + 1) ? 1.f : 0.f;
+  D.v[6] += (r == 2 * q) ? 1.f : 0.f;
+  D.v[7] += (r == 2 * q + 1) ? 1.f : 0.f;
+  return D;
+}
+__device__ __forceinline__ void negate(Frag &X) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) X.v[i] = -X.v[i];
+}
+
+// Block (bi, bj) of a row-major fp16 64 x 64 array with row stride LD.
+__device__ __forceinline__ Frag load_frag(const __half *M, int bi, int bj, int lane) {
+  const int r = lane >> 2, q = lane & 3;
+  const __half *base = M + (16 * bi + r) * LD + 16 * bj + 2 * q;
+  Frag F;
+  const float2 x0 = __half22float2(*reinterpret_cast<const __half2 *>(base));
+  const float2 x1 = __half22float2(*reinterpret_cast<const __half2 *>(base + 8 * LD));
+  const float2 x2 = __half22float2(*reinterpret_cast<const __half2 *>(base + 8));
+  const float2 x3 = __half22float2(*reinterpret_cast<const __half2 *>(base + 8 * LD + 8));
+  F.v[0] = x0.x;
+  F.v[1] = x0.y;
+  F.v[2] = x1.x;
+  F.v[3] = x1.y;
+  F.v[4] = x2.x;
+  F.v[5] = x2.y;
+  F.v[6] = x3.x;
+  F.v[7] = x3.y;
+  return F;
+}
+__device__ __forceinline__ void store_frag(__half *M, int bi, int bj, const Frag &F, int lane) {
+  const int r = lane >> 2, q = lane & 3;
+  __half *base = M + (16 * bi + r) * LD + 16 * bj + 2 * q;
+  *reinterpret_cast<uint32_t *>(base) = h2u(F.v[0], F.v[1]);
+  *reinterpret_cast<uint32_t *>(base + 8 * LD) = h2u(F.v[2], F.v[3]);
+  *reinterpret_cast<uint32_t *>(base + 8) = h2u(F.v[4], F.v[5]);
+  *reinterpret_cast<uint32_t *>(base + 8 * LD + 8) = h2u(F.v[6], F.v[7]);
+}
+
+// Called by every thread of the CTA (contains __syncthreads); warps 0..3 work.
+// Ah, AhT: A and A^T (fp16, row stride LD, zero on and above A's diagonal).
+// ThT: scratch for T^T (fp16, row stride LD).
+// put(bi, bj, F, lane): receives each lower block T_ij (i >= j) of the result.
+template <typename Put>
+__device__ __forceinline__ void inverse64(const __half *Ah, const __half *AhT, __half *ThT, int warp, int lane,
+                                          Put put) {
+  Frag Tii;  // diagonal block of this warp, kept for the off-diagonal levels
+  if (warp < 4) {
+    const int b = warp;
+    const Frag N = load_frag(Ah, b, b, lane);
+    const Frag Nt = load_frag(AhT, b, b, lane);
+    const Frag N2 = mul(N, Nt), N2t = mul(Nt, N);
+    const Frag N4 = mul(N2, N2t), N4t = mul(N2t, N2);
+    const Frag N8t = mul(N4t, N4);
+    const Frag X1 = eye_plus(N, -1.f, lane);
+    const Frag Y1t = eye_plus(N2t, 1.f, lane);
+    const Frag P1 = mul(X1, Y1t);
+    const Frag Y2t = eye_plus(N4t, 1.f, lane);
+    const Frag P2 = mul(P1, Y2t);
+    const Frag Y3t = eye_plus(N8t, 1.f, lane);
+    Tii = mul(P2, Y3t);
+    const Frag Tt = mul(Y3t, P2);
+    store_frag(ThT, b, b, Tt, lane);
+    put(b, b, Tii, lane);
+  }
+  __syncthreads();
+#pragma unroll 1
+  for (int d = 1; d < 4; ++d) {
+    if (warp >= d && warp < 4) {
+      const int i = warp, j = warp - d;
+      // Xt = X^T for X = sum_m A_im T_mj, accumulated as sum_m T_mj^T A_im^T
+      Frag Xt;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) Xt.v[e] = 0.f;
+      for (int m = j; m < i; ++m) {
+        const Frag Aim = load_frag(Ah, i, m, lane);
+        const Frag Tmjt = load_frag(ThT, j, m, lane);  // (T_mj)^T
+        mul_acc(Xt, Tmjt, Aim);
+      }
+      Frag Tij = mul(Tii, Xt);   // T_ii X
+      Frag Tijt = mul(Xt, Tii);  // X^T T_ii^T
+      negate(Tij);
+      negate(Tijt);
+      store_frag(ThT, j, i, Tijt, lane);
+      put(i, j, Tij, lane);
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace tri
+}  // namespace dr

@@ -7,6 +7,7 @@
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tri_inverse.cuh"
 
 namespace dr {
 
@@ -75,6 +76,32 @@ umma_selftest_kernel(const uint16_t *__restrict__ A, const uint16_t *__restrict_
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tb, 128);
+}
+
+// T = (I + A)^-1 for the strictly lower part of a 64 x 64 fp32 matrix A (row-major),
+// through the same warp-MMA routine the prefill kernel uses.  T (row-major fp32)
+// must be zeroed by the caller: only its lower blocks are written.  128 threads.
+__global__ void __launch_bounds__(128) tri_selftest_kernel(const float *__restrict__ A, float *__restrict__ Tout) {
+  __shared__ __align__(16) __half Ah[64 * tri::LD], AhT[64 * tri::LD], ThT[64 * tri::LD];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < 64 * 64; e += blockDim.x) {
+    const int r = e / 64, c = e % 64;
+    const __half a = __float2half_rn(c < r ? A[e] : 0.f);
+    Ah[r * tri::LD + c] = a;
+    AhT[c * tri::LD + r] = a;
+  }
+  __syncthreads();
+  tri::inverse64(Ah, AhT, ThT, warp, lane, [&](int bi, int bj, const tri::Frag &F, int ln) {
+    const int row = 16 * bi + (ln >> 2), col = 16 * bj + 2 * (ln & 3);
+    Tout[row * 64 + col] = F.v[0];
+    Tout[row * 64 + col + 1] = F.v[1];
+    Tout[(row + 8) * 64 + col] = F.v[2];
+    Tout[(row + 8) * 64 + col + 1] = F.v[3];
+    Tout[row * 64 + col + 8] = F.v[4];
+    Tout[row * 64 + col + 9] = F.v[5];
+    Tout[(row + 8) * 64 + col + 8] = F.v[6];
+    Tout[(row + 8) * 64 + col + 9] = F.v[7];
+  });
 }
 
 }  // namespace dr
