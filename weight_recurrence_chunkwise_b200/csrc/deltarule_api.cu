@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -12,13 +13,24 @@
 #include "../../include/deltarule_diag.h"
 #include "chunk_simt.cuh"
 #include "chunk_tc.cuh"
+#include "chunk_tc2.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "umma_selftest.cuh"
 
 namespace {
 
-constexpr size_t kWorkspaceBytes = 256;  // status word, padded to an allocation granule
+constexpr size_t kWorkspaceBytes = 256;
+
+// The two-CTA prefill is the default for dv = 128; DR_PREFILL_SINGLE_CTA=1 selects the
+// one-CTA-per-value-slice kernel instead (same results, used to compare the two).
+bool prefill_pair_enabled() {
+  static const bool on = [] {
+    const char *e = std::getenv("DR_PREFILL_SINGLE_CTA");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}  // status word, padded to an allocation granule
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -116,16 +128,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // 4-D map over a [B, T, H, D] row-major tensor (dims innermost first: D, H, T, B) with a box of
 // `box_d` elements x 1 head x `box_t` tokens x 1 batch row; out-of-range rows read as zero.
 bool make_map(CUtensorMap *m, CUtensorMapDataType dt, size_t esize, const void *base, int B, int T, int H, int D,
-              int box_d, int box_t) {
+              int box_d, int box_t, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
   const cuuint64_t strides[3] = {cuuint64_t(D) * esize, cuuint64_t(D) * H * esize, cuuint64_t(D) * H * T * esize};
   const cuuint32_t box[4] = {cuuint32_t(box_d), 1u, cuuint32_t(box_t), 1u};
   const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-  return enc(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 dr_status tc_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
@@ -154,6 +165,52 @@ dr_status tc_launch(const dr_problem *p, const void *q, const void *k, const voi
     return DR_ERR_CUDA;
   dim3 grid(p->dv / tc::VS, p->H, p->B);
   kern<<<grid, tc::NT, smem, st>>>(mq, mk, mv, mbv, prm);
+  return launch_status();
+}
+
+// Two-CTA cluster per (b, h): the value slices 0..63 and 64..127 share the chunk-local factors.
+dr_status tc_pair_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                         const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
+                         uint32_t *status, cudaStream_t st) {
+  using IO = __nv_bfloat16;
+  namespace tc = dr::tc;
+  namespace tc2 = dr::tc2;
+  alignas(64) CUtensorMap mq, mk, mv, mb;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_map(&mq, bf, 2, q, p->B, p->T, p->H, p->dk, tc::DK, tc::C) ||
+      !make_map(&mk, bf, 2, k, p->B, p->T, p->H, p->dk, 64, tc::C, sw) ||
+      !make_map(&mv, bf, 2, v, p->B, p->T, p->H, p->dv, tc::VS, tc::C, sw))
+    return DR_ERR_CUDA;
+  const bool bv = p->beta_v_mode == DR_CHANNEL;
+  const bool sym = p->beta_v_mode == DR_ABSENT && p->beta_k_mode == DR_CHANNEL;
+  if (bv || sym) {
+    if (!make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, bv ? static_cast<const void *>(beta_v) : beta_k, p->B,
+                  p->T, p->H, bv ? p->dv : p->dk, tc::VS, tc::C))
+      return DR_ERR_CUDA;
+  } else {
+    mb = mv;  // unused by the kernel in this mode
+  }
+  tc::Params prm{p->T, p->H, p->dv, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v, p->beta_v_mode,
+                 S0, o, S_T, status};
+  auto kern = tc2::chunk_fwd_pair_kernel<IO>;
+  constexpr size_t smem = tc2::SMEM_BYTES;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return DR_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, p->H, p->B);
+  cfg.blockDim = dim3(tc2::NT, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mb, prm) != cudaSuccess) return DR_ERR_CUDA;
   return launch_status();
 }
 
@@ -225,6 +282,8 @@ dr_status dr_chunk_fwd(const dr_problem *p, const void *q, const void *k, const 
   }
   if (p->io_dtype == DR_F32)
     return simt_dispatch<float>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+  if (p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv == 2 * dr::tc::VS && prefill_pair_enabled())
+    return tc_pair_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
   if (p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv % dr::tc::VS == 0)
     return tc_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
   return simt_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);

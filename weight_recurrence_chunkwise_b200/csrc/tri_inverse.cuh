@@ -108,18 +108,34 @@ __device__ __forceinline__ void store_frag(__half *M, int bi, int bj, const Frag
   *reinterpret_cast<uint32_t *>(base + 8 * LD + 8) = h2u(F.v[6], F.v[7]);
 }
 
-// Called by every thread of the CTA (contains __syncthreads); warps 0..3 work.
-// Ah, AhT: A and A^T (fp16, row stride LD, zero on and above A's diagonal).
-// ThT: scratch for T^T (fp16, row stride LD).
+// Block (bi, bj) of the transpose of a row-major fp16 array: F(X^T) for X = M[bi][bj].
+__device__ __forceinline__ Frag load_frag_t(const __half *M, int bi, int bj, int lane) {
+  const int r = lane >> 2, q = lane & 3;
+  const __half *base = M + (16 * bi + 2 * q) * LD + 16 * bj + r;
+  Frag F;
+  F.v[0] = __half2float(base[0]);
+  F.v[1] = __half2float(base[LD]);
+  F.v[2] = __half2float(base[8]);
+  F.v[3] = __half2float(base[LD + 8]);
+  F.v[4] = __half2float(base[8 * LD]);
+  F.v[5] = __half2float(base[9 * LD]);
+  F.v[6] = __half2float(base[8 * LD + 8]);
+  F.v[7] = __half2float(base[9 * LD + 8]);
+  return F;
+}
+
+// Called by every thread of the participating group (contains `sync()` barriers); warps 0..3 work.
+// Ah: A (fp16, row stride LD, zero on and above A's diagonal); AhT: A^T, or nullptr to read
+// the transposes from Ah.  ThT: scratch for T^T (fp16, row stride LD).
 // put(bi, bj, F, lane): receives each lower block T_ij (i >= j) of the result.
-template <typename Put>
+template <typename Put, typename Sync>
 __device__ __forceinline__ void inverse64(const __half *Ah, const __half *AhT, __half *ThT, int warp, int lane,
-                                          Put put) {
+                                          Put put, Sync sync) {
   Frag Tii;  // diagonal block of this warp, kept for the off-diagonal levels
   if (warp < 4) {
     const int b = warp;
     const Frag N = load_frag(Ah, b, b, lane);
-    const Frag Nt = load_frag(AhT, b, b, lane);
+    const Frag Nt = AhT ? load_frag(AhT, b, b, lane) : load_frag_t(Ah, b, b, lane);
     const Frag N2 = mul(N, Nt), N2t = mul(Nt, N);
     const Frag N4 = mul(N2, N2t), N4t = mul(N2t, N2);
     const Frag N8t = mul(N4t, N4);
@@ -134,7 +150,7 @@ __device__ __forceinline__ void inverse64(const __half *Ah, const __half *AhT, _
     store_frag(ThT, b, b, Tt, lane);
     put(b, b, Tii, lane);
   }
-  __syncthreads();
+  sync();
 #pragma unroll 1
   for (int d = 1; d < 4; ++d) {
     if (warp >= d && warp < 4) {
@@ -155,7 +171,7 @@ __device__ __forceinline__ void inverse64(const __half *Ah, const __half *AhT, _
       store_frag(ThT, j, i, Tijt, lane);
       put(i, j, Tij, lane);
     }
-    __syncthreads();
+    sync();
   }
 }
 

@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(128) tri_selftest_kernel(const float *__restri
     Tout[row * 64 + col + 9] = F.v[5];
     Tout[(row + 8) * 64 + col + 8] = F.v[6];
     Tout[(row + 8) * 64 + col + 9] = F.v[7];
-  });
+  }, [] { __syncthreads(); });
 }
 
 }  // namespace dr
