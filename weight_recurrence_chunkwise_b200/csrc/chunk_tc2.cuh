@@ -72,9 +72,11 @@ constexpr uint32_t SLOT_BYTES = 2 * 128 * 128 + 64 * 256 + 128 * 128 + 512;  // 
 constexpr uint32_t COL_D1 = 0;     // local: [P raw | A raw] (64)
 constexpr uint32_t COL_D2 = 64;    // local: W (128)
 constexpr uint32_t COL_U0 = 192;   // chain: U0 (64)
-constexpr uint32_t COL_D3 = 256;   // chain: [-W S | Qh S + P U] (64)
+constexpr uint32_t COL_D3 = 256;   // chain: [-W S | Qh S + P U] (64), even chunks
 constexpr uint32_t COL_D4 = 320;   // chain: Ac^T U (64)
+constexpr uint32_t COL_D3B = 384;  // chain: D3 of odd chunks (64)
 constexpr uint32_t TMEM_COLS = 512;
+__host__ __device__ constexpr uint32_t col_d3(int c) { return (c & 1) ? COL_D3B : COL_D3; }
 
 __host__ __device__ constexpr uint32_t off_ac(int s) { return s ? OFF_AC1 : OFF_AC0; }
 __host__ __device__ constexpr uint32_t off_tp(int s) { return s ? OFF_TP1 : OFF_TP0; }
@@ -161,9 +163,26 @@ chunk_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       tma_load_4d(sm + OFF_STK + 128 * 128, &tm_k, &bar_qk, 0, h, t0, b);             // raw k -> Bh rows
       tma_load_4d(sm + OFF_STK + STK_ROWS * 128 + 128 * 128, &tm_k, &bar_qk, 64, h, t0, b);
     };
+    // Scalar gates (alpha absent or per token, beta_k per token): warp 0 stages the 64 row gates
+    // of the next chunk in shared memory by cp.async (lane l: rows 2l, 2l+1); everything else is
+    // per element.
+    const bool gates_scalar = p.alpha_mode != MODE_CHANNEL && p.beta_k_mode == MODE_SCALAR;
+    float *sGate = reinterpret_cast<float *>(sm + OFF_PX) + 256;  // [0..63] alpha, [64..127] beta_k
     auto prefetch_gates = [&](int c) {  // loads only; masking and broadcast happen at use
       const int t0 = c * C, L = min(C, T - t0);
       const size_t thb = (static_cast<size_t>(b) * T + t0) * H + h;
+      if (gates_scalar) {
+        if (warp == 0) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const size_t th = thb + static_cast<size_t>(min(2 * lane + e, L - 1)) * H;
+            if (p.alpha_mode == MODE_SCALAR) cp_async4(sGate + 2 * lane + e, p.alpha + th);
+            cp_async4(sGate + 64 + 2 * lane + e, p.beta_k + th);
+          }
+          cp_async_commit();
+        }
+        return;
+      }
 #pragma unroll
       for (int j = 0; j < RGL; ++j) {
         const size_t th = thb + static_cast<size_t>(min(rgl * RGL + j, L - 1)) * H;
@@ -231,7 +250,65 @@ chunk_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       if (!wait_all(&bar_qk, ph_qk)) { aborted = true; break; }
 
       // -------------------------------------------------------------- K1 + a0: Qh, Bh (in place), Ac, gamma_C
-      {
+      if (gates_scalar) {
+        // row gates: gamma_r (inclusive product), 1/gamma_r, sqrt(beta_r); 64 rows over warp 0
+        float *sRow = sPX;  // [0..63] gamma, [64..127] 1/gamma, [128..191] sqrt(beta)
+        if (warp == 0) {
+          cp_async_wait_all();  // this lane's own staged rows
+          const float2 ga = *reinterpret_cast<const float2 *>(sGate + 2 * lane);
+          const float2 gb = *reinterpret_cast<const float2 *>(sGate + 64 + 2 * lane);
+          const bool asc = p.alpha_mode == MODE_SCALAR;
+          const float a0 = (asc && 2 * lane < L) ? ga.x : 1.f, a1 = (asc && 2 * lane + 1 < L) ? ga.y : 1.f;
+          const float b0 = (2 * lane < L) ? gb.x : 0.f, b1 = (2 * lane + 1 < L) ? gb.y : 0.f;
+          float pr = a0 * a1, incl = pr;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl *= y;
+          }
+          const float up = __shfl_up_sync(0xffffffffu, incl, 1);
+          const float ex = (lane == 0) ? 1.f : up;  // product of the rows before 2*lane
+          const float g0 = ex * a0, g1 = g0 * a1;
+          const float gC = __shfl_sync(0xffffffffu, incl, 31);
+          sRow[2 * lane] = g0;
+          sRow[2 * lane + 1] = g1;
+          sRow[64 + 2 * lane] = __fdividef(1.f, g0);
+          sRow[64 + 2 * lane + 1] = __fdividef(1.f, g1);
+          sRow[128 + 2 * lane] = tc::sqrt_fast(b0);
+          sRow[128 + 2 * lane + 1] = tc::sqrt_fast(b1);
+          *reinterpret_cast<float4 *>(sGC + 4 * lane) = make_float4(gC, gC, gC, gC);
+          if (lane == 0 && !(gC >= kMinChunkDecayF16)) raise_status(p.status, STATUS_RANGE);
+        }
+        bar_sync(BAR_LOCAL, NL);
+        // elements: (row r, 8-column chunk j8), four per thread, 16-byte loads and stores
+        const int j8 = ltid & 15;
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = (ltid >> 4) + 16 * i;
+          const float g = sRow[r], gi = sRow[64 + r], sb = sRow[128 + r];
+          const uint4 qraw = *reinterpret_cast<const uint4 *>(rQ + (r * DK + j8 * 8) * 2);
+          uint4 *pk = reinterpret_cast<uint4 *>(tQB + sw128_off16(128 + r, j8, STK_ROWS));
+          const uint4 kraw = *pk;
+          const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qraw);
+          const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kraw);
+          uint32_t oq[4], ob[4], oa[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 qf = __bfloat1622float2(q2[e]), kf = __bfloat1622float2(k2[e]);
+            const float b0 = sb * kf.x, b1 = sb * kf.y;
+            const float x0 = b0 * gi, x1 = b1 * gi;
+            amax = fmaxf(amax, fmaxf(fabsf(x0), fabsf(x1)));
+            oq[e] = pack_f16x2(g * qf.x, g * qf.y);
+            ob[e] = pack_f16x2(g * b0, g * b1);
+            oa[e] = pack_f16x2(x0, x1);
+          }
+          *reinterpret_cast<uint4 *>(tQB + sw128_off16(row_q(s) + r, j8, STK_ROWS)) = make_uint4(oq[0], oq[1], oq[2], oq[3]);
+          *pk = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+          *reinterpret_cast<uint4 *>(tAC + sw128_off16(r, j8, 64)) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+        }
+        if (!(amax < kF16Max)) raise_status(p.status, STATUS_RANGE);
+      } else {
 #pragma unroll
         for (int j = 0; j < RGL; ++j) {
           const bool valid = rgl * RGL + j < L;
@@ -305,15 +382,29 @@ chunk_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       }
       fence_async_smem();
       bar_sync(BAR_LOCAL, NL);
+      const uint32_t rbar = mapa_shared(smem_u32(&bar_full[s]), static_cast<uint32_t>(peer));
+      auto copy_part = [&](uint32_t off, uint32_t bytes) {
+        bulk_copy_to_peer(mapa_shared(sbase_addr + off, static_cast<uint32_t>(peer)), sm + off, bytes, rbar);
+      };
 
       // -------------------------------------------------------------- m1: D1 = [Qh; Bh] Ac^T (halves swapped for slot 1)
-      if (ltid == 0) {
-        tc_fence_after();
-        const uint32_t idesc = idesc_f16_f32(128, 64, false, false);
+      if (warp == 0) {
+        if (elect_one()) {
+          tc_fence_after();
+          const uint32_t idesc = idesc_f16_f32(128, 64, false, false);
 #pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk)
-          umma_f16(tmem + COL_D1, kstep(dM1, STK_ROWS, kk), kstep(dAcK, 64, kk), idesc, kk > 0);
-        umma_commit(&bar_lmma);
+          for (int kk = 0; kk < DK / 16; ++kk)
+            umma_f16(tmem + COL_D1, kstep(dM1, STK_ROWS, kk), kstep(dAcK, 64, kk), idesc, kk > 0);
+          umma_commit(&bar_lmma);
+          // Qh, Ac and gamma_C of this chunk are final: start moving them into the peer's slot.  The
+          // peer's full[s] phase completes on the copied bytes alone, so the arrive needs no release.
+          mbar_expect_tx_remote_relaxed(rbar, SLOT_BYTES);
+          copy_part(OFF_STK + row_q(s) * 128, 64 * 128);
+          copy_part(OFF_STK + STK_ROWS * 128 + row_q(s) * 128, 64 * 128);
+          copy_part(off_ac(s), 64 * 256);
+          copy_part(off_gc(s), 512);
+        }
+        __syncwarp();
       }
       if (c + 2 < nchunks) prefetch_gates(c + 2);
       if (!wait_one(&bar_lmma, ph_mma, false)) { aborted = true; break; }
@@ -336,12 +427,20 @@ chunk_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             for (int i = 0; i < 16; ++i) x[i] = (half * 32 + jh + i <= r) ? x[i] : 0.f;
             tc::st_h16x16(tTP, pl + r, half * 32 + jh, 128, x);
           } else {
+            const int col0 = half * 32 + jh;
 #pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-              const int col = half * 32 + jh + i;
-              const float x0 = (col < r) ? x[i] : 0.f, x1 = (col + 1 < r) ? x[i + 1] : 0.f;
-              *reinterpret_cast<uint32_t *>(sAh + r * tri::LD + col) = pack_f16x2(x0, x1);
-            }
+            for (int i = 0; i < 16; ++i) x[i] = (col0 + i < r) ? x[i] : 0.f;
+            uint4 lo, hi;  // 16-byte stores: rows are 144 bytes apart, conflict-free per 8 lanes
+            lo.x = pack_f16x2(x[0], x[1]);
+            lo.y = pack_f16x2(x[2], x[3]);
+            lo.z = pack_f16x2(x[4], x[5]);
+            lo.w = pack_f16x2(x[6], x[7]);
+            hi.x = pack_f16x2(x[8], x[9]);
+            hi.y = pack_f16x2(x[10], x[11]);
+            hi.z = pack_f16x2(x[12], x[13]);
+            hi.w = pack_f16x2(x[14], x[15]);
+            *reinterpret_cast<uint4 *>(sAh + r * tri::LD + col0) = lo;
+            *reinterpret_cast<uint4 *>(sAh + r * tri::LD + col0 + 8) = hi;
           }
         }
       }
@@ -361,13 +460,17 @@ chunk_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       bar_sync(BAR_LOCAL, NL);
 
       // -------------------------------------------------------------- m2: D2 = [T;P] Bh -> W at lanes tl
-      if (ltid == 0) {
-        tc_fence_after();
-        const uint32_t id2 = idesc_f16_f32(128, 128, false, true);
+      if (warp == 0) {
+        if (elect_one()) {
+          copy_part(off_tp(s), 128 * 128);  // [T; P] is final
+          tc_fence_after();
+          const uint32_t id2 = idesc_f16_f32(128, 128, false, true);
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk)
-          umma_f16(tmem + COL_D2, kstep(dTP, 128, kk), mstep(dBh, kk), id2, kk > 0);
-        umma_commit(&bar_lmma);
+          for (int kk = 0; kk < C / 16; ++kk)
+            umma_f16(tmem + COL_D2, kstep(dTP, 128, kk), mstep(dBh, kk), id2, kk > 0);
+          umma_commit(&bar_lmma);
+        }
+        __syncwarp();
       }
       if (!wait_one(&bar_lmma, ph_mma, false)) { aborted = true; break; }
       // Bh and the inverse scratch are free: fetch chunk c+2's raw q and k now
@@ -392,16 +495,8 @@ chunk_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
       // -------------------------------------------------------------- hand the slot to both state passes
       if (ltid == 0) {
-        const uint32_t rbar = mapa_shared(smem_u32(&bar_full[s]), static_cast<uint32_t>(peer));
-        mbar_arrive_expect_tx_remote(rbar, SLOT_BYTES);
-        auto copy = [&](uint32_t off, uint32_t bytes) {
-          bulk_copy_to_peer(mapa_shared(sbase_addr + off, static_cast<uint32_t>(peer)), sm + off, bytes, rbar);
-        };
-        copy(OFF_STK + row_chain(s) * 128, 128 * 128);
-        copy(OFF_STK + STK_ROWS * 128 + row_chain(s) * 128, 128 * 128);
-        copy(off_ac(s), 64 * 256);
-        copy(off_tp(s), 128 * 128);
-        copy(off_gc(s), 512);
+        copy_part(OFF_STK + row_w(s) * 128, 64 * 128);
+        copy_part(OFF_STK + STK_ROWS * 128 + row_w(s) * 128, 64 * 128);
         mbar_arrive(&bar_full[s]);
       }
     }
@@ -466,77 +561,119 @@ chunk_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       tc::st_h16x16(tS, trow, half * 32, 128, Sreg);
       tc::st_h16x16(tS, trow, half * 32 + 16, 128, Sreg + 16);
     }
-    if (nchunks > 0) {
-      if (ct == 0) issue_v(0);
-      prefetch_ws(0);
-    }
     const uint64_t dS = sdesc_sw128(sbase_addr + OFF_S, 128 * 128, 1024);
     const uint64_t dU = sdesc_sw128(sbase_addr + OFF_U, 64 * 128, 1024);
     const uint64_t dWr = sdesc_sw128(sbase_addr + OFF_WR, 64 * 128, 1024);
 
-    for (int c = 0; c < nchunks; ++c) {
-      const int s = c & 1, t0 = c * C, L = min(C, T - t0);
-      const int tl = lane_t(s), pl = lane_p(s);
-      if (!wait_all(&bar_v, ph_v, false)) { aborted = true; break; }
-      // -------------------------------------------------------------- write vectors, in place over raw v
-      {
-        float sc[16];
-        if (scale_tma) {
+    // write vectors of the chunk whose raw v sits in Wr, in place (after bar_v)
+    auto convert_wr = [&]() {
+      float sc[16];
+      if (scale_tma) {
 #pragma unroll
-          for (int i = 0; i < 16; i += 4) {
-            const float4 x = *reinterpret_cast<const float4 *>(rB + wc * VS + wjb * 8 + i);
-            sc[i] = x.x;
-            sc[i + 1] = x.y;
-            sc[i + 2] = x.z;
-            sc[i + 3] = x.w;
-          }
-          if (sym_channel) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) sc[i] = tc::sqrt_fast(sc[i]);
-          }
-        } else {
-          const float s0 = (p.beta_v_mode == MODE_SCALAR) ? pws : tc::sqrt_fast(pws);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) sc[i] = s0;
+        for (int i = 0; i < 16; i += 4) {
+          const float4 x = *reinterpret_cast<const float4 *>(rB + wc * VS + wjb * 8 + i);
+          sc[i] = x.x;
+          sc[i + 1] = x.y;
+          sc[i + 2] = x.z;
+          sc[i + 3] = x.w;
         }
+        if (sym_channel) {
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          uint4 *ptr = reinterpret_cast<uint4 *>(tWR + sw128_off16(wc, wjb + jj, 64));
-          const uint4 raw = *ptr;
-          const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-          float w8[8];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 vf = __bfloat1622float2(v2[i]);
-            w8[2 * i] = sc[jj * 8 + 2 * i] * vf.x;  // rows >= L: v = 0 (TMA fill)
-            w8[2 * i + 1] = sc[jj * 8 + 2 * i + 1] * vf.y;
-          }
-          uint4 out;
-          out.x = pack_f16x2(w8[0], w8[1]);
-          out.y = pack_f16x2(w8[2], w8[3]);
-          out.z = pack_f16x2(w8[4], w8[5]);
-          out.w = pack_f16x2(w8[6], w8[7]);
-          *ptr = out;
+          for (int i = 0; i < 16; ++i) sc[i] = tc::sqrt_fast(sc[i]);
         }
+      } else {
+        const float s0 = (p.beta_v_mode == MODE_SCALAR) ? pws : tc::sqrt_fast(pws);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sc[i] = s0;
+      }
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        uint4 *ptr = reinterpret_cast<uint4 *>(tWR + sw128_off16(wc, wjb + jj, 64));
+        const uint4 raw = *ptr;
+        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+        float w8[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 vf = __bfloat1622float2(v2[i]);
+          w8[2 * i] = sc[jj * 8 + 2 * i] * vf.x;  // rows >= L: v = 0 (TMA fill)
+          w8[2 * i + 1] = sc[jj * 8 + 2 * i + 1] * vf.y;
+        }
+        uint4 out;
+        out.x = pack_f16x2(w8[0], w8[1]);
+        out.y = pack_f16x2(w8[2], w8[3]);
+        out.z = pack_f16x2(w8[4], w8[5]);
+        out.w = pack_f16x2(w8[6], w8[7]);
+        *ptr = out;
+      }
+    };
+    // outputs of chunk c: its D3 columns at lanes pl hold Qh S + P U
+    auto store_o = [&](int c) {
+      const int pl = lane_p(c & 1), t0 = c * C, L = min(C, T - t0);
+      if ((quarter * 32 >= pl) && (quarter * 32 < pl + 64)) {
+        const int r = trow - pl;
+#pragma unroll
+        for (int j = 0; j < 32; j += 16) {
+          float x[16];
+          tmem_ld16(tmem_addr(tmem, quarter * 32, col_d3(c) + half * 32 + j), x);
+          tmem_ld_wait();
+          if (r < L) {
+            const size_t th = (static_cast<size_t>(b) * T + t0 + r) * H + h;
+            IO *dst = static_cast<IO *>(p.o) + th * DV + v0 + half * 32 + j;
+            uint4 lo, hi;
+            lo.x = pack_bf16x2(x[0], x[1]);
+            lo.y = pack_bf16x2(x[2], x[3]);
+            lo.z = pack_bf16x2(x[4], x[5]);
+            lo.w = pack_bf16x2(x[6], x[7]);
+            hi.x = pack_bf16x2(x[8], x[9]);
+            hi.y = pack_bf16x2(x[10], x[11]);
+            hi.z = pack_bf16x2(x[12], x[13]);
+            hi.w = pack_bf16x2(x[14], x[15]);
+            reinterpret_cast<uint4 *>(dst)[0] = lo;
+            reinterpret_cast<uint4 *>(dst)[1] = hi;
+          }
+        }
+      }
+    };
+
+    // Software pipeline: the write vectors of chunk c+1 are built while the second MMA group of
+    // chunk c runs, and the outputs of chunk c are stored while the first MMA group of chunk c+1
+    // runs (D3 alternates between two column sets), so the serial path per chunk is
+    // MMA group 1 -> U -> MMA group 2 -> S.
+    if (nchunks > 0) {
+      if (ct == 0) issue_v(0);
+      prefetch_ws(0);
+      if (wait_all(&bar_v, ph_v, false)) {
+        convert_wr();
+        if (nchunks > 1) prefetch_ws(1);
+      } else {
+        aborted = true;
       }
       fence_async_smem();
       bar_sync(BAR_CHAIN, NT - NL);
-      if (c + 1 < nchunks) prefetch_ws(c + 1);
+    }
+    for (int c = 0; c < nchunks && !aborted; ++c) {
+      const int s = c & 1;
+      const int tl = lane_t(s);
+      const uint32_t cD3 = col_d3(c);
       if (!wait_all(&bar_full[s], ph_full[s], true)) { aborted = true; break; }
       const float gc = reinterpret_cast<const float *>(sm + off_gc(s))[trow];
 
       // -------------------------------------------------------------- U0 = [T;P] Wr,  D3 = STK(s) S
-      if (ct == 0) {
-        tc_fence_after();
-        const uint64_t dTP = sdesc_sw128(sbase_addr + off_tp(s), 16, 1024);
-        const uint64_t dCh = sdesc_sw128(sbase_addr + OFF_STK + row_chain(s) * 128, 16, 1024);
-        const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
+      if (cw == 0) {
+        if (elect_one()) {
+          tc_fence_after();
+          const uint64_t dTP = sdesc_sw128(sbase_addr + off_tp(s), 16, 1024);
+          const uint64_t dCh = sdesc_sw128(sbase_addr + OFF_STK + row_chain(s) * 128, 16, 1024);
+          const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_U0, kstep(dTP, 128, kk), mstep(dWr, kk), id3, kk > 0);
+          for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_U0, kstep(dTP, 128, kk), mstep(dWr, kk), id3, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < DK / 16; ++kk) umma_f16(tmem + COL_D3, kstep(dCh, STK_ROWS, kk), mstep(dS, kk), id3, kk > 0);
-        umma_commit(&bar_cmma);
+          for (int kk = 0; kk < DK / 16; ++kk) umma_f16(tmem + cD3, kstep(dCh, STK_ROWS, kk), mstep(dS, kk), id3, kk > 0);
+          umma_commit(&bar_cmma);
+        }
+        __syncwarp();
       }
+      if (c > 0) store_o(c - 1);
       if (!wait_mma()) { aborted = true; break; }
       if (ct == 0 && c + 1 < nchunks) issue_v(c + 1);  // Wr and the scale staging are free
 
@@ -546,7 +683,7 @@ chunk_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
         for (int j = 0; j < 32; j += 16) {
           float ws[16], u0[16];
-          tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D3 + half * 32 + j), ws);
+          tmem_ld16(tmem_addr(tmem, quarter * 32, cD3 + half * 32 + j), ws);
           tmem_ld16(tmem_addr(tmem, quarter * 32, COL_U0 + half * 32 + j), u0);
           tmem_ld_wait();
           float mx = 0.f;
@@ -564,17 +701,27 @@ chunk_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       bar_sync(BAR_CHAIN, NT - NL);
 
       // -------------------------------------------------------------- D4 = Ac^T U,  D3 += [T;P] U
-      if (ct == 0) {
-        tc_fence_after();
-        const uint64_t dAcM = sdesc_sw128(sbase_addr + off_ac(s), 64 * 128, 1024);
-        const uint64_t dTP = sdesc_sw128(sbase_addr + off_tp(s), 16, 1024);
-        const uint32_t id4 = idesc_f16_f32(128, VS, true, true);
-        const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
+      if (cw == 0) {
+        if (elect_one()) {
+          tc_fence_after();
+          const uint64_t dAcM = sdesc_sw128(sbase_addr + off_ac(s), 64 * 128, 1024);
+          const uint64_t dTP = sdesc_sw128(sbase_addr + off_tp(s), 16, 1024);
+          const uint32_t id4 = idesc_f16_f32(128, VS, true, true);
+          const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_D4, mstep(dAcM, kk), mstep(dU, kk), id4, kk > 0);
+          for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_D4, mstep(dAcM, kk), mstep(dU, kk), id4, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_D3, kstep(dTP, 128, kk), mstep(dU, kk), id3, 1u);
-        umma_commit(&bar_cmma);
+          for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + cD3, kstep(dTP, 128, kk), mstep(dU, kk), id3, 1u);
+          umma_commit(&bar_cmma);
+        }
+        __syncwarp();
+      }
+      // write vectors of the next chunk while these MMAs run
+      if (c + 1 < nchunks) {
+        if (!wait_all(&bar_v, ph_v, false)) { aborted = true; break; }
+        convert_wr();
+        if (c + 2 < nchunks) prefetch_ws(c + 2);
+        fence_async_smem();
       }
       if (!wait_mma()) { aborted = true; break; }
       // this CTA's copy of slot s is no longer read
@@ -583,7 +730,7 @@ chunk_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         else mbar_arrive_remote(mapa_shared(smem_u32(&bar_peer_free), static_cast<uint32_t>(peer)));
       }
 
-      // -------------------------------------------------------------- E4: S update, outputs
+      // -------------------------------------------------------------- E4: S <- Diag(gamma_C) (S + Ac^T U)
       {
         float mx = 0.f;
 #pragma unroll
@@ -599,35 +746,12 @@ chunk_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           tc::st_h16x16(tS, trow, half * 32 + j, 128, Sreg + j);
         }
         if (!(mx < kF16Max)) raise_status(p.status, STATUS_RANGE);
-        if ((quarter * 32 >= pl) && (quarter * 32 < pl + 64)) {
-          const int r = trow - pl;
-#pragma unroll
-          for (int j = 0; j < 32; j += 16) {
-            float x[16];
-            tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D3 + half * 32 + j), x);
-            tmem_ld_wait();
-            if (r < L) {
-              const size_t th = (static_cast<size_t>(b) * T + t0 + r) * H + h;
-              IO *dst = static_cast<IO *>(p.o) + th * DV + v0 + half * 32 + j;
-              uint4 lo, hi;
-              lo.x = pack_bf16x2(x[0], x[1]);
-              lo.y = pack_bf16x2(x[2], x[3]);
-              lo.z = pack_bf16x2(x[4], x[5]);
-              lo.w = pack_bf16x2(x[6], x[7]);
-              hi.x = pack_bf16x2(x[8], x[9]);
-              hi.y = pack_bf16x2(x[10], x[11]);
-              hi.z = pack_bf16x2(x[12], x[13]);
-              hi.w = pack_bf16x2(x[14], x[15]);
-              reinterpret_cast<uint4 *>(dst)[0] = lo;
-              reinterpret_cast<uint4 *>(dst)[1] = hi;
-            }
-          }
-        }
       }
       fence_async_smem();
       tc_fence_before();
       bar_sync(BAR_CHAIN, NT - NL);
     }
+    if (!aborted && nchunks > 0) store_o(nchunks - 1);
     if (!aborted && p.S_T) {
       float *dst = p.S_T + sbase + static_cast<size_t>(trow) * DV + v0 + half * 32;
 #pragma unroll

@@ -113,6 +113,20 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t remote_bar
                "r"(bytes)
                : "memory");
 }
+// Same, without release ordering: for a barrier whose phase is completed by bulk-copy bytes only,
+// which carry their own visibility, so none of this thread's earlier writes need to be ordered.
+__device__ __forceinline__ void mbar_expect_tx_remote_relaxed(uint32_t remote_bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(remote_bar),
+               "r"(bytes)
+               : "memory");
+}
+// 4-byte asynchronous global -> shared copy (L1-allocating), and the wait for all of this
+// thread's outstanding ones.
+__device__ __forceinline__ void cp_async4(void *dst_smem, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 // Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from this CTA's shared
 // memory into another CTA's shared memory; completes on that CTA's barrier `remote_bar`.
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t remote_dst, const void *src, uint32_t bytes,
@@ -247,6 +261,17 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+// One lane of a converged warp (the lowest active one) returns true.  Issuing single-thread
+// instructions this way keeps the whole warp converged around them.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
 }
 // Arrive once on `bar` when every MMA previously issued by this thread has completed.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
