@@ -1,0 +1,802 @@
+// chunk_tc3.cuh -- chunkwise WY/UT prefill on a cluster of two CTAs per (b, h), with a ring of
+// three factor slots.
+//
+// Algebra (DeltaNet page, step 7; FG2-GDN page, section 2), per chunk of C = 64 tokens:
+//   chunk-local:  gamma, Qh = gamma q, Bh = gamma b, Ac = b / gamma, P = lower(Qh Ac^T),
+//                 T = (I + strictly-lower(Bh Ac^T))^-1, W = T Bh
+//   state pass:   U0 = T Wr, U = U0 - W S, O = Qh S + P U, S <- Diag(gamma_C)(S + Ac^T U)
+//
+// Work split (as in chunk_tc2.cuh): CTA r of the pair runs the state pass for value columns
+// 64r..64r+63 over every chunk (chain role, warps 8..15), and builds the chunk-local factors of
+// the chunks c with c % 2 == r (local role, warps 0..7), which it writes into slot c % 3 of both
+// CTAs (its own by plain stores, the peer's by DSMEM bulk copies).
+//
+// Three slots instead of two let the local role of chunk c start as soon as the state passes
+// are done with chunk c-3, so the local work of a chunk overlaps the state pass of the two
+// chunks before it.  To fit three slots in shared memory, every working buffer of the local role
+// lives inside the slot it is filling:
+//   X  (128 rows x 128 fp16, K-major, 128B-swizzled, two column blocks of 128 rows)
+//        rows 0..63:   raw k (TMA) -> Bh (in place) -> -W;  then U in the state pass
+//        rows 64..127: raw q (TMA) -> Qh (in place)
+//   AC (64 x 128): Ac
+//   TP (128 x 64): [T; P]; before that the gate rows of K1, then A (rows 0..63) and the T^T
+//        scratch of the inverse (rows 64..127)
+// so [Bh; Qh] (local MMA) and [-W; Qh] (state-pass MMA) are the same 128 rows, and every TMEM
+// lane map is fixed: lanes 0..63 carry A, W, U0, -W S; lanes 64..127 carry P, Qh S, O.
+//
+// Synchronisation (every wait bounded):
+//   full[j]  slot j holds the factors of its current chunk (local arrive in the producing CTA;
+//            remote arrive.expect_tx + copied bytes in the other)
+//   free[j]  (in the CTA producing the slot's next chunk) both state passes are done with it
+//   land[j]  (in the producing CTA) the other CTA has received the slot, so the bulk copies
+//            have finished reading it and the producing CTA's state pass may write U into it
+#pragma once
+#include "chunk_tc.cuh"
+
+namespace dr {
+namespace tc3 {
+
+using tc::C;
+using tc::DK;
+using tc::VS;
+using tc::kF16Max;
+using tc::kMinChunkDecayF16;
+using tc::Params;
+
+constexpr int NT = 512;  // threads
+constexpr int NL = 256;  // local role: threads 0..255
+constexpr int BAR_LOCAL = 1, BAR_CHAIN = 2;
+constexpr int RGL = 16;  // rows per local elementwise thread in the channel-gate K1
+constexpr int NSLOT = 3;
+
+// slot layout (bytes from the slot base); every tile 1024-aligned
+constexpr uint32_t SX = 0;             // X, two column blocks of 128 rows x 128 B
+constexpr uint32_t SX_CB = 128 * 128;  // column-block stride of X
+constexpr uint32_t SAC = 2 * SX_CB;    // Ac, two column blocks of 64 rows x 128 B
+constexpr uint32_t STP = SAC + 64 * 256;  // [T; P], one column block of 128 rows x 128 B
+constexpr uint32_t SLOT_STRIDE = STP + 128 * 128;  // 65536
+// shared memory (bytes from a 1024-aligned base)
+constexpr uint32_t OFF_S = NSLOT * SLOT_STRIDE;  // state, fp16 copy (128 x VS)
+constexpr uint32_t OFF_WR = OFF_S + 128 * 128;   // write vectors (raw v lands here, swizzled)
+constexpr uint32_t OFF_GC = OFF_WR + 64 * 128;   // gamma_C of each slot, 128 fp32 each
+constexpr uint32_t OFF_GS = OFF_GC + NSLOT * 512;  // scalar gates of the next own chunk (alpha, beta_k)
+constexpr uint32_t OFF_END = OFF_GS + 128 * 4;
+constexpr size_t SMEM_BYTES = OFF_END + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(SLOT_STRIDE % 1024 == 0 && OFF_S % 1024 == 0 && OFF_WR % 1024 == 0, "tile alignment");
+// bytes one chunk's slot sends to the other CTA: Qh, -W (both column blocks), Ac, [T; P], gamma_C
+constexpr uint32_t SLOT_BYTES = 4 * 64 * 128 + 64 * 256 + 128 * 128 + 512;
+
+// TMEM columns
+constexpr uint32_t COL_D1 = 0;     // local: [A raw | P raw] (64)
+constexpr uint32_t COL_D2 = 64;    // local: W (128)
+constexpr uint32_t COL_U0 = 192;   // chain: U0 (64)
+constexpr uint32_t COL_D3 = 256;   // chain: [-W S | Qh S + P U] (64), even chunks
+constexpr uint32_t COL_D4 = 320;   // chain: Ac^T U (64)
+constexpr uint32_t COL_D3B = 384;  // chain: D3 of odd chunks (64)
+constexpr uint32_t TMEM_COLS = 512;
+
+__host__ __device__ constexpr uint32_t slot_off(int j) { return static_cast<uint32_t>(j) * SLOT_STRIDE; }
+__host__ __device__ constexpr uint32_t gc_off(int j) { return OFF_GC + static_cast<uint32_t>(j) * 512; }
+__host__ __device__ constexpr uint32_t col_d3(int c) { return (c & 1) ? COL_D3B : COL_D3; }
+
+__device__ __forceinline__ bool mbar_test_cluster(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// kChanGates: the gates vary per key channel (alpha per channel, or beta_k per channel); else
+// they are one value per row (alpha absent or per token, beta_k per token).
+template <typename IO, bool kChanGates>
+__global__ void __launch_bounds__(NT, 1)
+chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_qk, bar_lmma, bar_cmma, bar_v;
+  __shared__ uint64_t bar_full[NSLOT], bar_free[NSLOT], bar_land[NSLOT];
+  __shared__ uint32_t tmem_base_sh;
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase_addr = smem_u32(sm);
+
+  const int T = p.T, H = p.H, DV = p.DV;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rank = static_cast<int>(cluster_ctarank());  // value slice; equals blockIdx.x
+  const int peer = rank ^ 1;
+  const int v0 = rank * VS, h = blockIdx.y, b = blockIdx.z;
+  const int nchunks = (T + C - 1) / C;
+  const bool sym_channel = p.beta_v_mode == MODE_ABSENT && p.beta_k_mode == MODE_CHANNEL;
+  const bool scale_col = p.beta_v_mode == MODE_CHANNEL || sym_channel;  // per-column write scales
+
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar_qk, 1);
+    mbar_init(&bar_lmma, 1);
+    mbar_init(&bar_cmma, 1);
+    mbar_init(&bar_v, 1);
+    for (int j = 0; j < NSLOT; ++j) {
+      mbar_init(&bar_full[j], 1);
+      mbar_init(&bar_free[j], 2);  // both state passes
+      mbar_init(&bar_land[j], 1);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive or copy
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  // descriptors (K steps added per MMA)
+  auto kstep = [](uint64_t d, int R, int kk) -> uint64_t {
+    return d + static_cast<uint64_t>(((kk >> 2) * R * 128 + (kk & 3) * 32) >> 4);
+  };
+  auto mstep = [](uint64_t d, int kk) -> uint64_t { return d + static_cast<uint64_t>(kk * 128); };
+
+  if (tid < NL) {
+    // ================================================================== local role
+    const int ltid = tid;
+    uint32_t ph_qk = 0, ph_mma = 0;
+    uint32_t ph_free = 0;  // bit j: parity of the next wait on free[j] (ltid 0 only)
+    const int kp = ltid & 63, rgl = ltid >> 6, c0 = 2 * kp;
+    const int quarter = warp & 3, half = warp >> 2;  // warps 0..7
+    constexpr bool gates_scalar = !kChanGates;
+    float *sGate = reinterpret_cast<float *>(sm + OFF_GS);  // [0..63] alpha, [64..127] beta_k
+    float pal[2 * RGL], pbe[2 * RGL];                        // channel-gate K1: this thread's gates
+#pragma unroll
+    for (int i = 0; i < 2 * RGL; ++i) pal[i] = pbe[i] = 1.f;
+
+    auto issue_qk = [&](int c) {  // raw q and k of chunk c, in place into slot c % 3
+      const int t0 = c * C;
+      uint8_t *X = sm + slot_off(c % NSLOT);
+      mbar_arrive_expect_tx(&bar_qk, 4 * 64 * 128);
+      tma_load_4d(X + 64 * 128, &tm_q, &bar_qk, 0, h, t0, b);
+      tma_load_4d(X + SX_CB + 64 * 128, &tm_q, &bar_qk, 64, h, t0, b);
+      tma_load_4d(X, &tm_k, &bar_qk, 0, h, t0, b);
+      tma_load_4d(X + SX_CB, &tm_k, &bar_qk, 64, h, t0, b);
+    };
+    // gates of chunk c: scalar ones staged by cp.async (warp 0, lane l: rows 2l, 2l+1); channel
+    // ones into registers.  Loads only; masking and broadcast happen at use.
+    auto prefetch_gates = [&](int c) {
+      const int t0 = c * C, L = min(C, T - t0);
+      const size_t thb = (static_cast<size_t>(b) * T + t0) * H + h;
+      if constexpr (gates_scalar) {
+        if (warp == 0) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const size_t th = thb + static_cast<size_t>(min(2 * lane + e, L - 1)) * H;
+            if (p.alpha_mode == MODE_SCALAR) cp_async4(sGate + 2 * lane + e, p.alpha + th);
+            cp_async4(sGate + 64 + 2 * lane + e, p.beta_k + th);
+          }
+          cp_async_commit();
+        }
+      } else {
+#pragma unroll
+      for (int j = 0; j < RGL; ++j) {
+        const size_t th = thb + static_cast<size_t>(min(rgl * RGL + j, L - 1)) * H;
+        if (p.alpha_mode == MODE_CHANNEL) {
+          const float2 a = __ldg(reinterpret_cast<const float2 *>(p.alpha + th * DK + c0));
+          pal[2 * j] = a.x;
+          pal[2 * j + 1] = a.y;
+        } else if (p.alpha_mode == MODE_SCALAR) {
+          pal[2 * j] = __ldg(p.alpha + th);
+        }
+        if (p.beta_k_mode == MODE_CHANNEL) {
+          const float2 bt = __ldg(reinterpret_cast<const float2 *>(p.beta_k + th * DK + c0));
+          pbe[2 * j] = bt.x;
+          pbe[2 * j + 1] = bt.y;
+        } else {
+          pbe[2 * j] = __ldg(p.beta_k + th);
+        }
+      }
+      }
+    };
+    // TMA data: every thread waits; signals: one thread waits, the group barrier releases the others
+    auto wait_all = [&](uint64_t *bar, uint32_t &ph) -> bool {
+      const bool ok = mbar_wait(bar, ph & 1u, kWaitLimitNs);
+      ph++;
+      const bool fail = bar_or(BAR_LOCAL, NL, !ok);
+      if (fail && ltid == 0) raise_status(p.status, STATUS_TIMEOUT);
+      return !fail;
+    };
+    auto wait_one = [&](uint64_t *bar, uint32_t &ph) -> bool {
+      bool ok = true;
+      if (ltid == 0) ok = mbar_wait(bar, ph & 1u, kWaitLimitNs);
+      ph++;
+      const bool fail = bar_or(BAR_LOCAL, NL, !ok);
+      tc_fence_after();
+      if (fail && ltid == 0) raise_status(p.status, STATUS_TIMEOUT);
+      return !fail;
+    };
+
+    // the first own chunk uses a slot nobody has touched yet
+    auto prefetch_qk_l2 = [&](int c) {
+      for (int x = 0; x < DK; x += 64) {
+        tma_prefetch_l2_4d(&tm_q, x, h, c * C, b);
+        tma_prefetch_l2_4d(&tm_k, x, h, c * C, b);
+      }
+    };
+    if (rank < nchunks) {
+      if (ltid == 0) {
+        issue_qk(rank);
+        if (rank + 2 < nchunks) prefetch_qk_l2(rank + 2);
+      }
+      prefetch_gates(rank);
+    }
+    for (int c = rank; c < nchunks; c += 2) {
+      const int j = c % NSLOT, t0 = c * C, L = min(C, T - t0);
+      uint8_t *X = sm + slot_off(j);
+      uint8_t *tAC = X + SAC;
+      uint8_t *tTP = X + STP;
+      float *sGC = reinterpret_cast<float *>(sm + gc_off(j));
+      const uint32_t xaddr = sbase_addr + slot_off(j);
+      const uint32_t rbar = mapa_shared(smem_u32(&bar_full[j]), static_cast<uint32_t>(peer));
+      auto copy_part = [&](uint32_t off, uint32_t bytes) {  // offset from the smem base
+        bulk_copy_to_peer(mapa_shared(sbase_addr + off, static_cast<uint32_t>(peer)), sm + off, bytes, rbar);
+      };
+      if (ltid == 0 && c + 4 < nchunks) prefetch_qk_l2(c + 4);
+      if (!wait_all(&bar_qk, ph_qk)) break;
+
+      // -------------------------------------------------------------- K1: Qh, Bh (in place), Ac, gamma_C
+      if constexpr (gates_scalar) {
+        // row gates gamma_r (inclusive product), 1/gamma_r, sqrt(beta_r), kept in the TP tile
+        float *sRow = reinterpret_cast<float *>(tTP);
+        if (warp == 0) {
+          cp_async_wait_all();  // this lane's own staged rows
+          const float2 ga = *reinterpret_cast<const float2 *>(sGate + 2 * lane);
+          const float2 gb = *reinterpret_cast<const float2 *>(sGate + 64 + 2 * lane);
+          const bool asc = p.alpha_mode == MODE_SCALAR;
+          const float a0 = (asc && 2 * lane < L) ? ga.x : 1.f, a1 = (asc && 2 * lane + 1 < L) ? ga.y : 1.f;
+          const float b0 = (2 * lane < L) ? gb.x : 0.f, b1 = (2 * lane + 1 < L) ? gb.y : 0.f;
+          float incl = a0 * a1;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl *= y;
+          }
+          const float up = __shfl_up_sync(0xffffffffu, incl, 1);
+          const float ex = (lane == 0) ? 1.f : up;  // product of the rows before 2*lane
+          const float g0 = ex * a0, g1 = g0 * a1;
+          const float gC = __shfl_sync(0xffffffffu, incl, 31);
+          *reinterpret_cast<float2 *>(sRow + 2 * lane) = make_float2(g0, g1);
+          *reinterpret_cast<float2 *>(sRow + 64 + 2 * lane) = make_float2(__fdividef(1.f, g0), __fdividef(1.f, g1));
+          *reinterpret_cast<float2 *>(sRow + 128 + 2 * lane) = make_float2(tc::sqrt_fast(b0), tc::sqrt_fast(b1));
+          *reinterpret_cast<float4 *>(sGC + 4 * lane) = make_float4(gC, gC, gC, gC);
+          if (lane == 0 && !(gC >= kMinChunkDecayF16)) raise_status(p.status, STATUS_RANGE);
+        }
+        bar_sync(BAR_LOCAL, NL);
+        // elements: (row r, 8-column group j8), four per thread, 16-byte loads and stores
+        const int j8 = ltid & 15;
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = (ltid >> 4) + 16 * i;
+          const float g = sRow[r], gi = sRow[64 + r], sb = sRow[128 + r];
+          uint4 *pq = reinterpret_cast<uint4 *>(X + sw128_off16(64 + r, j8, 128));
+          uint4 *pk = reinterpret_cast<uint4 *>(X + sw128_off16(r, j8, 128));
+          const uint4 qraw = *pq, kraw = *pk;
+          const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qraw);
+          const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kraw);
+          uint32_t oq[4], ob[4], oa[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 qf = __bfloat1622float2(q2[e]), kf = __bfloat1622float2(k2[e]);
+            const float b0 = sb * kf.x, b1 = sb * kf.y;
+            const float x0 = b0 * gi, x1 = b1 * gi;
+            amax = fmaxf(amax, fmaxf(fabsf(x0), fabsf(x1)));
+            oq[e] = pack_f16x2(g * qf.x, g * qf.y);
+            ob[e] = pack_f16x2(g * b0, g * b1);
+            oa[e] = pack_f16x2(x0, x1);
+          }
+          *pq = make_uint4(oq[0], oq[1], oq[2], oq[3]);
+          *pk = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+          *reinterpret_cast<uint4 *>(tAC + sw128_off16(r, j8, 64)) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+        }
+        if (!(amax < kF16Max)) raise_status(p.status, STATUS_RANGE);
+      } else {
+        float *sPX = reinterpret_cast<float *>(tTP);  // row-group gate products, 4 x 128 fp32
+#pragma unroll
+        for (int jj = 0; jj < RGL; ++jj) {
+          const bool valid = rgl * RGL + jj < L;
+          if (p.alpha_mode != MODE_CHANNEL) pal[2 * jj + 1] = pal[2 * jj];
+          if (p.alpha_mode == MODE_ABSENT || !valid) pal[2 * jj] = pal[2 * jj + 1] = 1.f;
+          if (p.beta_k_mode != MODE_CHANNEL) pbe[2 * jj + 1] = pbe[2 * jj];
+          if (!valid) pbe[2 * jj] = pbe[2 * jj + 1] = 0.f;
+        }
+        float p0 = 1.f, p1 = 1.f;  // gate product of my row group
+#pragma unroll
+        for (int jj = 0; jj < RGL; ++jj) {
+          p0 *= pal[2 * jj];
+          p1 *= pal[2 * jj + 1];
+        }
+        *reinterpret_cast<float2 *>(sPX + rgl * 128 + c0) = make_float2(p0, p1);
+        bar_sync(BAR_LOCAL, NL);
+        float h0 = 1.f, h1 = 1.f, t0a = 1.f, t1a = 1.f;  // products of the groups before / after mine
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float2 x = *reinterpret_cast<const float2 *>(sPX + g * 128 + c0);
+          if (g < rgl) {
+            h0 *= x.x;
+            h1 *= x.y;
+          } else if (g > rgl) {
+            t0a *= x.x;
+            t1a *= x.y;
+          }
+        }
+        if (rgl == 0) {
+          const float g0 = h0 * p0 * t0a, g1 = h1 * p1 * t1a;
+          *reinterpret_cast<float2 *>(sGC + c0) = make_float2(g0, g1);
+          if (!(fminf(g0, g1) >= kMinChunkDecayF16)) raise_status(p.status, STATUS_RANGE);
+        }
+        const bool beta_scalar = p.beta_k_mode == MODE_SCALAR;
+        const uint32_t blk = static_cast<uint32_t>(kp >> 5), ch = static_cast<uint32_t>((kp & 31) >> 2);
+        const uint32_t inb = static_cast<uint32_t>((kp & 3) * 4);
+        uint8_t *pQ = X + blk * SX_CB + (64 + rgl * RGL) * 128 + inb;
+        uint8_t *pB = X + blk * SX_CB + (rgl * RGL) * 128 + inb;
+        uint8_t *pA = tAC + blk * 64 * 128 + (rgl * RGL) * 128 + inb;
+        float amax = 0.f;
+        float ga = h0, gb = h1;  // gamma_r of the current row, two key channels
+#pragma unroll
+        for (int jj = 0; jj < RGL; ++jj) {
+          const uint32_t sw = ((ch ^ static_cast<uint32_t>(jj & 7)) << 4) + jj * 128;
+          const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(pB + sw);  // raw k
+          const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(pQ + sw);  // raw q
+          const float2 kf = __bfloat1622float2(k2), qf = __bfloat1622float2(q2);
+          float s0, s1;
+          if (beta_scalar) {
+            s0 = s1 = tc::sqrt_fast(pbe[2 * jj]);
+          } else {
+            s0 = tc::sqrt_fast(pbe[2 * jj]);
+            s1 = tc::sqrt_fast(pbe[2 * jj + 1]);
+          }
+          ga *= pal[2 * jj];
+          gb *= pal[2 * jj + 1];
+          const float b0 = s0 * kf.x, b1 = s1 * kf.y;
+          const float a0 = b0 * __fdividef(1.f, ga), a1 = b1 * __fdividef(1.f, gb);  // b / gamma_r
+          amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
+          *reinterpret_cast<uint32_t *>(pQ + sw) = pack_f16x2(ga * qf.x, gb * qf.y);  // Qh (in place of q)
+          *reinterpret_cast<uint32_t *>(pB + sw) = pack_f16x2(ga * b0, gb * b1);      // Bh (in place of k)
+          *reinterpret_cast<uint32_t *>(pA + sw) = pack_f16x2(a0, a1);                // Ac
+        }
+        if (!(amax < kF16Max)) raise_status(p.status, STATUS_RANGE);
+      }
+      fence_async_smem();
+      bar_sync(BAR_LOCAL, NL);
+
+      // -------------------------------------------------------------- m1: D1 = [Bh; Qh] Ac^T
+      if (warp == 0) {
+        if (elect_one()) {
+          tc_fence_after();
+          const uint64_t dX = sdesc_sw128(xaddr + SX, 16, 1024);
+          const uint64_t dAcK = sdesc_sw128(xaddr + SAC, 16, 1024);
+          const uint32_t idesc = idesc_f16_f32(128, 64, false, false);
+#pragma unroll
+          for (int kk = 0; kk < DK / 16; ++kk)
+            umma_f16(tmem + COL_D1, kstep(dX, 128, kk), kstep(dAcK, 64, kk), idesc, kk > 0);
+          umma_commit(&bar_lmma);
+          // Qh, Ac and gamma_C are final: start moving them into the peer's slot.  The peer's
+          // full[j] phase completes on the copied bytes alone, so the arrive needs no release.
+          mbar_expect_tx_remote_relaxed(rbar, SLOT_BYTES);
+          copy_part(slot_off(j) + SX + 64 * 128, 64 * 128);
+          copy_part(slot_off(j) + SX + SX_CB + 64 * 128, 64 * 128);
+          copy_part(slot_off(j) + SAC, 64 * 256);
+          copy_part(gc_off(j), 512);
+        }
+        __syncwarp();
+      }
+      if (gates_scalar && c + 2 < nchunks) prefetch_gates(c + 2);
+      if (!wait_one(&bar_lmma, ph_mma)) break;
+
+      // -------------------------------------------------------------- E1a: A -> TP rows 0..63 (inverse input)
+      if (quarter < 2) {
+        const int r = quarter * 32 + lane;
+#pragma unroll 1
+        for (int jh = 0; jh < 32; jh += 16) {
+          float x[16];
+          const int col0 = half * 32 + jh;
+          tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D1 + col0), x);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) x[i] = (col0 + i < r) ? x[i] : 0.f;
+          tc::st_h16x16(tTP, r, col0, 128, x);
+        }
+      }
+      tc_fence_before();
+      bar_sync(BAR_LOCAL, NL);
+
+      // -------------------------------------------------------------- K2: T = (I + A)^-1 (warp MMAs)
+      {
+        tri::Frag Trow[4];
+        tri::inverse64_rows<tri::Sw128Layout>(tTP, tTP + 64 * 128, warp, lane, Trow,
+                                              [] { bar_sync(BAR_LOCAL, NL); });
+        if (warp < 4) {  // every read of A is done: T replaces it
+          const int rr = lane >> 2, qq = lane & 3;
+#pragma unroll
+          for (int d = 0; d < 4; ++d) {
+            if (d <= warp) {
+              const tri::Frag &F = Trow[d];
+              const int row = 16 * warp + rr, col = 16 * (warp - d) + 2 * qq;
+              *reinterpret_cast<uint32_t *>(tTP + sw128_off(row, col, 128)) = pack_f16x2(F.v[0], F.v[1]);
+              *reinterpret_cast<uint32_t *>(tTP + sw128_off(row + 8, col, 128)) = pack_f16x2(F.v[2], F.v[3]);
+              *reinterpret_cast<uint32_t *>(tTP + sw128_off(row, col + 8, 128)) = pack_f16x2(F.v[4], F.v[5]);
+              *reinterpret_cast<uint32_t *>(tTP + sw128_off(row + 8, col + 8, 128)) = pack_f16x2(F.v[6], F.v[7]);
+            }
+          }
+        }
+      }
+      fence_async_smem();
+      bar_sync(BAR_LOCAL, NL);
+
+      // -------------------------------------------------------------- m2: D2 = [T; .] Bh -> W at lanes 0..63
+      bool qk_next = false;  // ltid 0: raw q/k of chunk c+2 already requested
+      if (warp == 0) {
+        if (elect_one()) {
+          tc_fence_after();
+          const uint64_t dTP = sdesc_sw128(xaddr + STP, 16, 1024);
+          const uint64_t dBh = sdesc_sw128(xaddr + SX, SX_CB, 1024);
+          const uint32_t id2 = idesc_f16_f32(128, 128, false, true);
+#pragma unroll
+          for (int kk = 0; kk < C / 16; ++kk)
+            umma_f16(tmem + COL_D2, kstep(dTP, 128, kk), mstep(dBh, kk), id2, kk > 0);
+          umma_commit(&bar_lmma);
+        }
+        __syncwarp();
+      }
+      if (!gates_scalar && c + 2 < nchunks) prefetch_gates(c + 2);
+      // raw q/k of chunk c+2, if its slot is already free (else after the hand-off)
+      if (ltid == 0 && c + 2 < nchunks) {
+        const int jn = (c + 2) % NSLOT;
+        if (c + 2 < NSLOT) {
+          issue_qk(c + 2);
+          qk_next = true;
+        } else if (mbar_test_cluster(&bar_free[jn], (ph_free >> jn) & 1u)) {
+          ph_free ^= 1u << jn;
+          issue_qk(c + 2);
+          qk_next = true;
+        }
+      }
+      if (!wait_one(&bar_lmma, ph_mma)) break;
+
+      // -------------------------------------------------------------- E2: -W -> X rows 0..63;  E1b: P -> TP rows 64..127
+      if (quarter < 2) {
+        const int r = quarter * 32 + lane;
+#pragma unroll 1
+        for (int jw = 0; jw < 64; jw += 16) {
+          float x[16];
+          tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D2 + half * 64 + jw), x);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) x[i] = -x[i];
+          tc::st_h16x16(X, r, half * 64 + jw, 128, x);
+        }
+      } else {
+        const int r = (quarter - 2) * 32 + lane;
+#pragma unroll 1
+        for (int jh = 0; jh < 32; jh += 16) {
+          float x[16];
+          const int col0 = half * 32 + jh;
+          tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D1 + col0), x);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) x[i] = (col0 + i <= r) ? x[i] : 0.f;
+          tc::st_h16x16(tTP, 64 + r, col0, 128, x);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      bar_sync(BAR_LOCAL, NL);
+
+      // -------------------------------------------------------------- hand the slot to both state passes
+      if (ltid == 0) {
+        copy_part(slot_off(j) + SX, 64 * 128);
+        copy_part(slot_off(j) + SX + SX_CB, 64 * 128);
+        copy_part(slot_off(j) + STP, 128 * 128);
+        mbar_arrive(&bar_full[j]);
+        if (c + 2 < nchunks && !qk_next) {
+          const int jn = (c + 2) % NSLOT;
+          if (mbar_wait_cluster(&bar_free[jn], (ph_free >> jn) & 1u, kWaitLimitNs)) {
+            ph_free ^= 1u << jn;
+            issue_qk(c + 2);
+          } else {
+            raise_status(p.status, STATUS_TIMEOUT);  // the next wait for raw q/k then fails for all
+          }
+        }
+      }
+    }
+  } else {
+    // ================================================================== chain role
+    const int ct = tid - NL;
+    const int cw = warp - 8;
+    const int quarter = cw & 3, half = cw >> 2;
+    const int trow = quarter * 32 + lane;
+    uint32_t ph_v = 0, ph_mma = 0;
+    uint32_t ph_full = 0, ph_land = 0;  // bit j: parity of the next wait on full[j] / land[j]
+    bool aborted = false;
+    const size_t sbase = (static_cast<size_t>(b) * H + h) * DK * DV;
+    uint8_t *tS = sm + OFF_S;
+    uint8_t *tWR = sm + OFF_WR;
+    const int wc = ct >> 2, wjb = (ct & 3) * 2;  // write-vector row and its two 8-column groups
+
+    auto issue_v = [&](int c) {
+      mbar_arrive_expect_tx(&bar_v, 64 * 128);
+      tma_load_4d(tWR, &tm_v, &bar_v, v0, h, c * C, b);
+    };
+    // write scales of row wc of chunk c: one scalar (raw; square root at use if symmetric), or 16
+    // per-column values (beta_v, or beta_k of the same channels when the write is symmetric)
+    float pws = 0.f;
+    float psc[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) psc[i] = 0.f;
+    auto prefetch_ws = [&](int c) {
+      const int t0 = c * C, L = min(C, T - t0);
+      const size_t th = (static_cast<size_t>(b) * T + t0 + min(wc, L - 1)) * H + h;
+      if (scale_col) {
+        const float *src = (p.beta_v_mode == MODE_CHANNEL ? p.beta_v + th * DV : p.beta_k + th * DK) + v0 + wjb * 8;
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          const float4 x = __ldg(reinterpret_cast<const float4 *>(src + i));
+          psc[i] = x.x;
+          psc[i + 1] = x.y;
+          psc[i + 2] = x.z;
+          psc[i + 3] = x.w;
+        }
+      } else {
+        pws = __ldg((p.beta_v_mode == MODE_SCALAR ? p.beta_v : p.beta_k) + th);
+      }
+    };
+    // ph: phase bits, bit `bit` is this barrier's parity
+    auto wait_all = [&](uint64_t *bar, uint32_t &ph, int bit, bool cluster_scope) -> bool {
+      const uint32_t par = (ph >> bit) & 1u;
+      const bool ok = cluster_scope ? mbar_wait_cluster(bar, par, kWaitLimitNs) : mbar_wait(bar, par, kWaitLimitNs);
+      ph ^= 1u << bit;
+      const bool fail = bar_or(BAR_CHAIN, NT - NL, !ok);
+      if (fail && ct == 0) raise_status(p.status, STATUS_TIMEOUT);
+      return !fail;
+    };
+    auto wait_one = [&](uint64_t *bar, uint32_t &ph, int bit, bool cluster_scope) -> bool {
+      const uint32_t par = (ph >> bit) & 1u;
+      bool ok = true;
+      if (ct == 0)
+        ok = cluster_scope ? mbar_wait_cluster(bar, par, kWaitLimitNs) : mbar_wait(bar, par, kWaitLimitNs);
+      ph ^= 1u << bit;
+      const bool fail = bar_or(BAR_CHAIN, NT - NL, !ok);
+      tc_fence_after();
+      if (fail && ct == 0) raise_status(p.status, STATUS_TIMEOUT);
+      return !fail;
+    };
+    // write vectors of the chunk whose raw v sits in Wr, in place (after bar_v)
+    auto convert_wr = [&]() {
+      float sc[16];
+      if (scale_col) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sc[i] = sym_channel ? tc::sqrt_fast(psc[i]) : psc[i];
+      } else {
+        const float s0 = (p.beta_v_mode == MODE_SCALAR) ? pws : tc::sqrt_fast(pws);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sc[i] = s0;
+      }
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        uint4 *ptr = reinterpret_cast<uint4 *>(tWR + sw128_off16(wc, wjb + jj, 64));
+        const uint4 raw = *ptr;
+        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+        float w8[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 vf = __bfloat1622float2(v2[i]);
+          w8[2 * i] = sc[jj * 8 + 2 * i] * vf.x;  // rows >= L: v = 0 (TMA fill)
+          w8[2 * i + 1] = sc[jj * 8 + 2 * i + 1] * vf.y;
+        }
+        uint4 out;
+        out.x = pack_f16x2(w8[0], w8[1]);
+        out.y = pack_f16x2(w8[2], w8[3]);
+        out.z = pack_f16x2(w8[4], w8[5]);
+        out.w = pack_f16x2(w8[6], w8[7]);
+        *ptr = out;
+      }
+    };
+    // outputs of chunk c: lanes 64..127 of its D3 columns hold Qh S + P U
+    auto store_o = [&](int c) {
+      const int t0 = c * C, L = min(C, T - t0);
+      if (quarter >= 2) {
+        const int r = trow - 64;
+#pragma unroll 1
+        for (int j = 0; j < 32; j += 16) {
+          float x[16];
+          tmem_ld16(tmem_addr(tmem, quarter * 32, col_d3(c) + half * 32 + j), x);
+          tmem_ld_wait();
+          if (r < L) {
+            const size_t th = (static_cast<size_t>(b) * T + t0 + r) * H + h;
+            IO *dst = static_cast<IO *>(p.o) + th * DV + v0 + half * 32 + j;
+            uint4 lo, hi;
+            lo.x = pack_bf16x2(x[0], x[1]);
+            lo.y = pack_bf16x2(x[2], x[3]);
+            lo.z = pack_bf16x2(x[4], x[5]);
+            lo.w = pack_bf16x2(x[6], x[7]);
+            hi.x = pack_bf16x2(x[8], x[9]);
+            hi.y = pack_bf16x2(x[10], x[11]);
+            hi.z = pack_bf16x2(x[12], x[13]);
+            hi.w = pack_bf16x2(x[14], x[15]);
+            reinterpret_cast<uint4 *>(dst)[0] = lo;
+            reinterpret_cast<uint4 *>(dst)[1] = hi;
+          }
+        }
+      }
+    };
+
+    // fp32 state slice: row trow, columns half*32 .. half*32+31 of this CTA's value slice
+    float Sreg[32];
+    {
+      const float *src = p.S0 ? p.S0 + sbase + static_cast<size_t>(trow) * DV + v0 + half * 32 : nullptr;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const float4 x = src ? *reinterpret_cast<const float4 *>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        Sreg[j] = x.x;
+        Sreg[j + 1] = x.y;
+        Sreg[j + 2] = x.z;
+        Sreg[j + 3] = x.w;
+      }
+      tc::st_h16x16(tS, trow, half * 32, 128, Sreg);
+      tc::st_h16x16(tS, trow, half * 32 + 16, 128, Sreg + 16);
+    }
+    const uint64_t dS = sdesc_sw128(sbase_addr + OFF_S, 128 * 128, 1024);
+    const uint64_t dWr = sdesc_sw128(sbase_addr + OFF_WR, 64 * 128, 1024);
+
+    // Software pipeline: the write vectors of chunk c+1 are built while the second MMA group of
+    // chunk c runs, and the outputs of chunk c are stored while the first MMA group of chunk c+1
+    // runs (D3 alternates between two column sets).
+    if (nchunks > 0) {
+      if (ct == 0) {
+        issue_v(0);
+        for (int c = 1; c < 3 && c < nchunks; ++c) tma_prefetch_l2_4d(&tm_v, v0, h, c * C, b);
+      }
+      prefetch_ws(0);
+      if (wait_all(&bar_v, ph_v, 0, false)) {
+        convert_wr();
+      } else {
+        aborted = true;
+      }
+      fence_async_smem();
+      bar_sync(BAR_CHAIN, NT - NL);
+    }
+    for (int c = 0; c < nchunks && !aborted; ++c) {
+      const int j = c % NSLOT;
+      const bool producer = (c & 1) == rank;
+      const uint32_t xaddr = sbase_addr + slot_off(j);
+      const uint32_t cD3 = col_d3(c);
+      if (!wait_all(&bar_full[j], ph_full, j, true)) { aborted = true; break; }
+      // the other CTA's copies of this slot have all landed: its bulk reads are done
+      if (!producer && ct == 0)
+        mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&bar_land[j]), static_cast<uint32_t>(peer)));
+      const float gc = reinterpret_cast<const float *>(sm + gc_off(j))[trow];
+
+      // -------------------------------------------------------------- U0 = [T;P] Wr,  D3 = [-W; Qh] S
+      if (cw == 0) {
+        if (elect_one()) {
+          tc_fence_after();
+          const uint64_t dTP = sdesc_sw128(xaddr + STP, 16, 1024);
+          const uint64_t dX = sdesc_sw128(xaddr + SX, 16, 1024);
+          const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
+#pragma unroll
+          for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_U0, kstep(dTP, 128, kk), mstep(dWr, kk), id3, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < DK / 16; ++kk) umma_f16(tmem + cD3, kstep(dX, 128, kk), mstep(dS, kk), id3, kk > 0);
+          umma_commit(&bar_cmma);
+        }
+        __syncwarp();
+      }
+      if (c > 0) store_o(c - 1);
+      if (!wait_one(&bar_cmma, ph_mma, 0, false)) { aborted = true; break; }
+      if (ct == 0) {
+        if (c + 1 < nchunks) issue_v(c + 1);  // Wr is free
+        if (c + 3 < nchunks) tma_prefetch_l2_4d(&tm_v, v0, h, (c + 3) * C, b);
+      }
+      if (c + 1 < nchunks) prefetch_ws(c + 1);
+      // U goes into X rows 0..63 of this slot: in the producing CTA, only once the copies are read
+      if (producer && !wait_one(&bar_land[j], ph_land, j, false)) { aborted = true; break; }
+
+      // -------------------------------------------------------------- E3: U = U0 - W S -> X rows 0..63
+      uint8_t *tU = sm + slot_off(j) + SX;
+      if (quarter < 2) {
+#pragma unroll 1
+        for (int jj = 0; jj < 32; jj += 16) {
+          float ws[16], u0[16];
+          tmem_ld16(tmem_addr(tmem, quarter * 32, cD3 + half * 32 + jj), ws);
+          tmem_ld16(tmem_addr(tmem, quarter * 32, COL_U0 + half * 32 + jj), u0);
+          tmem_ld_wait();
+          float mx = 0.f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            u0[i] += ws[i];
+            mx = fmaxf(mx, fabsf(u0[i]));
+          }
+          if (!(mx < kF16Max)) raise_status(p.status, STATUS_RANGE);
+          tc::st_h16x16(tU, trow, half * 32 + jj, 128, u0);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      bar_sync(BAR_CHAIN, NT - NL);
+
+      // -------------------------------------------------------------- D4 = Ac^T U,  D3 += [T;P] U
+      if (cw == 0) {
+        if (elect_one()) {
+          tc_fence_after();
+          const uint64_t dAcM = sdesc_sw128(xaddr + SAC, 64 * 128, 1024);
+          const uint64_t dTP = sdesc_sw128(xaddr + STP, 16, 1024);
+          const uint64_t dU = sdesc_sw128(xaddr + SX, 128 * 128, 1024);
+          const uint32_t id4 = idesc_f16_f32(128, VS, true, true);
+          const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
+#pragma unroll
+          for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_D4, mstep(dAcM, kk), mstep(dU, kk), id4, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + cD3, kstep(dTP, 128, kk), mstep(dU, kk), id3, 1u);
+          umma_commit(&bar_cmma);
+        }
+        __syncwarp();
+      }
+      // write vectors of the next chunk while these MMAs run
+      if (c + 1 < nchunks) {
+        if (!wait_all(&bar_v, ph_v, 0, false)) { aborted = true; break; }
+        convert_wr();
+        fence_async_smem();
+      }
+      if (!wait_one(&bar_cmma, ph_mma, 0, false)) { aborted = true; break; }
+      // this CTA is done with slot j: tell the CTA that produces chunk c+3 into it
+      if (ct == 0) {
+        if (((c + 3) & 1) == rank) mbar_arrive(&bar_free[j]);
+        else mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&bar_free[j]), static_cast<uint32_t>(peer)));
+      }
+
+      // -------------------------------------------------------------- E4: S <- Diag(gamma_C) (S + Ac^T U)
+      {
+        float mx = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 32; jj += 16) {
+          float ds[16];
+          tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D4 + half * 32 + jj), ds);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            Sreg[jj + i] = gc * (Sreg[jj + i] + ds[i]);
+            mx = fmaxf(mx, fabsf(Sreg[jj + i]));
+          }
+          tc::st_h16x16(tS, trow, half * 32 + jj, 128, Sreg + jj);
+        }
+        if (!(mx < kF16Max)) raise_status(p.status, STATUS_RANGE);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      bar_sync(BAR_CHAIN, NT - NL);
+    }
+    if (!aborted && nchunks > 0) store_o(nchunks - 1);
+    if (!aborted && p.S_T) {
+      float *dst = p.S_T + sbase + static_cast<size_t>(trow) * DV + v0 + half * 32;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4 *>(dst + j) = make_float4(Sreg[j], Sreg[j + 1], Sreg[j + 2], Sreg[j + 3]);
+    }
+  }
+
+  // both roles done; keep this CTA's shared memory alive until the peer is done with it
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace tc3
+}  // namespace dr

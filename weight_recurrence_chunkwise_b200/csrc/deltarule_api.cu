@@ -14,23 +14,28 @@
 #include "chunk_simt.cuh"
 #include "chunk_tc.cuh"
 #include "chunk_tc2.cuh"
+#include "chunk_tc3.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "umma_selftest.cuh"
 
 namespace {
 
-constexpr size_t kWorkspaceBytes = 256;
+constexpr size_t kWorkspaceBytes = 256;  // status word, padded to an allocation granule
 
-// The two-CTA prefill is the default for dv = 128; DR_PREFILL_SINGLE_CTA=1 selects the
-// one-CTA-per-value-slice kernel instead (same results, used to compare the two).
-bool prefill_pair_enabled() {
-  static const bool on = [] {
-    const char *e = std::getenv("DR_PREFILL_SINGLE_CTA");
-    return !(e && e[0] == '1');
+// Tensor-core prefill kernel for dk = dv = 128, chunk 64: the two-CTA kernel with a three-slot
+// ring by default; DR_PREFILL_KERNEL=pair selects the two-slot two-CTA kernel and
+// DR_PREFILL_KERNEL=single the one-CTA-per-value-slice kernel (same results; for comparison).
+enum PrefillKernel { kRing, kPair, kSingle };
+PrefillKernel prefill_kernel() {
+  static const PrefillKernel k = [] {
+    const char *e = std::getenv("DR_PREFILL_KERNEL");
+    if (e && std::strcmp(e, "pair") == 0) return kPair;
+    if (e && std::strcmp(e, "single") == 0) return kSingle;
+    return kRing;
   }();
-  return on;
-}  // status word, padded to an allocation granule
+  return k;
+}
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -214,6 +219,43 @@ dr_status tc_pair_launch(const dr_problem *p, const void *q, const void *k, cons
   return launch_status();
 }
 
+dr_status tc_ring_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                         const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
+                         uint32_t *status, cudaStream_t st) {
+  using IO = __nv_bfloat16;
+  namespace tc = dr::tc;
+  namespace tc3 = dr::tc3;
+  alignas(64) CUtensorMap mq, mk, mv;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_map(&mq, bf, 2, q, p->B, p->T, p->H, p->dk, 64, tc::C, sw) ||
+      !make_map(&mk, bf, 2, k, p->B, p->T, p->H, p->dk, 64, tc::C, sw) ||
+      !make_map(&mv, bf, 2, v, p->B, p->T, p->H, p->dv, tc::VS, tc::C, sw))
+    return DR_ERR_CUDA;
+  tc::Params prm{p->T, p->H, p->dv, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v, p->beta_v_mode,
+                 S0, o, S_T, status};
+  const bool chan_gates = p->alpha_mode == DR_CHANNEL || p->beta_k_mode != DR_SCALAR;
+  auto kern = chan_gates ? tc3::chunk_fwd_ring_kernel<IO, true> : tc3::chunk_fwd_ring_kernel<IO, false>;
+  constexpr size_t smem = tc3::SMEM_BYTES;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return DR_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, p->H, p->B);
+  cfg.blockDim = dim3(tc3::NT, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, prm) != cudaSuccess) return DR_ERR_CUDA;
+  return launch_status();
+}
+
 // ----------------------------------------------------------------- decode
 template <typename IO, int DK, int DV>
 dr_status decode_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
@@ -282,8 +324,9 @@ dr_status dr_chunk_fwd(const dr_problem *p, const void *q, const void *k, const 
   }
   if (p->io_dtype == DR_F32)
     return simt_dispatch<float>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
-  if (p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv == 2 * dr::tc::VS && prefill_pair_enabled())
-    return tc_pair_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+  if (p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv == 2 * dr::tc::VS && prefill_kernel() != kSingle)
+    return prefill_kernel() == kPair ? tc_pair_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st)
+                                     : tc_ring_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
   if (p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv % dr::tc::VS == 0)
     return tc_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
   return simt_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);

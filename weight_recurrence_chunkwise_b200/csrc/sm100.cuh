@@ -54,8 +54,8 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 // Bounded wait for the phase with the given parity to complete: gives up
 // (returns false) once `limit_ns` of wall time has passed.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path kept out of line: every wait site shares one copy of the polling loop.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
 #pragma unroll 1
@@ -63,6 +63,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
       if (mbar_try_wait(bar, parity)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, limit_ns);
 }
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint64_t limit_ns);
 // Wall-time limit of every wait on an MMA or copy completion.
@@ -82,8 +85,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
   return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
+__device__ __noinline__ bool mbar_wait_cluster_slow(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
 #pragma unroll 1
@@ -91,6 +93,9 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
       if (mbar_try_wait_cluster(bar, parity)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+  return mbar_try_wait_cluster(bar, parity) || mbar_wait_cluster_slow(bar, parity, limit_ns);
 }
 
 // ------------------------------------------------------------------ clusters and DSMEM
@@ -112,6 +117,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t remote_bar
   asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(remote_bar),
                "r"(bytes)
                : "memory");
+}
+// Arrive on another CTA's barrier without release ordering: for a signal that carries no data of
+// this thread (e.g. "reads of your buffer are complete", known from an earlier acquire or MMA commit).
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
 // Same, without release ordering: for a barrier whose phase is completed by bulk-copy bytes only,
 // which carry their own visibility, so none of this thread's earlier writes need to be ordered.
@@ -174,6 +184,13 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
+}
+
+// Prefetch a 4-D tile into L2 (no shared memory, no completion signal).
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(map), "r"(c0),
+               "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
 }
 
 // ------------------------------------------------------------------ TMEM
