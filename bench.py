@@ -61,21 +61,41 @@ def decode_bytes(B, H, dk, dv, io=2, alpha_ch=True, beta_ch=True):
 
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the ncu captures
-# summarised under profiles/, each valid only for the kernel source it was taken on.
+# summarised under profiles/, each valid only for the kernel sources it was taken on: the key is
+# a digest of every file under csrc/ (see csrc_digest), so any source change voids the number.
 MEASURED_TRAFFIC = {
-    "chunk_fwd_tc_kernel": ("weight_recurrence_chunkwise_b200/csrc/chunk_tc.cuh", "fe02ddc59e95", 251.734272e6),
-    "decode_step_kernel": ("weight_recurrence_chunkwise_b200/csrc/decode.cuh", "f563c5e8b358", 1031.6032e6),
+    "decode_step_kernel": ("f563c5e8b358", 1031.6032e6, "decode.cuh"),
 }
+
+# Prefill kernel the library runs for dk = dv = 128, chunk 64 (DR_PREFILL_KERNEL selects it).
+PREFILL_KERNELS = {"ring": "chunk_fwd_ring_kernel", "pair": "chunk_fwd_pair_kernel", "single": "chunk_fwd_tc_kernel"}
+
+
+def prefill_kernel_name():
+    return PREFILL_KERNELS.get(os.environ.get("DR_PREFILL_KERNEL", "ring"), "chunk_fwd_ring_kernel")
+
+
+def csrc_digest(only=None):
+    """sha1 over the kernel sources (all of csrc/, or the one file `only`), in name order."""
+    import hashlib
+
+    d = os.path.join(ROOT, "weight_recurrence_chunkwise_b200", "csrc")
+    h = hashlib.sha1()
+    for name in sorted(os.listdir(d)):
+        if only is not None and name != only:
+            continue
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def measured_traffic(kernel):
-    """Bytes per launch from the committed ncu summary, or None once the kernel source changed."""
-    import hashlib
-
-    path, prefix, nbytes = MEASURED_TRAFFIC[kernel]
+    """Bytes per launch from the committed ncu summary, or None once the kernel sources changed."""
+    if kernel not in MEASURED_TRAFFIC:
+        return None
+    prefix, nbytes, only = MEASURED_TRAFFIC[kernel]
     try:
-        with open(os.path.join(ROOT, path), "rb") as f:
-            digest = hashlib.sha1(f.read()).hexdigest()
+        digest = csrc_digest(only)
     except OSError:
         return None
     return nbytes if digest.startswith(prefix) else None
@@ -329,9 +349,9 @@ def main():
     achieved_gbs = byts / (prefill_ms / 1e3) / 1e9
     t_roof_ms = max(byts / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops_sustained"] * 1e12)) * 1e3
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": measured_traffic("chunk_fwd_tc_kernel"),
+                "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": measured_traffic(prefill_kernel_name()),
                 "peak_source": peaks_src,
-                "kernel": "chunk_fwd_tc_kernel", "algorithmic_bytes_per_launch": byts,
+                "kernel": prefill_kernel_name(), "algorithmic_bytes_per_launch": byts,
                 "algorithmic_flops_per_launch": flops,
                 "tensor_tflops_achieved": flops / (prefill_ms / 1e3) / 1e12,
                 "roofline_time_ms": t_roof_ms, "frac_of_max_roofline": t_roof_ms / prefill_ms}

@@ -60,7 +60,8 @@ constexpr uint32_t OFF_S = NSLOT * SLOT_STRIDE;  // state, fp16 copy (128 x VS)
 constexpr uint32_t OFF_WR = OFF_S + 128 * 128;   // write vectors (raw v lands here, swizzled)
 constexpr uint32_t OFF_GC = OFF_WR + 64 * 128;   // gamma_C of each slot, 128 fp32 each
 constexpr uint32_t OFF_GS = OFF_GC + NSLOT * 512;  // scalar gates of the next own chunk (alpha, beta_k)
-constexpr uint32_t OFF_END = OFF_GS + 128 * 4;
+constexpr uint32_t OFF_ROW = OFF_GS + 128 * 4;     // its row gates: gamma, 1/gamma, sqrt(beta_k), gamma_C
+constexpr uint32_t OFF_END = OFF_ROW + 256 * 4;
 constexpr size_t SMEM_BYTES = OFF_END + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(SLOT_STRIDE % 1024 == 0 && OFF_S % 1024 == 0 && OFF_WR % 1024 == 0, "tile alignment");
@@ -149,7 +150,10 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // ================================================================== local role
     const int ltid = tid;
     uint32_t ph_qk = 0, ph_mma = 0;
-    uint32_t ph_free = 0;  // bit j: parity of the next wait on free[j] (ltid 0 only)
+    // Single-thread work is spread over two warps: warp 0 issues the MMAs; ltid 128 (warp 4) issues
+    // the TMA loads, L2 prefetches and DSMEM copies and tracks the free[] phases.
+    constexpr int kIo = 128;
+    uint32_t ph_free = 0;  // bit j: parity of the next wait on free[j] (ltid kIo only)
     const int kp = ltid & 63, rgl = ltid >> 6, c0 = 2 * kp;
     const int quarter = warp & 3, half = warp >> 2;  // warps 0..7
     constexpr bool gates_scalar = !kChanGates;
@@ -167,8 +171,10 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       tma_load_4d(X, &tm_k, &bar_qk, 0, h, t0, b);
       tma_load_4d(X + SX_CB, &tm_k, &bar_qk, 64, h, t0, b);
     };
-    // gates of chunk c: scalar ones staged by cp.async (warp 0, lane l: rows 2l, 2l+1); channel
-    // ones into registers.  Loads only; masking and broadcast happen at use.
+    // gates of chunk c.  Scalar: staged by cp.async (warp 0, lane l: rows 2l, 2l+1), one own chunk
+    // ahead.  Channel: L2 prefetch one own chunk ahead (prefetch_gates), then loaded into registers
+    // at the top of the chunk's iteration (load_gates), so they are live only until K1.
+    // Loads only; masking and broadcast happen at use.
     auto prefetch_gates = [&](int c) {
       const int t0 = c * C, L = min(C, T - t0);
       const size_t thb = (static_cast<size_t>(b) * T + t0) * H + h;
@@ -183,6 +189,16 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           cp_async_commit();
         }
       } else {
+        // thread ltid: 128-byte line (ltid & 3) of row (ltid >> 2) of each channel-wise gate
+        const size_t th = thb + static_cast<size_t>(min(ltid >> 2, L - 1)) * H;
+        const size_t off = th * DK + (ltid & 3) * 32;
+        if (p.alpha_mode == MODE_CHANNEL) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.alpha + off));
+        if (p.beta_k_mode == MODE_CHANNEL) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.beta_k + off));
+      }
+    };
+    auto load_gates = [&](int c) {  // channel-gate K1 only
+      const int t0 = c * C, L = min(C, T - t0);
+      const size_t thb = (static_cast<size_t>(b) * T + t0) * H + h;
 #pragma unroll
       for (int j = 0; j < RGL; ++j) {
         const size_t th = thb + static_cast<size_t>(min(rgl * RGL + j, L - 1)) * H;
@@ -201,7 +217,32 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           pbe[2 * j] = __ldg(p.beta_k + th);
         }
       }
+    };
+    // Scalar gates, warp 0: the row gates of own chunk c from its staged alpha, beta_k -- gamma_r
+    // (inclusive product), 1/gamma_r, sqrt(beta_r) and gamma_C -- done one own chunk ahead, so that
+    // K1 starts on the elements at once.
+    float *sRow = reinterpret_cast<float *>(sm + OFF_ROW);
+    auto scan_gates = [&](int c) {
+      const int L = min(C, T - c * C);
+      cp_async_wait_all();  // this lane's own staged rows
+      const float2 ga = *reinterpret_cast<const float2 *>(sGate + 2 * lane);
+      const float2 gb = *reinterpret_cast<const float2 *>(sGate + 64 + 2 * lane);
+      const bool asc = p.alpha_mode == MODE_SCALAR;
+      const float a0 = (asc && 2 * lane < L) ? ga.x : 1.f, a1 = (asc && 2 * lane + 1 < L) ? ga.y : 1.f;
+      const float b0 = (2 * lane < L) ? gb.x : 0.f, b1 = (2 * lane + 1 < L) ? gb.y : 0.f;
+      float incl = a0 * a1;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl *= y;
       }
+      const float up = __shfl_up_sync(0xffffffffu, incl, 1);
+      const float ex = (lane == 0) ? 1.f : up;  // product of the rows before 2*lane
+      const float g0 = ex * a0, g1 = g0 * a1;
+      *reinterpret_cast<float2 *>(sRow + 2 * lane) = make_float2(g0, g1);
+      *reinterpret_cast<float2 *>(sRow + 64 + 2 * lane) = make_float2(__fdividef(1.f, g0), __fdividef(1.f, g1));
+      *reinterpret_cast<float2 *>(sRow + 128 + 2 * lane) = make_float2(tc::sqrt_fast(b0), tc::sqrt_fast(b1));
+      if (lane == 31) sRow[192] = incl;
     };
     // TMA data: every thread waits; signals: one thread waits, the group barrier releases the others
     auto wait_all = [&](uint64_t *bar, uint32_t &ph) -> bool {
@@ -229,11 +270,14 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       }
     };
     if (rank < nchunks) {
-      if (ltid == 0) {
+      if (ltid == kIo) {
         issue_qk(rank);
         if (rank + 2 < nchunks) prefetch_qk_l2(rank + 2);
       }
       prefetch_gates(rank);
+      if constexpr (gates_scalar) {
+        if (warp == 0) scan_gates(rank);
+      }
     }
     for (int c = rank; c < nchunks; c += 2) {
       const int j = c % NSLOT, t0 = c * C, L = min(C, T - t0);
@@ -246,41 +290,22 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       auto copy_part = [&](uint32_t off, uint32_t bytes) {  // offset from the smem base
         bulk_copy_to_peer(mapa_shared(sbase_addr + off, static_cast<uint32_t>(peer)), sm + off, bytes, rbar);
       };
-      if (ltid == 0 && c + 4 < nchunks) prefetch_qk_l2(c + 4);
+      if (ltid == kIo && c + 4 < nchunks) prefetch_qk_l2(c + 4);
+      if constexpr (!gates_scalar) load_gates(c);
       if (!wait_all(&bar_qk, ph_qk)) break;
 
       // -------------------------------------------------------------- K1: Qh, Bh (in place), Ac, gamma_C
       if constexpr (gates_scalar) {
-        // row gates gamma_r (inclusive product), 1/gamma_r, sqrt(beta_r), kept in the TP tile
-        float *sRow = reinterpret_cast<float *>(tTP);
+        // row gates: computed by scan_gates at the end of the previous own chunk (or before the loop)
         if (warp == 0) {
-          cp_async_wait_all();  // this lane's own staged rows
-          const float2 ga = *reinterpret_cast<const float2 *>(sGate + 2 * lane);
-          const float2 gb = *reinterpret_cast<const float2 *>(sGate + 64 + 2 * lane);
-          const bool asc = p.alpha_mode == MODE_SCALAR;
-          const float a0 = (asc && 2 * lane < L) ? ga.x : 1.f, a1 = (asc && 2 * lane + 1 < L) ? ga.y : 1.f;
-          const float b0 = (2 * lane < L) ? gb.x : 0.f, b1 = (2 * lane + 1 < L) ? gb.y : 0.f;
-          float incl = a0 * a1;
-#pragma unroll
-          for (int off = 1; off < 32; off <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl *= y;
-          }
-          const float up = __shfl_up_sync(0xffffffffu, incl, 1);
-          const float ex = (lane == 0) ? 1.f : up;  // product of the rows before 2*lane
-          const float g0 = ex * a0, g1 = g0 * a1;
-          const float gC = __shfl_sync(0xffffffffu, incl, 31);
-          *reinterpret_cast<float2 *>(sRow + 2 * lane) = make_float2(g0, g1);
-          *reinterpret_cast<float2 *>(sRow + 64 + 2 * lane) = make_float2(__fdividef(1.f, g0), __fdividef(1.f, g1));
-          *reinterpret_cast<float2 *>(sRow + 128 + 2 * lane) = make_float2(tc::sqrt_fast(b0), tc::sqrt_fast(b1));
+          const float gC = sRow[192];
           *reinterpret_cast<float4 *>(sGC + 4 * lane) = make_float4(gC, gC, gC, gC);
           if (lane == 0 && !(gC >= kMinChunkDecayF16)) raise_status(p.status, STATUS_RANGE);
         }
-        bar_sync(BAR_LOCAL, NL);
         // elements: (row r, 8-column group j8), four per thread, 16-byte loads and stores
         const int j8 = ltid & 15;
         float amax = 0.f;
-#pragma unroll
+#pragma unroll 1
         for (int i = 0; i < 4; ++i) {
           const int r = (ltid >> 4) + 16 * i;
           const float g = sRow[r], gi = sRow[64 + r], sb = sRow[128 + r];
@@ -382,19 +407,20 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           const uint64_t dX = sdesc_sw128(xaddr + SX, 16, 1024);
           const uint64_t dAcK = sdesc_sw128(xaddr + SAC, 16, 1024);
           const uint32_t idesc = idesc_f16_f32(128, 64, false, false);
-#pragma unroll
+#pragma unroll 1
           for (int kk = 0; kk < DK / 16; ++kk)
             umma_f16(tmem + COL_D1, kstep(dX, 128, kk), kstep(dAcK, 64, kk), idesc, kk > 0);
           umma_commit(&bar_lmma);
-          // Qh, Ac and gamma_C are final: start moving them into the peer's slot.  The peer's
-          // full[j] phase completes on the copied bytes alone, so the arrive needs no release.
-          mbar_expect_tx_remote_relaxed(rbar, SLOT_BYTES);
-          copy_part(slot_off(j) + SX + 64 * 128, 64 * 128);
-          copy_part(slot_off(j) + SX + SX_CB + 64 * 128, 64 * 128);
-          copy_part(slot_off(j) + SAC, 64 * 256);
-          copy_part(gc_off(j), 512);
         }
         __syncwarp();
+      } else if (ltid == kIo) {
+        // Qh, Ac and gamma_C are final: start moving them into the peer's slot.  The peer's
+        // full[j] phase completes on the copied bytes alone, so the arrive needs no release.
+        mbar_expect_tx_remote_relaxed(rbar, SLOT_BYTES);
+        copy_part(slot_off(j) + SX + 64 * 128, 64 * 128);
+        copy_part(slot_off(j) + SX + SX_CB + 64 * 128, 64 * 128);
+        copy_part(slot_off(j) + SAC, 64 * 256);
+        copy_part(gc_off(j), 512);
       }
       if (gates_scalar && c + 2 < nchunks) prefetch_gates(c + 2);
       if (!wait_one(&bar_lmma, ph_mma)) break;
@@ -440,14 +466,14 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       bar_sync(BAR_LOCAL, NL);
 
       // -------------------------------------------------------------- m2: D2 = [T; .] Bh -> W at lanes 0..63
-      bool qk_next = false;  // ltid 0: raw q/k of chunk c+2 already requested
+      bool qk_next = false;  // ltid kIo: raw q/k of chunk c+2 already requested
       if (warp == 0) {
         if (elect_one()) {
           tc_fence_after();
           const uint64_t dTP = sdesc_sw128(xaddr + STP, 16, 1024);
           const uint64_t dBh = sdesc_sw128(xaddr + SX, SX_CB, 1024);
           const uint32_t id2 = idesc_f16_f32(128, 128, false, true);
-#pragma unroll
+#pragma unroll 1
           for (int kk = 0; kk < C / 16; ++kk)
             umma_f16(tmem + COL_D2, kstep(dTP, 128, kk), mstep(dBh, kk), id2, kk > 0);
           umma_commit(&bar_lmma);
@@ -456,7 +482,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       }
       if (!gates_scalar && c + 2 < nchunks) prefetch_gates(c + 2);
       // raw q/k of chunk c+2, if its slot is already free (else after the hand-off)
-      if (ltid == 0 && c + 2 < nchunks) {
+      if (ltid == kIo && c + 2 < nchunks) {
         const int jn = (c + 2) % NSLOT;
         if (c + 2 < NSLOT) {
           issue_qk(c + 2);
@@ -499,7 +525,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       bar_sync(BAR_LOCAL, NL);
 
       // -------------------------------------------------------------- hand the slot to both state passes
-      if (ltid == 0) {
+      if (ltid == kIo) {
         copy_part(slot_off(j) + SX, 64 * 128);
         copy_part(slot_off(j) + SX + SX_CB, 64 * 128);
         copy_part(slot_off(j) + STP, 128 * 128);
@@ -513,6 +539,9 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             raise_status(p.status, STATUS_TIMEOUT);  // the next wait for raw q/k then fails for all
           }
         }
+      }
+      if constexpr (gates_scalar) {
+        if (warp == 0 && c + 2 < nchunks) scan_gates(c + 2);
       }
     }
   } else {
@@ -654,52 +683,57 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint64_t dS = sdesc_sw128(sbase_addr + OFF_S, 128 * 128, 1024);
     const uint64_t dWr = sdesc_sw128(sbase_addr + OFF_WR, 64 * 128, 1024);
 
-    // Software pipeline: the write vectors of chunk c+1 are built while the second MMA group of
-    // chunk c runs, and the outputs of chunk c are stored while the first MMA group of chunk c+1
-    // runs (D3 alternates between two column sets).
+    // Software pipeline: the write vectors of chunk c+1 are built at the end of chunk c (their v is
+    // requested as soon as the first MMA group of chunk c has read Wr), and the outputs of chunk c
+    // are stored while the first MMA group of chunk c+1 runs (D3 alternates between two column sets).
     if (nchunks > 0) {
       if (ct == 0) {
         issue_v(0);
         for (int c = 1; c < 3 && c < nchunks; ++c) tma_prefetch_l2_4d(&tm_v, v0, h, c * C, b);
       }
       prefetch_ws(0);
-      if (wait_all(&bar_v, ph_v, 0, false)) {
-        convert_wr();
-      } else {
-        aborted = true;
-      }
-      fence_async_smem();
-      bar_sync(BAR_CHAIN, NT - NL);
     }
-    for (int c = 0; c < nchunks && !aborted; ++c) {
+    // iteration c builds the write vectors of chunk c and runs its state pass; the extra last
+    // iteration only stores the outputs of the final chunk
+    for (int c = 0; c <= nchunks && !aborted; ++c) {
+      const bool run = c < nchunks;
       const int j = c % NSLOT;
       const bool producer = (c & 1) == rank;
       const uint32_t xaddr = sbase_addr + slot_off(j);
       const uint32_t cD3 = col_d3(c);
-      if (!wait_all(&bar_full[j], ph_full, j, true)) { aborted = true; break; }
-      // the other CTA's copies of this slot have all landed: its bulk reads are done
-      if (!producer && ct == 0)
-        mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&bar_land[j]), static_cast<uint32_t>(peer)));
-      const float gc = reinterpret_cast<const float *>(sm + gc_off(j))[trow];
+      float gc = 0.f;
+      if (run) {
+        if (!wait_all(&bar_v, ph_v, 0, false)) { aborted = true; break; }
+        convert_wr();
+        fence_async_smem();
+        if (!wait_all(&bar_full[j], ph_full, j, true)) { aborted = true; break; }
+        // the other CTA's copies of this slot have all landed: its bulk reads are done
+        if (!producer && ct == 128)
+          mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&bar_land[j]), static_cast<uint32_t>(peer)));
+        gc = reinterpret_cast<const float *>(sm + gc_off(j))[trow];
 
-      // -------------------------------------------------------------- U0 = [T;P] Wr,  D3 = [-W; Qh] S
-      if (cw == 0) {
-        if (elect_one()) {
-          tc_fence_after();
-          const uint64_t dTP = sdesc_sw128(xaddr + STP, 16, 1024);
-          const uint64_t dX = sdesc_sw128(xaddr + SX, 16, 1024);
-          const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
-#pragma unroll
-          for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_U0, kstep(dTP, 128, kk), mstep(dWr, kk), id3, kk > 0);
-#pragma unroll
-          for (int kk = 0; kk < DK / 16; ++kk) umma_f16(tmem + cD3, kstep(dX, 128, kk), mstep(dS, kk), id3, kk > 0);
-          umma_commit(&bar_cmma);
+        // ------------------------------------------------------------ U0 = [T;P] Wr,  D3 = [-W; Qh] S
+        if (cw == 0) {
+          if (elect_one()) {
+            tc_fence_after();
+            const uint64_t dTP = sdesc_sw128(xaddr + STP, 16, 1024);
+            const uint64_t dX = sdesc_sw128(xaddr + SX, 16, 1024);
+            const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
+#pragma unroll 1
+            for (int kk = 0; kk < C / 16; ++kk)
+              umma_f16(tmem + COL_U0, kstep(dTP, 128, kk), mstep(dWr, kk), id3, kk > 0);
+#pragma unroll 1
+            for (int kk = 0; kk < DK / 16; ++kk)
+              umma_f16(tmem + cD3, kstep(dX, 128, kk), mstep(dS, kk), id3, kk > 0);
+            umma_commit(&bar_cmma);
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
-      if (c > 0) store_o(c - 1);
+      if (c > 0) store_o(c - 1);  // overlaps the MMAs above
+      if (!run) break;
       if (!wait_one(&bar_cmma, ph_mma, 0, false)) { aborted = true; break; }
-      if (ct == 0) {
+      if (ct == 128) {
         if (c + 1 < nchunks) issue_v(c + 1);  // Wr is free
         if (c + 3 < nchunks) tma_prefetch_l2_4d(&tm_v, v0, h, (c + 3) * C, b);
       }
@@ -739,23 +773,17 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           const uint64_t dU = sdesc_sw128(xaddr + SX, 128 * 128, 1024);
           const uint32_t id4 = idesc_f16_f32(128, VS, true, true);
           const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
-#pragma unroll
+#pragma unroll 1
           for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_D4, mstep(dAcM, kk), mstep(dU, kk), id4, kk > 0);
-#pragma unroll
+#pragma unroll 1
           for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + cD3, kstep(dTP, 128, kk), mstep(dU, kk), id3, 1u);
           umma_commit(&bar_cmma);
         }
         __syncwarp();
       }
-      // write vectors of the next chunk while these MMAs run
-      if (c + 1 < nchunks) {
-        if (!wait_all(&bar_v, ph_v, 0, false)) { aborted = true; break; }
-        convert_wr();
-        fence_async_smem();
-      }
       if (!wait_one(&bar_cmma, ph_mma, 0, false)) { aborted = true; break; }
       // this CTA is done with slot j: tell the CTA that produces chunk c+3 into it
-      if (ct == 0) {
+      if (ct == 128) {
         if (((c + 3) & 1) == rank) mbar_arrive(&bar_free[j]);
         else mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&bar_free[j]), static_cast<uint32_t>(peer)));
       }
@@ -781,7 +809,6 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       tc_fence_before();
       bar_sync(BAR_CHAIN, NT - NL);
     }
-    if (!aborted && nchunks > 0) store_o(nchunks - 1);
     if (!aborted && p.S_T) {
       float *dst = p.S_T + sbase + static_cast<size_t>(trow) * DV + v0 + half * 32;
 #pragma unroll

@@ -236,35 +236,45 @@ __device__ __forceinline__ void inverse64_rows(const uint8_t *Ah, uint8_t *ThT, 
                                                Sync sync) {
   if (warp < 4) {
     const int b = warp;
-    const Frag N = load_frag_l<Lay>(Ah, b, b, lane);
-    const Frag Nt = load_frag_t_l<Lay>(Ah, b, b, lane);
-    const Frag N2 = mul(N, Nt), N2t = mul(Nt, N);
-    const Frag N4 = mul(N2, N2t), N4t = mul(N2t, N2);
-    const Frag N8t = mul(N4t, N4);
-    const Frag X1 = eye_plus(N, -1.f, lane);
-    const Frag Y1t = eye_plus(N2t, 1.f, lane);
-    const Frag P1 = mul(X1, Y1t);
-    const Frag Y2t = eye_plus(N4t, 1.f, lane);
-    const Frag P2 = mul(P1, Y2t);
-    const Frag Y3t = eye_plus(N8t, 1.f, lane);
-    Trow[0] = mul(P2, Y3t);
-    store_frag_l<Lay>(ThT, b, b, mul(Y3t, P2), lane);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) Trow[1].v[e] = Trow[2].v[e] = Trow[3].v[e] = 0.f;
+    // (I + N)^-1 = (I - N)(I + N^2)(I + N^4)(I + N^8): P <- P (I + M), M <- M^2, as a loop
+    Frag M = load_frag_l<Lay>(Ah, b, b, lane);
+    Frag Mt = load_frag_t_l<Lay>(Ah, b, b, lane);
+    Frag P = eye_plus(M, -1.f, lane), Yt;
+#pragma unroll 1
+    for (int k = 0; k < 3; ++k) {
+      const Frag M2 = mul(M, Mt);
+      Mt = mul(Mt, M);
+      M = M2;
+      Yt = eye_plus(Mt, 1.f, lane);
+      if (k < 2) P = mul(P, Yt);
+    }
+    Trow[0] = mul(P, Yt);
+    store_frag_l<Lay>(ThT, b, b, mul(Yt, P), lane);
   }
   sync();
-#pragma unroll
+  // one copy of the level code: the result goes to Trow[d] through a select, not an indexed store
+#pragma unroll 1
   for (int d = 1; d < 4; ++d) {
     if (warp >= d && warp < 4) {
       const int i = warp, j = warp - d;
       Frag Xt;  // X^T for X = sum_m A_im T_mj
 #pragma unroll
       for (int e = 0; e < 8; ++e) Xt.v[e] = 0.f;
+#pragma unroll 1
       for (int m = j; m < i; ++m) mul_acc(Xt, load_frag_l<Lay>(ThT, j, m, lane), load_frag_l<Lay>(Ah, i, m, lane));
       Frag Tij = mul(Trow[0], Xt);
       Frag Tijt = mul(Xt, Trow[0]);
       negate(Tij);
       negate(Tijt);
       store_frag_l<Lay>(ThT, j, i, Tijt, lane);
-      Trow[d] = Tij;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        Trow[1].v[e] = (d == 1) ? Tij.v[e] : Trow[1].v[e];
+        Trow[2].v[e] = (d == 2) ? Tij.v[e] : Trow[2].v[e];
+        Trow[3].v[e] = (d == 3) ? Tij.v[e] : Trow[3].v[e];
+      }
     }
     sync();
   }
