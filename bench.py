@@ -64,6 +64,7 @@ def decode_bytes(B, H, dk, dv, io=2, alpha_ch=True, beta_ch=True):
 # summarised under profiles/, each valid only for the kernel sources it was taken on: the key is
 # a digest of every file under csrc/ (see csrc_digest), so any source change voids the number.
 MEASURED_TRAFFIC = {
+    "chunk_fwd_ring_kernel": ("5946d073e482", 248.945664e6, None),
     "decode_step_kernel": ("f563c5e8b358", 1031.6032e6, "decode.cuh"),
 }
 
@@ -182,9 +183,9 @@ def barrier(ws):
         dist.barrier()
 
 
-def rank_problem(rank):
+def rank_problem(rank, workload=WORKLOAD):
     """The workload a rank runs: same shape, its own seed (heads are independent, no exchange)."""
-    base = CONFIGS[WORKLOAD]
+    base = CONFIGS[workload]
     return base.replace(seed=base.seed + 1000 * rank)
 
 
@@ -277,6 +278,8 @@ def main():
                     help="profiling aid: time only the prefill step (no decode workload, e2e or CPU leg)")
     ap.add_argument("--only-decode", action="store_true",
                     help="profiling aid: time only the decode workload")
+    ap.add_argument("--config", default=WORKLOAD, choices=list(CONFIGS),
+                    help="with --only-prefill: the prefill workload to time (default: the headline one)")
     args = ap.parse_args()
     ws, rank, local = dist_env()
     if args.impl == "reference":
@@ -295,7 +298,7 @@ def main():
     st = torch.cuda.current_stream()
 
     # ---------------- prefill -> decode step workload (every rank its own seeded batch)
-    p = rank_problem(rank)
+    p = rank_problem(rank, args.config if args.only_prefill else WORKLOAD)
     x = to_dev(make_inputs(p), dev)
     nxt = to_dev(make_inputs(p.replace(T=1, seed=p.seed + 500)), dev)  # the token after the prompt
     o = torch.empty_like(x["v"])
@@ -308,7 +311,8 @@ def main():
     def step():
         dr.dr_chunk_fwd(x["q"], x["k"], x["v"], x["beta_k"], alpha=x["alpha"], beta_v=x["beta_v"], S0=None,
                         chunk=p.chunk, o=o, S_T=S, workspace=ws_buf, stream=st)
-        dr.dr_decode_step(nxt["q"], nxt["k"], nxt["v"], nxt["beta_k"], S, alpha=nxt["alpha"], o=o1, stream=st)
+        if not args.only_prefill:
+            dr.dr_decode_step(nxt["q"], nxt["k"], nxt["v"], nxt["beta_k"], S, alpha=nxt["alpha"], o=o1, stream=st)
 
     if args.only_decode:
         return run_decode_only(args, dr, dev, st, ws)
@@ -331,7 +335,9 @@ def main():
             dr.dr_chunk_fwd(x["q"], x["k"], x["v"], x["beta_k"], alpha=x["alpha"], beta_v=x["beta_v"], S0=None,
                             chunk=p.chunk, o=o, S_T=S, workspace=ws_buf, stream=st)
             ev[i][1].record(st)
-            dr.dr_decode_step(nxt["q"], nxt["k"], nxt["v"], nxt["beta_k"], S, alpha=nxt["alpha"], o=o1, stream=st)
+            if not args.only_prefill:
+                dr.dr_decode_step(nxt["q"], nxt["k"], nxt["v"], nxt["beta_k"], S, alpha=nxt["alpha"], o=o1,
+                                  stream=st)
             ev[i][2].record(st)
         t_end.record(st)
         torch.cuda.synchronize()
