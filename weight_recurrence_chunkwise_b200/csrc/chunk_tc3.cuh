@@ -45,7 +45,7 @@ using tc::Params;
 
 constexpr int NT = 512;  // threads
 constexpr int NL = 256;  // local role: threads 0..255
-constexpr int BAR_LOCAL = 1, BAR_CHAIN = 2;
+constexpr int BAR_LOCAL = 1, BAR_CHAIN = 2, BAR_INV = 3;  // BAR_INV: warps 0..3 in the UT inverse
 constexpr int RGL = 16;  // rows per local elementwise thread in the channel-gate K1
 constexpr int NSLOT = 3;
 
@@ -444,10 +444,11 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
       // -------------------------------------------------------------- K2: T = (I + A)^-1 (warp MMAs)
       {
-        tri::Frag Trow[4];
-        tri::inverse64_rows<tri::Sw128Layout>(tTP, tTP + 64 * 128, warp, lane, Trow,
-                                              [] { bar_sync(BAR_LOCAL, NL); });
-        if (warp < 4) {  // every read of A is done: T replaces it
+        if (warp < 4) {
+          tri::Frag Trow[4];
+          tri::inverse64_rows<tri::Sw128Layout>(tTP, tTP + 64 * 128, warp, lane, Trow,
+                                                [] { bar_sync(BAR_INV, 128); });
+          // every read of A is done: T replaces it
           const int rr = lane >> 2, qq = lane & 3;
 #pragma unroll
           for (int d = 0; d < 4; ++d) {
@@ -703,10 +704,19 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const uint32_t cD3 = col_d3(c);
       float gc = 0.f;
       if (run) {
-        if (!wait_all(&bar_v, ph_v, 0, false)) { aborted = true; break; }
-        convert_wr();
+        // v of this chunk (TMA data: every thread waits), its write vectors, then the slot; one
+        // group barrier decides both waits and orders the conversion before the MMAs
+        const bool ok_v = mbar_wait(&bar_v, ph_v & 1u, kWaitLimitNs);
+        ph_v ^= 1u;
+        if (ok_v) convert_wr();
         fence_async_smem();
-        if (!wait_all(&bar_full[j], ph_full, j, true)) { aborted = true; break; }
+        const bool ok_f = mbar_wait_cluster(&bar_full[j], (ph_full >> j) & 1u, kWaitLimitNs);
+        ph_full ^= 1u << j;
+        if (bar_or(BAR_CHAIN, NT - NL, !(ok_v && ok_f))) {
+          if (ct == 0) raise_status(p.status, STATUS_TIMEOUT);
+          aborted = true;
+          break;
+        }
         // the other CTA's copies of this slot have all landed: its bulk reads are done
         if (!producer && ct == 128)
           mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&bar_land[j]), static_cast<uint32_t>(peer)));
@@ -732,14 +742,29 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       }
       if (c > 0) store_o(c - 1);  // overlaps the MMAs above
       if (!run) break;
-      if (!wait_one(&bar_cmma, ph_mma, 0, false)) { aborted = true; break; }
+      // MMA group 1 done; U goes into X rows 0..63 of this slot, which in the producing CTA must
+      // wait until the copies out of it have landed in the other CTA
+      {
+        bool ok = true;
+        if (ct == 0) {
+          ok = mbar_wait(&bar_cmma, ph_mma & 1u, kWaitLimitNs);
+          if (ok && producer) ok = mbar_wait(&bar_land[j], (ph_land >> j) & 1u, kWaitLimitNs);
+        }
+        ph_mma ^= 1u;
+        if (producer) ph_land ^= 1u << j;
+        const bool fail = bar_or(BAR_CHAIN, NT - NL, !ok);
+        tc_fence_after();
+        if (fail) {
+          if (ct == 0) raise_status(p.status, STATUS_TIMEOUT);
+          aborted = true;
+          break;
+        }
+      }
       if (ct == 128) {
         if (c + 1 < nchunks) issue_v(c + 1);  // Wr is free
         if (c + 3 < nchunks) tma_prefetch_l2_4d(&tm_v, v0, h, (c + 3) * C, b);
       }
       if (c + 1 < nchunks) prefetch_ws(c + 1);
-      // U goes into X rows 0..63 of this slot: in the producing CTA, only once the copies are read
-      if (producer && !wait_one(&bar_land[j], ph_land, j, false)) { aborted = true; break; }
 
       // -------------------------------------------------------------- E3: U = U0 - W S -> X rows 0..63
       uint8_t *tU = sm + slot_off(j) + SX;
