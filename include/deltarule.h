@@ -127,6 +127,33 @@ DR_API dr_status dr_decode_step(const dr_problem *p,
                          float *S, void *o, void *stream);
 
 /*
+ * OSDN per-feature write-side key scaling (OSDN summary page, "Method": the
+ * diagonal preconditioner scales the key of the write while the read keeps
+ * the erase key).  Same as dr_chunk_fwd / dr_decode_step, with the
+ * transition S_t = (I - a_t b_t^T) Diag(alpha_t) S_{t-1} + a_t w_t^T, i.e.
+ *   u_t = w_t - (Diag(alpha_t) S_{t-1})^T b_t,   S_t = Diag(alpha_t) S_{t-1} + a_t u_t^T,
+ * where b_t = sqrt(beta_k_t) (.) k_t is the erase (read) key and
+ * a_t = s_t (.) b_t the write key.
+ *   s : [B, T, H, dk] fp32 (decode: [B, 1, H, dk]), 16-byte aligned, caller
+ *       owned, read only.  NULL gives a = b, the same result as
+ *       dr_chunk_fwd / dr_decode_step.
+ * The preconditioner's own update rule is not part of the operation: s is
+ * an input.  Every other argument, layout, the workspace and the errors are
+ * those of dr_chunk_fwd / dr_decode_step.  With s, a bf16 prefill with
+ * dk = dv = 128 and chunk 64 runs the tensor-core ring kernel whatever
+ * DR_PREFILL_KERNEL says; other shapes run the CUDA-core kernel.
+ */
+DR_API dr_status dr_chunk_fwd_osdn(const dr_problem *p,
+                                   const void *q, const void *k, const void *v,
+                                   const float *alpha, const float *beta_k, const float *beta_v,
+                                   const float *s, const float *S0, void *o, float *S_T,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+DR_API dr_status dr_decode_step_osdn(const dr_problem *p,
+                                     const void *q, const void *k, const void *v,
+                                     const float *alpha, const float *beta_k, const float *beta_v,
+                                     const float *s, float *S, void *o, void *stream);
+
+/*
  * dr_chunk_fwd for callers that cannot allocate device memory.  (The pages
  * have no counterpart; this is a deployment variant of dr_chunk_fwd.)  Some
  * hosts pre-plan every byte of device memory and give a kernel no workspace

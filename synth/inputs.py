@@ -11,6 +11,9 @@ the fixed order q, k, v, x_alpha, x_beta_k, x_beta_v, S0, skipping absent ones):
 * beta = sigmoid(x), x ~ N(0, 1): scalar or per channel (erase strength
   beta_k, and the decoupled write strength beta_v when present).
 * S0 = 0, or N(0, 0.01) read as variance 0.01 (standard deviation 0.1).
+* s (OSDN write-side key scale, optional; drawn last so the other draws do not
+  change) = exp(0.25 x), x ~ N(0, 1) per (b, t, h, key channel): a positive
+  per-feature scale around 1.  The OSDN summary gives no distribution for it.
 
 Draws are float32; q, k, v are then rounded to the I/O dtype (bf16 by
 round-to-nearest-even through torch) and the gates stay float32.  Arrays are
@@ -44,6 +47,7 @@ class Problem:
     beta_v: str        # "none", "scalar" or "channel"
     S0: str            # "zero" or "normal"
     seed: int
+    s_scale: str = "none"  # "none" or "channel": OSDN write-side key scale s [B,T,H,dk]
 
     @property
     def token_heads(self) -> int:
@@ -113,7 +117,7 @@ def _gate_shape(mode, lead, width):
 
 
 def make_inputs(p: Problem) -> dict:
-    """Draw one problem's inputs.  Keys: q, k, v, alpha, beta_k, beta_v, S0 (absent -> None)."""
+    """Draw one problem's inputs.  Keys: q, k, v, alpha, beta_k, beta_v, S0, s (absent -> None)."""
     rng = np.random.Generator(np.random.PCG64(p.seed))
     lead = (p.B, p.T, p.H)
     q = _l2_rows(_normal(rng, lead + (p.dk,)))
@@ -123,6 +127,7 @@ def make_inputs(p: Problem) -> dict:
     beta_k = _sigmoid(_normal(rng, _gate_shape(p.beta_k, lead, p.dk)))
     beta_v = _sigmoid(_normal(rng, _gate_shape(p.beta_v, lead, p.dv))) if p.beta_v != "none" else None
     S0 = (np.float32(0.1) * _normal(rng, (p.B, p.H, p.dk, p.dv))) if p.S0 == "normal" else None
+    s = np.exp(np.float32(0.25) * _normal(rng, lead + (p.dk,))).astype(np.float32) if p.s_scale != "none" else None
     io = _IO[p.io]
     t = torch.from_numpy
     return {
@@ -131,6 +136,7 @@ def make_inputs(p: Problem) -> dict:
         "beta_k": t(beta_k),
         "beta_v": None if beta_v is None else t(beta_v),
         "S0": None if S0 is None else t(S0),
+        "s": None if s is None else t(s),
     }
 
 

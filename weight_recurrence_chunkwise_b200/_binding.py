@@ -38,7 +38,8 @@ class DeltaRuleError(RuntimeError):
 
 _lib = None
 
-EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_chunk_fwd_noalloc", "dr_decode_step",
+EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_chunk_fwd_osdn", "dr_chunk_fwd_noalloc", "dr_decode_step",
+           "dr_decode_step_osdn",
            "dr_workspace_status", "dr_status_string", "dr_version", "dr_diag_umma_selftest",
            "dr_diag_tri_inverse")
 
@@ -59,6 +60,10 @@ def lib():
         L.dr_chunk_fwd_noalloc.restype = ctypes.c_int
         L.dr_decode_step.argtypes = [P] + [vp] * 8 + [vp]
         L.dr_decode_step.restype = ctypes.c_int
+        L.dr_chunk_fwd_osdn.argtypes = [P] + [vp] * 10 + [vp, sz, vp]
+        L.dr_chunk_fwd_osdn.restype = ctypes.c_int
+        L.dr_decode_step_osdn.argtypes = [P] + [vp] * 9 + [vp]
+        L.dr_decode_step_osdn.restype = ctypes.c_int
         L.dr_workspace_status.argtypes = [vp, vp]
         L.dr_workspace_status.restype = ctypes.c_int
         L.dr_status_string.argtypes = [ctypes.c_int]
@@ -120,6 +125,16 @@ def workspace_bytes(problem: dr_problem) -> int:
 def dr_chunk_fwd(q, k, v, beta_k, alpha=None, beta_v=None, S0=None, chunk=64, o=None, S_T=None,
                  workspace=None, stream=None, final_state=True):
     """Chunkwise prefill.  Returns ``(o, S_T)``; S_T is None when ``final_state`` is False."""
+    return _chunk_fwd(None, q, k, v, beta_k, alpha, beta_v, S0, chunk, o, S_T, workspace, stream, final_state)
+
+
+def dr_chunk_fwd_osdn(q, k, v, beta_k, s, alpha=None, beta_v=None, S0=None, chunk=64, o=None, S_T=None,
+                      workspace=None, stream=None, final_state=True):
+    """Chunkwise prefill with OSDN's write-side key scale ``s`` [B, T, H, dk] (write key a = s * b)."""
+    return _chunk_fwd(s, q, k, v, beta_k, alpha, beta_v, S0, chunk, o, S_T, workspace, stream, final_state)
+
+
+def _chunk_fwd(s, q, k, v, beta_k, alpha, beta_v, S0, chunk, o, S_T, workspace, stream, final_state):
     p = make_problem(q, v, alpha, beta_k, beta_v, chunk)
     dev = q.device
     if o is None:
@@ -127,15 +142,24 @@ def dr_chunk_fwd(q, k, v, beta_k, alpha=None, beta_v=None, S0=None, chunk=64, o=
     if S_T is None and final_state:
         S_T = torch.empty((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=dev)
     _check_tensors(q.dtype, [("q", q), ("k", k), ("v", v), ("o", o), ("alpha", alpha),
-                             ("beta_k", beta_k), ("beta_v", beta_v), ("S0", S0), ("S_T", S_T)])
+                             ("beta_k", beta_k), ("beta_v", beta_v), ("s", s), ("S0", S0), ("S_T", S_T)])
+    if s is not None and tuple(s.shape) != tuple(q.shape):
+        raise ValueError("s must have the shape of q / k: [B, T, H, dk]")
     need = workspace_bytes(p)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    rc = lib().dr_chunk_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
-                            _ptr(beta_v), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
-                            ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if s is None:
+        rc = lib().dr_chunk_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
+                                _ptr(beta_v), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+                                ctypes.c_size_t(workspace.numel()), _stream(stream))
+        name = "dr_chunk_fwd"
+    else:
+        rc = lib().dr_chunk_fwd_osdn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
+                                     _ptr(beta_v), _ptr(s), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+                                     ctypes.c_size_t(workspace.numel()), _stream(stream))
+        name = "dr_chunk_fwd_osdn"
     if rc != DR_OK:
-        raise DeltaRuleError(rc, "dr_chunk_fwd")
+        raise DeltaRuleError(rc, name)
     return o, S_T
 
 
@@ -166,15 +190,32 @@ def dr_decode_step(q, k, v, beta_k, S, alpha=None, beta_v=None, o=None, stream=N
 
     q, k: [B, 1, H, dk]; v: [B, 1, H, dv]; gates [B, 1, H] or [B, 1, H, d]; S [B, H, dk, dv].
     """
+    return _decode_step(None, q, k, v, beta_k, S, alpha, beta_v, o, stream)
+
+
+def dr_decode_step_osdn(q, k, v, beta_k, S, s, alpha=None, beta_v=None, o=None, stream=None):
+    """dr_decode_step with OSDN's write-side key scale ``s`` [B, 1, H, dk] (write key a = s * b)."""
+    return _decode_step(s, q, k, v, beta_k, S, alpha, beta_v, o, stream)
+
+
+def _decode_step(s, q, k, v, beta_k, S, alpha, beta_v, o, stream):
     p = make_problem(q, v, alpha, beta_k, beta_v, 0)
     if o is None:
         o = torch.empty(q.shape[:3] + (p.dv,), dtype=q.dtype, device=q.device)
     _check_tensors(q.dtype, [("q", q), ("k", k), ("v", v), ("o", o), ("alpha", alpha),
-                             ("beta_k", beta_k), ("beta_v", beta_v), ("S", S)])
-    rc = lib().dr_decode_step(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
-                              _ptr(beta_v), _ptr(S), _ptr(o), _stream(stream))
+                             ("beta_k", beta_k), ("beta_v", beta_v), ("s", s), ("S", S)])
+    if s is not None and tuple(s.shape) != tuple(q.shape):
+        raise ValueError("s must have the shape of q / k: [B, 1, H, dk]")
+    if s is None:
+        rc = lib().dr_decode_step(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
+                                  _ptr(beta_v), _ptr(S), _ptr(o), _stream(stream))
+        name = "dr_decode_step"
+    else:
+        rc = lib().dr_decode_step_osdn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
+                                       _ptr(beta_v), _ptr(s), _ptr(S), _ptr(o), _stream(stream))
+        name = "dr_decode_step_osdn"
     if rc != DR_OK:
-        raise DeltaRuleError(rc, "dr_decode_step")
+        raise DeltaRuleError(rc, name)
     return o
 
 

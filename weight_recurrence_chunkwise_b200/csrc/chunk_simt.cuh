@@ -7,7 +7,8 @@
 // from state S (dk x VS slice of value columns):
 //
 //   gamma_r = prod_{j<=r} alpha_j             cumulative gate (K1)
-//   Bh_r = gamma_r b_r,  Ac_r = b_r / gamma_r,  Qh_r = gamma_r q_r
+//   Bh_r = gamma_r b_r,  Ac_r = a_r / gamma_r,  Qh_r = gamma_r q_r
+//   (write key a = b, or a = s (.) b under OSDN's write-side key scaling)
 //   A = strictly-lower(Bh Ac^T),  T = (I + A)^-1,  P = lower(Qh Ac^T)   (K2)
 //   U = T (Wr - Bh S)                         (K2 + K3: rows u_r of the chunk)
 //   O = Qh S + P U                            (K4)
@@ -35,7 +36,7 @@ __global__ void __launch_bounds__(256)
 chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restrict__ k,
                       const IO *__restrict__ v, const float *__restrict__ alpha, int alpha_mode,
                       const float *__restrict__ beta_k, int beta_k_mode, const float *__restrict__ beta_v,
-                      int beta_v_mode, const float *__restrict__ S0, IO *__restrict__ o,
+                      int beta_v_mode, const float *__restrict__ s_scale, const float *__restrict__ S0, IO *__restrict__ o,
                       float *__restrict__ S_T, uint32_t *__restrict__ status) {
   using L_ = SimtSmem<DK, VS, C>;
   constexpr int LDK = L_::LDK, LC = L_::LC, LV = L_::LV;
@@ -72,7 +73,8 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
           g *= gate_at(alpha, alpha_mode, th, DK, tid);
           const float bk = sqrtf(gate_at(beta_k, beta_k_mode, th, DK, tid)) * to_f32(k[th * DK + tid]);
           Bh[r * LDK + tid] = g * bk;
-          Ac[r * LDK + tid] = bk / g;
+          const float ak = s_scale ? s_scale[th * DK + tid] * bk : bk;  // write key a
+          Ac[r * LDK + tid] = ak / g;
           Qh[r * LDK + tid] = g * to_f32(q[th * DK + tid]);
         } else {
           Bh[r * LDK + tid] = 0.f;

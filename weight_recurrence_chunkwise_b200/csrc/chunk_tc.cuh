@@ -90,6 +90,7 @@ struct Params {
   void *o;
   float *S_T;
   uint32_t *status;
+  const float *s = nullptr;  // write-side key scale [B,T,H,dk] (a = s (.) b); only the ring kernel reads it
 };
 
 __device__ __forceinline__ void st_h16x8(uint8_t *tile, int row, int col0, int R, const float *v) {

@@ -1,8 +1,10 @@
 // chunk_tc3.cuh -- chunkwise WY/UT prefill on a cluster of two CTAs per (b, h), with a ring of
 // three factor slots.
 //
-// Algebra (DeltaNet page, step 7; FG2-GDN page, section 2), per chunk of C = 64 tokens:
-//   chunk-local:  gamma, Qh = gamma q, Bh = gamma b, Ac = b / gamma, P = lower(Qh Ac^T),
+// Algebra (DeltaNet page, step 7; FG2-GDN page, section 2), per chunk of C = 64 tokens, with the
+// erase key b = sqrt(beta_k) (.) k and the write key a = b, or a = s (.) b under OSDN's per-feature
+// write-side key scaling (OSDN summary page, "Method"; kernel flag kScaled):
+//   chunk-local:  gamma, Qh = gamma q, Bh = gamma b, Ac = a / gamma, P = lower(Qh Ac^T),
 //                 T = (I + strictly-lower(Bh Ac^T))^-1, W = T Bh
 //   state pass:   U0 = T Wr, U = U0 - W S, O = Qh S + P U, S <- Diag(gamma_C)(S + Ac^T U)
 //
@@ -95,7 +97,8 @@ __device__ __forceinline__ bool mbar_test_cluster(uint64_t *bar, uint32_t parity
 
 // kChanGates: the gates vary per key channel (alpha per channel, or beta_k per channel); else
 // they are one value per row (alpha absent or per token, beta_k per token).
-template <typename IO, bool kChanGates>
+// kScaled: a write-side key scale s [B,T,H,dk] is given (Params::s).
+template <typename IO, bool kChanGates, bool kScaled>
 __global__ void __launch_bounds__(NT, 1)
 chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -178,6 +181,10 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     auto prefetch_gates = [&](int c) {
       const int t0 = c * C, L = min(C, T - t0);
       const size_t thb = (static_cast<size_t>(b) * T + t0) * H + h;
+      if constexpr (kScaled) {  // thread ltid: 128-byte line (ltid & 3) of row (ltid >> 2) of s
+        const size_t th = thb + static_cast<size_t>(min(ltid >> 2, L - 1)) * H;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p.s + th * DK + (ltid & 3) * 32));
+      }
       if constexpr (gates_scalar) {
         if (warp == 0) {
 #pragma unroll
@@ -305,7 +312,19 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // elements: (row r, 8-column group j8), four per thread, 16-byte loads and stores
         const int j8 = ltid & 15;
         float amax = 0.f;
-#pragma unroll 1
+        float ssc[kScaled ? 4 : 1][kScaled ? 8 : 1];  // write-side key scales of my four rows
+        if constexpr (kScaled) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = min((ltid >> 4) + 16 * i, L - 1);
+            const float4 *src = reinterpret_cast<const float4 *>(
+                p.s + ((static_cast<size_t>(b) * T + t0 + r) * H + h) * DK + j8 * 8);
+            const float4 lo = __ldg(src), hi = __ldg(src + 1);
+            ssc[i][0] = lo.x; ssc[i][1] = lo.y; ssc[i][2] = lo.z; ssc[i][3] = lo.w;
+            ssc[i][4] = hi.x; ssc[i][5] = hi.y; ssc[i][6] = hi.z; ssc[i][7] = hi.w;
+          }
+        }
+#pragma unroll(kScaled ? 4 : 1)
         for (int i = 0; i < 4; ++i) {
           const int r = (ltid >> 4) + 16 * i;
           const float g = sRow[r], gi = sRow[64 + r], sb = sRow[128 + r];
@@ -319,7 +338,11 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           for (int e = 0; e < 4; ++e) {
             const float2 qf = __bfloat1622float2(q2[e]), kf = __bfloat1622float2(k2[e]);
             const float b0 = sb * kf.x, b1 = sb * kf.y;
-            const float x0 = b0 * gi, x1 = b1 * gi;
+            float x0 = b0 * gi, x1 = b1 * gi;
+            if constexpr (kScaled) {
+              x0 *= ssc[i][2 * e];
+              x1 *= ssc[i][2 * e + 1];
+            }
             amax = fmaxf(amax, fmaxf(fabsf(x0), fabsf(x1)));
             oq[e] = pack_f16x2(g * qf.x, g * qf.y);
             ob[e] = pack_f16x2(g * b0, g * b1);
@@ -389,7 +412,13 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           ga *= pal[2 * jj];
           gb *= pal[2 * jj + 1];
           const float b0 = s0 * kf.x, b1 = s1 * kf.y;
-          const float a0 = b0 * __fdividef(1.f, ga), a1 = b1 * __fdividef(1.f, gb);  // b / gamma_r
+          float a0 = b0 * __fdividef(1.f, ga), a1 = b1 * __fdividef(1.f, gb);  // a / gamma_r
+          if constexpr (kScaled) {
+            const size_t th = (static_cast<size_t>(b) * T + t0 + min(rgl * RGL + jj, L - 1)) * H + h;
+            const float2 sc = __ldg(reinterpret_cast<const float2 *>(p.s + th * DK + c0));
+            a0 *= sc.x;
+            a1 *= sc.y;
+          }
           amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
           *reinterpret_cast<uint32_t *>(pQ + sw) = pack_f16x2(ga * qf.x, gb * qf.y);  // Qh (in place of q)
           *reinterpret_cast<uint32_t *>(pB + sw) = pack_f16x2(ga * b0, gb * b1);      // Bh (in place of k)
@@ -407,7 +436,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           const uint64_t dX = sdesc_sw128(xaddr + SX, 16, 1024);
           const uint64_t dAcK = sdesc_sw128(xaddr + SAC, 16, 1024);
           const uint32_t idesc = idesc_f16_f32(128, 64, false, false);
-#pragma unroll 1
+#pragma unroll
           for (int kk = 0; kk < DK / 16; ++kk)
             umma_f16(tmem + COL_D1, kstep(dX, 128, kk), kstep(dAcK, 64, kk), idesc, kk > 0);
           umma_commit(&bar_lmma);
@@ -474,7 +503,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           const uint64_t dTP = sdesc_sw128(xaddr + STP, 16, 1024);
           const uint64_t dBh = sdesc_sw128(xaddr + SX, SX_CB, 1024);
           const uint32_t id2 = idesc_f16_f32(128, 128, false, true);
-#pragma unroll 1
+#pragma unroll
           for (int kk = 0; kk < C / 16; ++kk)
             umma_f16(tmem + COL_D2, kstep(dTP, 128, kk), mstep(dBh, kk), id2, kk > 0);
           umma_commit(&bar_lmma);
@@ -729,10 +758,10 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const uint64_t dTP = sdesc_sw128(xaddr + STP, 16, 1024);
             const uint64_t dX = sdesc_sw128(xaddr + SX, 16, 1024);
             const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
-#pragma unroll 1
+#pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
               umma_f16(tmem + COL_U0, kstep(dTP, 128, kk), mstep(dWr, kk), id3, kk > 0);
-#pragma unroll 1
+#pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
               umma_f16(tmem + cD3, kstep(dX, 128, kk), mstep(dS, kk), id3, kk > 0);
             umma_commit(&bar_cmma);
@@ -798,9 +827,9 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           const uint64_t dU = sdesc_sw128(xaddr + SX, 128 * 128, 1024);
           const uint32_t id4 = idesc_f16_f32(128, VS, true, true);
           const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
-#pragma unroll 1
+#pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_D4, mstep(dAcM, kk), mstep(dU, kk), id4, kk > 0);
-#pragma unroll 1
+#pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + cD3, kstep(dTP, 128, kk), mstep(dU, kk), id3, 1u);
           umma_commit(&bar_cmma);
         }

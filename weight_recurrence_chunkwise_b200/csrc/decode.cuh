@@ -3,8 +3,10 @@
 // For every head (b, h), with D = Diag(alpha):
 //   r = (D S)^T b,  p = (D S)^T q          two reductions over the key dimension
 //   u = w - r                              error of the read against the write vector
-//   o = p + u (b . q)                      = S_new^T q
-//   S <- D S + b u^T                       = (I - b b^T) D S + b w^T
+//   o = p + u (a . q)                      = S_new^T q
+//   S <- D S + a u^T                       = (I - a b^T) D S + a w^T
+// with the write key a = b, or a = s (.) b under OSDN's per-feature write-side key scaling
+// (OSDN summary page, "Method").
 // DeltaNet page, steps 3-6 (read, error, rank-1 write, output from the
 // updated state); FG2-GDN page, section 2 (decay first, sqrt(beta) scaling,
 // decoupled beta^v for FG2-GDN+).
@@ -27,14 +29,14 @@ __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
                    const float *__restrict__ alpha, int alpha_mode, const float *__restrict__ beta_k,
                    int beta_k_mode, const float *__restrict__ beta_v, int beta_v_mode,
-                   float *__restrict__ S, IO *__restrict__ o) {
+                   const float *__restrict__ s_scale, float *__restrict__ S, IO *__restrict__ o) {
   constexpr int NW = 8;
   constexpr int RPW = DK / NW;
   constexpr int CPL = DV / 32;
   using V = typename VecF<CPL>::T;
   static_assert(DK % NW == 0 && DV % 64 == 0, "unsupported head dims");
 
-  __shared__ float s_al[DK], s_b[DK], s_q[DK], s_w[DV], s_u[DV];
+  __shared__ float s_al[DK], s_b[DK], s_a[DK], s_q[DK], s_w[DV], s_u[DV];
   __shared__ float s_red_r[NW][DV], s_red_p[NW][DV];
   __shared__ float s_bq;
 
@@ -53,10 +55,12 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
     for (int c = 0; c < CPL; ++c) s[rr][c] = xf[c];
   }
 
-  // 2. per-row factors: decay, erase key b = sqrt(beta_k) k, query; write vector w
+  // 2. per-row factors: decay, erase key b = sqrt(beta_k) k, write key a, query; write vector w
   if (tid < DK) {
     const float bk = gate_at(beta_k, beta_k_mode, bh, DK, tid);
-    s_b[tid] = sqrtf(bk) * to_f32(k[bh * DK + tid]);
+    const float bt = sqrtf(bk) * to_f32(k[bh * DK + tid]);
+    s_b[tid] = bt;
+    s_a[tid] = s_scale ? s_scale[bh * DK + tid] * bt : bt;
     s_q[tid] = to_f32(q[bh * DK + tid]);
     s_al[tid] = gate_at(alpha, alpha_mode, bh, DK, tid);
   }
@@ -70,7 +74,7 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
   __syncthreads();
   if (warp == 0) {
     float acc = 0.f;
-    for (int i = lane; i < DK; i += 32) acc += s_b[i] * s_q[i];
+    for (int i = lane; i < DK; i += 32) acc += s_a[i] * s_q[i];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) s_bq = acc;
@@ -116,11 +120,11 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr) {
     const int i = warp + rr * NW;
-    const float bi = s_b[i];
+    const float ai = s_a[i];
     V x;
     float *xf = reinterpret_cast<float *>(&x);
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) xf[c] = fmaf(bi, s_u[lane * CPL + c], s[rr][c]);
+    for (int c = 0; c < CPL; ++c) xf[c] = fmaf(ai, s_u[lane * CPL + c], s[rr][c]);
     __stcs(reinterpret_cast<V *>(Sh + i * DV + lane * CPL), x);
   }
 }

@@ -77,8 +77,8 @@ dr_status launch_status() {
 // ----------------------------------------------------------------- prefill, CUDA-core path
 template <typename IO, int DK, int DV, int C>
 dr_status simt_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                      const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
-                      uint32_t *status, cudaStream_t st) {
+                      const float *beta_k, const float *beta_v, const float *s_scale, const float *S0, void *o,
+                      float *S_T, uint32_t *status, cudaStream_t st) {
   constexpr int VS = 32;
   auto kern = dr::chunk_fwd_simt_kernel<IO, DK, DV, VS, C>;
   constexpr size_t smem = dr::SimtSmem<DK, VS, C>::bytes;
@@ -88,32 +88,32 @@ dr_status simt_launch(const dr_problem *p, const void *q, const void *k, const v
   dim3 grid(DV / VS, p->H, p->B);
   kern<<<grid, 256, smem, st>>>(p->T, p->H, static_cast<const IO *>(q), static_cast<const IO *>(k),
                                 static_cast<const IO *>(v), alpha, p->alpha_mode, beta_k, p->beta_k_mode,
-                                beta_v, p->beta_v_mode, S0, static_cast<IO *>(o), S_T, status);
+                                beta_v, p->beta_v_mode, s_scale, S0, static_cast<IO *>(o), S_T, status);
   return launch_status();
 }
 
 template <typename IO, int DK, int DV>
 dr_status simt_by_chunk(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                        const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
-                        uint32_t *status, cudaStream_t st) {
+                        const float *beta_k, const float *beta_v, const float *s_scale, const float *S0, void *o,
+                        float *S_T, uint32_t *status, cudaStream_t st) {
   switch (p->chunk) {
-    case 16: return simt_launch<IO, DK, DV, 16>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
-    case 32: return simt_launch<IO, DK, DV, 32>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
-    default: return simt_launch<IO, DK, DV, 64>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+    case 16: return simt_launch<IO, DK, DV, 16>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+    case 32: return simt_launch<IO, DK, DV, 32>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+    default: return simt_launch<IO, DK, DV, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
   }
 }
 
 template <typename IO>
 dr_status simt_dispatch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                        const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
-                        uint32_t *status, cudaStream_t st) {
+                        const float *beta_k, const float *beta_v, const float *s_scale, const float *S0, void *o,
+                        float *S_T, uint32_t *status, cudaStream_t st) {
   if (p->dk == 128 && p->dv == 128)
-    return simt_by_chunk<IO, 128, 128>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+    return simt_by_chunk<IO, 128, 128>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
   if (p->dk == 128 && p->dv == 64)
-    return simt_by_chunk<IO, 128, 64>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+    return simt_by_chunk<IO, 128, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
   if (p->dk == 64 && p->dv == 128)
-    return simt_by_chunk<IO, 64, 128>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
-  return simt_by_chunk<IO, 64, 64>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+    return simt_by_chunk<IO, 64, 128>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+  return simt_by_chunk<IO, 64, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
 }
 
 // ----------------------------------------------------------------- prefill, tensor-core path (bf16 I/O)
@@ -220,8 +220,8 @@ dr_status tc_pair_launch(const dr_problem *p, const void *q, const void *k, cons
 }
 
 dr_status tc_ring_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                         const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
-                         uint32_t *status, cudaStream_t st) {
+                         const float *beta_k, const float *beta_v, const float *s_scale, const float *S0, void *o,
+                         float *S_T, uint32_t *status, cudaStream_t st) {
   using IO = __nv_bfloat16;
   namespace tc = dr::tc;
   namespace tc3 = dr::tc3;
@@ -233,9 +233,12 @@ dr_status tc_ring_launch(const dr_problem *p, const void *q, const void *k, cons
       !make_map(&mv, bf, 2, v, p->B, p->T, p->H, p->dv, tc::VS, tc::C, sw))
     return DR_ERR_CUDA;
   tc::Params prm{p->T, p->H, p->dv, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v, p->beta_v_mode,
-                 S0, o, S_T, status};
+                 S0, o, S_T, status, s_scale};
   const bool chan_gates = p->alpha_mode == DR_CHANNEL || p->beta_k_mode != DR_SCALAR;
-  auto kern = chan_gates ? tc3::chunk_fwd_ring_kernel<IO, true> : tc3::chunk_fwd_ring_kernel<IO, false>;
+  auto kern = s_scale ? (chan_gates ? tc3::chunk_fwd_ring_kernel<IO, true, true>
+                                    : tc3::chunk_fwd_ring_kernel<IO, false, true>)
+                      : (chan_gates ? tc3::chunk_fwd_ring_kernel<IO, true, false>
+                                    : tc3::chunk_fwd_ring_kernel<IO, false, false>);
   constexpr size_t smem = tc3::SMEM_BYTES;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
@@ -259,22 +262,76 @@ dr_status tc_ring_launch(const dr_problem *p, const void *q, const void *k, cons
 // ----------------------------------------------------------------- decode
 template <typename IO, int DK, int DV>
 dr_status decode_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                        const float *beta_k, const float *beta_v, float *S, void *o, cudaStream_t st) {
+                        const float *beta_k, const float *beta_v, const float *s_scale, float *S, void *o,
+                        cudaStream_t st) {
   const long long heads = static_cast<long long>(p->B) * p->H;
   if (heads > 0x7fffffffLL) return DR_ERR_INVALID_ARG;
   dr::decode_step_kernel<IO, DK, DV><<<static_cast<unsigned>(heads), 256, 0, st>>>(
       static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v), alpha, p->alpha_mode,
-      beta_k, p->beta_k_mode, beta_v, p->beta_v_mode, S, static_cast<IO *>(o));
+      beta_k, p->beta_k_mode, beta_v, p->beta_v_mode, s_scale, S, static_cast<IO *>(o));
   return launch_status();
 }
 
 template <typename IO>
 dr_status decode_dispatch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                          const float *beta_k, const float *beta_v, float *S, void *o, cudaStream_t st) {
-  if (p->dk == 128 && p->dv == 128) return decode_launch<IO, 128, 128>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
-  if (p->dk == 128 && p->dv == 64) return decode_launch<IO, 128, 64>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
-  if (p->dk == 64 && p->dv == 128) return decode_launch<IO, 64, 128>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
-  return decode_launch<IO, 64, 64>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
+                          const float *beta_k, const float *beta_v, const float *s_scale, float *S, void *o,
+                          cudaStream_t st) {
+  if (p->dk == 128 && p->dv == 128)
+    return decode_launch<IO, 128, 128>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
+  if (p->dk == 128 && p->dv == 64)
+    return decode_launch<IO, 128, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
+  if (p->dk == 64 && p->dv == 128)
+    return decode_launch<IO, 64, 128>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
+  return decode_launch<IO, 64, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
+}
+
+// Prefill with an optional write-side key scale (NULL: a = b).
+dr_status chunk_fwd_impl(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                         const float *beta_k, const float *beta_v, const float *s_scale, const float *S0, void *o,
+                         float *S_T, void *workspace, size_t workspace_bytes, void *stream) {
+  dr_status s = check_common(p, false);
+  if (s != DR_OK) return s;
+  s = check_pointers(p, q, k, v, alpha, beta_k, beta_v, o);
+  if (s != DR_OK) return s;
+  if ((S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)) || (s_scale && !aligned16(s_scale)))
+    return DR_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < kWorkspaceBytes) return DR_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return DR_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *status = static_cast<uint32_t *>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DR_ERR_CUDA;
+  const size_t state_bytes = sizeof(float) * size_t(p->B) * p->H * p->dk * p->dv;
+  if (p->T == 0) {  // nothing to scan: the final state is the initial state
+    if (!S_T) return DR_OK;
+    const cudaError_t e = S0 ? (S0 == S_T ? cudaSuccess
+                                          : cudaMemcpyAsync(S_T, S0, state_bytes, cudaMemcpyDeviceToDevice, st))
+                             : cudaMemsetAsync(S_T, 0, state_bytes, st);
+    return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+  }
+  if (p->io_dtype == DR_F32)
+    return simt_dispatch<float>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+  const bool ring_shape = p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv == 2 * dr::tc::VS;
+  if (ring_shape && (s_scale || prefill_kernel() == kRing))
+    return tc_ring_launch(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+  if (!s_scale && ring_shape && prefill_kernel() == kPair)
+    return tc_pair_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+  if (!s_scale && p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv % dr::tc::VS == 0)
+    return tc_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+  return simt_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+}
+
+dr_status decode_step_impl(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                           const float *beta_k, const float *beta_v, const float *s_scale, float *S, void *o,
+                           void *stream) {
+  dr_status s = check_common(p, true);
+  if (s != DR_OK) return s;
+  s = check_pointers(p, q, k, v, alpha, beta_k, beta_v, o);
+  if (s != DR_OK) return s;
+  if (!S) return DR_ERR_INVALID_ARG;
+  if (!aligned16(S) || (s_scale && !aligned16(s_scale))) return DR_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p->io_dtype == DR_F32) return decode_dispatch<float>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
+  return decode_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
 }
 
 }  // namespace
@@ -304,45 +361,24 @@ size_t dr_chunk_fwd_workspace(const dr_problem *p) {
 dr_status dr_chunk_fwd(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
                        const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
                        void *workspace, size_t workspace_bytes, void *stream) {
-  dr_status s = check_common(p, false);
-  if (s != DR_OK) return s;
-  s = check_pointers(p, q, k, v, alpha, beta_k, beta_v, o);
-  if (s != DR_OK) return s;
-  if ((S0 && !aligned16(S0)) || (S_T && !aligned16(S_T))) return DR_ERR_ALIGNMENT;
-  if (!workspace || workspace_bytes < kWorkspaceBytes) return DR_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return DR_ERR_ALIGNMENT;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint32_t *status = static_cast<uint32_t *>(workspace);
-  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DR_ERR_CUDA;
-  const size_t state_bytes = sizeof(float) * size_t(p->B) * p->H * p->dk * p->dv;
-  if (p->T == 0) {  // nothing to scan: the final state is the initial state
-    if (!S_T) return DR_OK;
-    const cudaError_t e = S0 ? (S0 == S_T ? cudaSuccess
-                                          : cudaMemcpyAsync(S_T, S0, state_bytes, cudaMemcpyDeviceToDevice, st))
-                             : cudaMemsetAsync(S_T, 0, state_bytes, st);
-    return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
-  }
-  if (p->io_dtype == DR_F32)
-    return simt_dispatch<float>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
-  if (p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv == 2 * dr::tc::VS && prefill_kernel() != kSingle)
-    return prefill_kernel() == kPair ? tc_pair_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st)
-                                     : tc_ring_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
-  if (p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv % dr::tc::VS == 0)
-    return tc_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
-  return simt_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
+  return chunk_fwd_impl(p, q, k, v, alpha, beta_k, beta_v, nullptr, S0, o, S_T, workspace, workspace_bytes, stream);
+}
+
+dr_status dr_chunk_fwd_osdn(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                            const float *beta_k, const float *beta_v, const float *s, const float *S0, void *o,
+                            float *S_T, void *workspace, size_t workspace_bytes, void *stream) {
+  return chunk_fwd_impl(p, q, k, v, alpha, beta_k, beta_v, s, S0, o, S_T, workspace, workspace_bytes, stream);
 }
 
 dr_status dr_decode_step(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
                          const float *beta_k, const float *beta_v, float *S, void *o, void *stream) {
-  dr_status s = check_common(p, true);
-  if (s != DR_OK) return s;
-  s = check_pointers(p, q, k, v, alpha, beta_k, beta_v, o);
-  if (s != DR_OK) return s;
-  if (!S) return DR_ERR_INVALID_ARG;
-  if (!aligned16(S)) return DR_ERR_ALIGNMENT;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (p->io_dtype == DR_F32) return decode_dispatch<float>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
-  return decode_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, S, o, st);
+  return decode_step_impl(p, q, k, v, alpha, beta_k, beta_v, nullptr, S, o, stream);
+}
+
+dr_status dr_decode_step_osdn(const dr_problem *p, const void *q, const void *k, const void *v,
+                              const float *alpha, const float *beta_k, const float *beta_v, const float *s, float *S,
+                              void *o, void *stream) {
+  return decode_step_impl(p, q, k, v, alpha, beta_k, beta_v, s, S, o, stream);
 }
 
 // ----------------------------------------------------------------- prefill without allocation
