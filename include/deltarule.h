@@ -154,6 +154,33 @@ DR_API dr_status dr_decode_step_osdn(const dr_problem *p,
                                      const float *s, float *S, void *o, void *stream);
 
 /*
+ * Packed variable-length batch: the chunkwise prefill of several sequences of
+ * different lengths laid end to end, each an independent recurrence from its
+ * own initial state.  The DeltaNet page's deployment setting (a chunkwise pass
+ * over each prompt, then constant-state recurrent steps) in serving form: after
+ * this call, dr_decode_step / dr_decode_step_osdn with B = number of sequences
+ * continue every sequence from its row of S_T.
+ *   p->B        number of sequences N;  p->T  total tokens Ttot of the packed arrays
+ *   cu_seqlens  device int32 [N + 1], 4-byte aligned, cu[0] = 0, non-decreasing,
+ *               cu[N] = Ttot: sequence n is tokens cu[n] .. cu[n+1]-1.  Empty
+ *               sequences are allowed (their S_T is their S0).  Offsets are
+ *               clamped to [0, Ttot] on the device, so malformed ones give wrong
+ *               results but never an out-of-range access.
+ *   q, k, o     [1, Ttot, H, dk|dv] (the dense layout with B = 1); v likewise
+ *   alpha, beta_k, beta_v, s   [1, Ttot, H] or [1, Ttot, H, d] as in dr_chunk_fwd
+ *               (s: the OSDN write-side key scale, or NULL)
+ *   S0, S_T     [N, H, dk, dv] fp32, one state per sequence (S0 NULL: zero)
+ * Workspace, stream, dtypes, chunk sizes and errors are those of dr_chunk_fwd;
+ * cu_seqlens NULL returns DR_ERR_INVALID_ARG.  bf16 with dk = dv = 128 and
+ * chunk 64 runs the tensor-core ring kernel, other shapes the CUDA-core kernel.
+ */
+DR_API dr_status dr_chunk_fwd_varlen(const dr_problem *p, const int *cu_seqlens,
+                                     const void *q, const void *k, const void *v,
+                                     const float *alpha, const float *beta_k, const float *beta_v,
+                                     const float *s, const float *S0, void *o, float *S_T,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * dr_chunk_fwd for callers that cannot allocate device memory.  (The pages
  * have no counterpart; this is a deployment variant of dr_chunk_fwd.)  Some
  * hosts pre-plan every byte of device memory and give a kernel no workspace

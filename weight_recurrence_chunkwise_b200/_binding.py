@@ -38,7 +38,8 @@ class DeltaRuleError(RuntimeError):
 
 _lib = None
 
-EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_chunk_fwd_osdn", "dr_chunk_fwd_noalloc", "dr_decode_step",
+EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_chunk_fwd_osdn", "dr_chunk_fwd_varlen",
+           "dr_chunk_fwd_noalloc", "dr_decode_step",
            "dr_decode_step_osdn",
            "dr_workspace_status", "dr_status_string", "dr_version", "dr_diag_umma_selftest",
            "dr_diag_tri_inverse")
@@ -62,6 +63,8 @@ def lib():
         L.dr_decode_step.restype = ctypes.c_int
         L.dr_chunk_fwd_osdn.argtypes = [P] + [vp] * 10 + [vp, sz, vp]
         L.dr_chunk_fwd_osdn.restype = ctypes.c_int
+        L.dr_chunk_fwd_varlen.argtypes = [P] + [vp] * 11 + [vp, sz, vp]
+        L.dr_chunk_fwd_varlen.restype = ctypes.c_int
         L.dr_decode_step_osdn.argtypes = [P] + [vp] * 9 + [vp]
         L.dr_decode_step_osdn.restype = ctypes.c_int
         L.dr_workspace_status.argtypes = [vp, vp]
@@ -132,6 +135,44 @@ def dr_chunk_fwd_osdn(q, k, v, beta_k, s, alpha=None, beta_v=None, S0=None, chun
                       workspace=None, stream=None, final_state=True):
     """Chunkwise prefill with OSDN's write-side key scale ``s`` [B, T, H, dk] (write key a = s * b)."""
     return _chunk_fwd(s, q, k, v, beta_k, alpha, beta_v, S0, chunk, o, S_T, workspace, stream, final_state)
+
+
+def dr_chunk_fwd_varlen(q, k, v, beta_k, cu_seqlens, alpha=None, beta_v=None, s=None, S0=None, chunk=64, o=None,
+                        S_T=None, workspace=None, stream=None):
+    """Prefill of a packed batch: sequence n is tokens cu_seqlens[n] .. cu_seqlens[n+1]-1.
+
+    q, k, v (and gates, s): [1, Ttot, H, d]; cu_seqlens: int32 CUDA tensor [N + 1]; S0 and the
+    returned S_T: [N, H, dk, dv].  Returns ``(o, S_T)``.
+    """
+    if q.shape[0] != 1:
+        raise ValueError("a packed batch has leading dimension 1: [1, Ttot, H, d]")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be a 1-D int32 CUDA tensor")
+    n = cu_seqlens.numel() - 1
+    if n < 1:
+        raise ValueError("cu_seqlens needs at least two entries")
+    p = make_problem(q, v, alpha, beta_k, beta_v, chunk)
+    p.B = n
+    dev = q.device
+    if o is None:
+        o = torch.empty(q.shape[:3] + (p.dv,), dtype=q.dtype, device=dev)
+    if S_T is None:
+        S_T = torch.empty((n, p.H, p.dk, p.dv), dtype=torch.float32, device=dev)
+    _check_tensors(q.dtype, [("q", q), ("k", k), ("v", v), ("o", o), ("alpha", alpha),
+                             ("beta_k", beta_k), ("beta_v", beta_v), ("s", s), ("S0", S0), ("S_T", S_T)])
+    if s is not None and tuple(s.shape) != tuple(q.shape):
+        raise ValueError("s must have the shape of q / k")
+    if S0 is not None and tuple(S0.shape) != (n, p.H, p.dk, p.dv):
+        raise ValueError("S0 must be [N, H, dk, dv]")
+    need = workspace_bytes(p)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    rc = lib().dr_chunk_fwd_varlen(ctypes.byref(p), _ptr(cu_seqlens), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                   _ptr(beta_k), _ptr(beta_v), _ptr(s), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+                                   ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if rc != DR_OK:
+        raise DeltaRuleError(rc, "dr_chunk_fwd_varlen")
+    return o, S_T
 
 
 def _chunk_fwd(s, q, k, v, beta_k, alpha, beta_v, S0, chunk, o, S_T, workspace, stream, final_state):

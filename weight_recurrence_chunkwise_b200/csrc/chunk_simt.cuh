@@ -36,8 +36,9 @@ __global__ void __launch_bounds__(256)
 chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restrict__ k,
                       const IO *__restrict__ v, const float *__restrict__ alpha, int alpha_mode,
                       const float *__restrict__ beta_k, int beta_k_mode, const float *__restrict__ beta_v,
-                      int beta_v_mode, const float *__restrict__ s_scale, const float *__restrict__ S0, IO *__restrict__ o,
-                      float *__restrict__ S_T, uint32_t *__restrict__ status) {
+                      int beta_v_mode, const float *__restrict__ s_scale, const int *__restrict__ cu_seqlens,
+                      const float *__restrict__ S0, IO *__restrict__ o, float *__restrict__ S_T,
+                      uint32_t *__restrict__ status) {
   using L_ = SimtSmem<DK, VS, C>;
   constexpr int LDK = L_::LDK, LC = L_::LC, LV = L_::LV;
   extern __shared__ float sm[];
@@ -54,6 +55,14 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
 
   const int tid = threadIdx.x;
   const int v0 = blockIdx.x * VS, h = blockIdx.y, b = blockIdx.z;
+  // dense batch: tokens b*T ..; packed batch: sequence b is tokens cu[b] .. cu[b+1]-1 (clamped to
+  // [0, Ttot] so that malformed offsets cannot address outside the arrays)
+  size_t tok0 = static_cast<size_t>(b) * T;
+  if (cu_seqlens) {
+    const int cs = min(max(cu_seqlens[b], 0), T);
+    tok0 = static_cast<size_t>(cs);
+    T = min(max(cu_seqlens[b + 1], cs), T) - cs;
+  }
   const size_t sbase = (static_cast<size_t>(b) * H + h) * DK * DV;
 
   for (int e = tid; e < DK * VS; e += blockDim.x) {
@@ -69,7 +78,7 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
       float g = 1.f;
       for (int r = 0; r < C; ++r) {
         if (r < L) {
-          const size_t th = (static_cast<size_t>(b) * T + t0 + r) * H + h;
+          const size_t th = (tok0 + t0 + r) * H + h;
           g *= gate_at(alpha, alpha_mode, th, DK, tid);
           const float bk = sqrtf(gate_at(beta_k, beta_k_mode, th, DK, tid)) * to_f32(k[th * DK + tid]);
           Bh[r * LDK + tid] = g * bk;
@@ -89,7 +98,7 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
         const int r = e / VS, j = e % VS;
         float w = 0.f;
         if (r < L) {
-          const size_t th = (static_cast<size_t>(b) * T + t0 + r) * H + h;
+          const size_t th = (tok0 + t0 + r) * H + h;
           const float vj = to_f32(v[th * DV + v0 + j]);
           const float ws = (beta_v_mode != MODE_ABSENT) ? gate_at(beta_v, beta_v_mode, th, DV, v0 + j)
                                                         : sqrtf(gate_at(beta_k, beta_k_mode, th, DK, v0 + j));
@@ -170,7 +179,7 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
         for (int jj = 0; jj < PER; ++jj) o1[jj] = fmaf(pv, Wr[m * LV + j0 + jj], o1[jj]);
       }
       if (r < L) {
-        const size_t th = (static_cast<size_t>(b) * T + t0 + r) * H + h;
+        const size_t th = (tok0 + t0 + r) * H + h;
 #pragma unroll
         for (int jj = 0; jj < PER; ++jj) o[th * DV + v0 + j0 + jj] = from_f32<IO>(o1[jj]);
       }

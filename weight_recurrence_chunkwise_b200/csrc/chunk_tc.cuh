@@ -91,6 +91,7 @@ struct Params {
   float *S_T;
   uint32_t *status;
   const float *s = nullptr;  // write-side key scale [B,T,H,dk] (a = s (.) b); only the ring kernel reads it
+  const int *cu_seqlens = nullptr;  // packed batch: sequence b is tokens cu[b] .. cu[b+1]-1 (ring kernel only)
 };
 
 __device__ __forceinline__ void st_h16x8(uint8_t *tile, int row, int col0, int R, const float *v) {

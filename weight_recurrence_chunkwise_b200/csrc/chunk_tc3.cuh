@@ -109,11 +109,21 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase_addr = smem_u32(sm);
 
-  const int T = p.T, H = p.H, DV = p.DV;
+  const int H = p.H, DV = p.DV;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rank = static_cast<int>(cluster_ctarank());  // value slice; equals blockIdx.x
   const int peer = rank ^ 1;
-  const int v0 = rank * VS, h = blockIdx.y, b = blockIdx.z;
+  const int v0 = rank * VS, h = blockIdx.y, b = blockIdx.z;  // b: batch row, or sequence of a packed batch
+  // Token range of this sequence.  Dense batch: tokens b*T .. b*T+T-1 of the [B,T,H,.] arrays, TMA
+  // coordinates (t, b).  Packed batch (cu_seqlens): tokens cu[b] .. cu[b+1]-1 of the [1,Ttot,H,.]
+  // arrays, TMA coordinates (cu[b] + t, 0).  Rows past the sequence end inside a chunk may hold the
+  // next sequence's tokens; they act as identity transitions like the padded rows of a dense batch.
+  // The offsets are clamped to [0, Ttot], so malformed ones cannot address outside the arrays.
+  const int *cu = p.cu_seqlens;
+  const int cs = cu ? min(max(cu[b], 0), p.T) : 0;
+  const int T = cu ? min(max(cu[b + 1], cs), p.T) - cs : p.T;
+  const size_t tok0 = cu ? static_cast<size_t>(cs) : static_cast<size_t>(b) * p.T;
+  const int tt0 = cs, tb = cu ? 0 : b;
   const int nchunks = (T + C - 1) / C;
   const bool sym_channel = p.beta_v_mode == MODE_ABSENT && p.beta_k_mode == MODE_CHANNEL;
   const bool scale_col = p.beta_v_mode == MODE_CHANNEL || sym_channel;  // per-column write scales
@@ -169,10 +179,10 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const int t0 = c * C;
       uint8_t *X = sm + slot_off(c % NSLOT);
       mbar_arrive_expect_tx(&bar_qk, 4 * 64 * 128);
-      tma_load_4d(X + 64 * 128, &tm_q, &bar_qk, 0, h, t0, b);
-      tma_load_4d(X + SX_CB + 64 * 128, &tm_q, &bar_qk, 64, h, t0, b);
-      tma_load_4d(X, &tm_k, &bar_qk, 0, h, t0, b);
-      tma_load_4d(X + SX_CB, &tm_k, &bar_qk, 64, h, t0, b);
+      tma_load_4d(X + 64 * 128, &tm_q, &bar_qk, 0, h, tt0 + t0, tb);
+      tma_load_4d(X + SX_CB + 64 * 128, &tm_q, &bar_qk, 64, h, tt0 + t0, tb);
+      tma_load_4d(X, &tm_k, &bar_qk, 0, h, tt0 + t0, tb);
+      tma_load_4d(X + SX_CB, &tm_k, &bar_qk, 64, h, tt0 + t0, tb);
     };
     // gates of chunk c.  Scalar: staged by cp.async (warp 0, lane l: rows 2l, 2l+1), one own chunk
     // ahead.  Channel: L2 prefetch one own chunk ahead (prefetch_gates), then loaded into registers
@@ -180,7 +190,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // Loads only; masking and broadcast happen at use.
     auto prefetch_gates = [&](int c) {
       const int t0 = c * C, L = min(C, T - t0);
-      const size_t thb = (static_cast<size_t>(b) * T + t0) * H + h;
+      const size_t thb = (tok0 + t0) * H + h;
       if constexpr (kScaled) {  // thread ltid: 128-byte line (ltid & 3) of row (ltid >> 2) of s
         const size_t th = thb + static_cast<size_t>(min(ltid >> 2, L - 1)) * H;
         asm volatile("prefetch.global.L2 [%0];" ::"l"(p.s + th * DK + (ltid & 3) * 32));
@@ -205,7 +215,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     };
     auto load_gates = [&](int c) {  // channel-gate K1 only
       const int t0 = c * C, L = min(C, T - t0);
-      const size_t thb = (static_cast<size_t>(b) * T + t0) * H + h;
+      const size_t thb = (tok0 + t0) * H + h;
 #pragma unroll
       for (int j = 0; j < RGL; ++j) {
         const size_t th = thb + static_cast<size_t>(min(rgl * RGL + j, L - 1)) * H;
@@ -272,8 +282,8 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // the first own chunk uses a slot nobody has touched yet
     auto prefetch_qk_l2 = [&](int c) {
       for (int x = 0; x < DK; x += 64) {
-        tma_prefetch_l2_4d(&tm_q, x, h, c * C, b);
-        tma_prefetch_l2_4d(&tm_k, x, h, c * C, b);
+        tma_prefetch_l2_4d(&tm_q, x, h, tt0 + c * C, tb);
+        tma_prefetch_l2_4d(&tm_k, x, h, tt0 + c * C, tb);
       }
     };
     if (rank < nchunks) {
@@ -318,7 +328,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           for (int i = 0; i < 4; ++i) {
             const int r = min((ltid >> 4) + 16 * i, L - 1);
             const float4 *src = reinterpret_cast<const float4 *>(
-                p.s + ((static_cast<size_t>(b) * T + t0 + r) * H + h) * DK + j8 * 8);
+                p.s + ((tok0 + t0 + r) * H + h) * DK + j8 * 8);
             const float4 lo = __ldg(src), hi = __ldg(src + 1);
             ssc[i][0] = lo.x; ssc[i][1] = lo.y; ssc[i][2] = lo.z; ssc[i][3] = lo.w;
             ssc[i][4] = hi.x; ssc[i][5] = hi.y; ssc[i][6] = hi.z; ssc[i][7] = hi.w;
@@ -414,7 +424,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           const float b0 = s0 * kf.x, b1 = s1 * kf.y;
           float a0 = b0 * __fdividef(1.f, ga), a1 = b1 * __fdividef(1.f, gb);  // a / gamma_r
           if constexpr (kScaled) {
-            const size_t th = (static_cast<size_t>(b) * T + t0 + min(rgl * RGL + jj, L - 1)) * H + h;
+            const size_t th = (tok0 + t0 + min(rgl * RGL + jj, L - 1)) * H + h;
             const float2 sc = __ldg(reinterpret_cast<const float2 *>(p.s + th * DK + c0));
             a0 *= sc.x;
             a1 *= sc.y;
@@ -590,7 +600,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
     auto issue_v = [&](int c) {
       mbar_arrive_expect_tx(&bar_v, 64 * 128);
-      tma_load_4d(tWR, &tm_v, &bar_v, v0, h, c * C, b);
+      tma_load_4d(tWR, &tm_v, &bar_v, v0, h, tt0 + c * C, tb);
     };
     // write scales of row wc of chunk c: one scalar (raw; square root at use if symmetric), or 16
     // per-column values (beta_v, or beta_k of the same channels when the write is symmetric)
@@ -600,7 +610,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     for (int i = 0; i < 16; ++i) psc[i] = 0.f;
     auto prefetch_ws = [&](int c) {
       const int t0 = c * C, L = min(C, T - t0);
-      const size_t th = (static_cast<size_t>(b) * T + t0 + min(wc, L - 1)) * H + h;
+      const size_t th = (tok0 + t0 + min(wc, L - 1)) * H + h;
       if (scale_col) {
         const float *src = (p.beta_v_mode == MODE_CHANNEL ? p.beta_v + th * DV : p.beta_k + th * DK) + v0 + wjb * 8;
 #pragma unroll
@@ -636,7 +646,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       return !fail;
     };
     // write vectors of the chunk whose raw v sits in Wr, in place (after bar_v)
-    auto convert_wr = [&]() {
+    auto convert_wr = [&](int wL) {  // wL: valid rows of the chunk
       float sc[16];
       if (scale_col) {
 #pragma unroll
@@ -655,8 +665,12 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float2 vf = __bfloat1622float2(v2[i]);
-          w8[2 * i] = sc[jj * 8 + 2 * i] * vf.x;  // rows >= L: v = 0 (TMA fill)
+          w8[2 * i] = sc[jj * 8 + 2 * i] * vf.x;
           w8[2 * i + 1] = sc[jj * 8 + 2 * i + 1] * vf.y;
+        }
+        if (wc >= wL) {  // past the sequence end: TMA zero fill, or the next packed sequence's v
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w8[i] = 0.f;
         }
         uint4 out;
         out.x = pack_f16x2(w8[0], w8[1]);
@@ -677,7 +691,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           tmem_ld16(tmem_addr(tmem, quarter * 32, col_d3(c) + half * 32 + j), x);
           tmem_ld_wait();
           if (r < L) {
-            const size_t th = (static_cast<size_t>(b) * T + t0 + r) * H + h;
+            const size_t th = (tok0 + t0 + r) * H + h;
             IO *dst = static_cast<IO *>(p.o) + th * DV + v0 + half * 32 + j;
             uint4 lo, hi;
             lo.x = pack_bf16x2(x[0], x[1]);
@@ -719,7 +733,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (nchunks > 0) {
       if (ct == 0) {
         issue_v(0);
-        for (int c = 1; c < 3 && c < nchunks; ++c) tma_prefetch_l2_4d(&tm_v, v0, h, c * C, b);
+        for (int c = 1; c < 3 && c < nchunks; ++c) tma_prefetch_l2_4d(&tm_v, v0, h, tt0 + c * C, tb);
       }
       prefetch_ws(0);
     }
@@ -737,7 +751,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // group barrier decides both waits and orders the conversion before the MMAs
         const bool ok_v = mbar_wait(&bar_v, ph_v & 1u, kWaitLimitNs);
         ph_v ^= 1u;
-        if (ok_v) convert_wr();
+        if (ok_v) convert_wr(min(C, T - c * C));
         fence_async_smem();
         const bool ok_f = mbar_wait_cluster(&bar_full[j], (ph_full >> j) & 1u, kWaitLimitNs);
         ph_full ^= 1u << j;
@@ -791,7 +805,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       }
       if (ct == 128) {
         if (c + 1 < nchunks) issue_v(c + 1);  // Wr is free
-        if (c + 3 < nchunks) tma_prefetch_l2_4d(&tm_v, v0, h, (c + 3) * C, b);
+        if (c + 3 < nchunks) tma_prefetch_l2_4d(&tm_v, v0, h, tt0 + (c + 3) * C, tb);
       }
       if (c + 1 < nchunks) prefetch_ws(c + 1);
 

@@ -76,9 +76,9 @@ dr_status launch_status() {
 
 // ----------------------------------------------------------------- prefill, CUDA-core path
 template <typename IO, int DK, int DV, int C>
-dr_status simt_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                      const float *beta_k, const float *beta_v, const float *s_scale, const float *S0, void *o,
-                      float *S_T, uint32_t *status, cudaStream_t st) {
+dr_status simt_launch(const dr_problem *p, const int *cu, const void *q, const void *k, const void *v,
+                      const float *alpha, const float *beta_k, const float *beta_v, const float *s_scale,
+                      const float *S0, void *o, float *S_T, uint32_t *status, cudaStream_t st) {
   constexpr int VS = 32;
   auto kern = dr::chunk_fwd_simt_kernel<IO, DK, DV, VS, C>;
   constexpr size_t smem = dr::SimtSmem<DK, VS, C>::bytes;
@@ -88,32 +88,35 @@ dr_status simt_launch(const dr_problem *p, const void *q, const void *k, const v
   dim3 grid(DV / VS, p->H, p->B);
   kern<<<grid, 256, smem, st>>>(p->T, p->H, static_cast<const IO *>(q), static_cast<const IO *>(k),
                                 static_cast<const IO *>(v), alpha, p->alpha_mode, beta_k, p->beta_k_mode,
-                                beta_v, p->beta_v_mode, s_scale, S0, static_cast<IO *>(o), S_T, status);
+                                beta_v, p->beta_v_mode, s_scale, cu, S0, static_cast<IO *>(o), S_T, status);
   return launch_status();
 }
 
 template <typename IO, int DK, int DV>
-dr_status simt_by_chunk(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                        const float *beta_k, const float *beta_v, const float *s_scale, const float *S0, void *o,
-                        float *S_T, uint32_t *status, cudaStream_t st) {
+dr_status simt_by_chunk(const dr_problem *p, const int *cu, const void *q, const void *k, const void *v,
+                        const float *alpha, const float *beta_k, const float *beta_v, const float *s_scale,
+                        const float *S0, void *o, float *S_T, uint32_t *status, cudaStream_t st) {
   switch (p->chunk) {
-    case 16: return simt_launch<IO, DK, DV, 16>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
-    case 32: return simt_launch<IO, DK, DV, 32>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
-    default: return simt_launch<IO, DK, DV, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+    case 16:
+      return simt_launch<IO, DK, DV, 16>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+    case 32:
+      return simt_launch<IO, DK, DV, 32>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+    default:
+      return simt_launch<IO, DK, DV, 64>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
   }
 }
 
 template <typename IO>
-dr_status simt_dispatch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                        const float *beta_k, const float *beta_v, const float *s_scale, const float *S0, void *o,
-                        float *S_T, uint32_t *status, cudaStream_t st) {
+dr_status simt_dispatch(const dr_problem *p, const int *cu, const void *q, const void *k, const void *v,
+                        const float *alpha, const float *beta_k, const float *beta_v, const float *s_scale,
+                        const float *S0, void *o, float *S_T, uint32_t *status, cudaStream_t st) {
   if (p->dk == 128 && p->dv == 128)
-    return simt_by_chunk<IO, 128, 128>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+    return simt_by_chunk<IO, 128, 128>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
   if (p->dk == 128 && p->dv == 64)
-    return simt_by_chunk<IO, 128, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+    return simt_by_chunk<IO, 128, 64>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
   if (p->dk == 64 && p->dv == 128)
-    return simt_by_chunk<IO, 64, 128>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
-  return simt_by_chunk<IO, 64, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+    return simt_by_chunk<IO, 64, 128>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+  return simt_by_chunk<IO, 64, 64>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
 }
 
 // ----------------------------------------------------------------- prefill, tensor-core path (bf16 I/O)
@@ -219,21 +222,22 @@ dr_status tc_pair_launch(const dr_problem *p, const void *q, const void *k, cons
   return launch_status();
 }
 
-dr_status tc_ring_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                         const float *beta_k, const float *beta_v, const float *s_scale, const float *S0, void *o,
-                         float *S_T, uint32_t *status, cudaStream_t st) {
+dr_status tc_ring_launch(const dr_problem *p, const int *cu, const void *q, const void *k, const void *v,
+                         const float *alpha, const float *beta_k, const float *beta_v, const float *s_scale,
+                         const float *S0, void *o, float *S_T, uint32_t *status, cudaStream_t st) {
   using IO = __nv_bfloat16;
   namespace tc = dr::tc;
   namespace tc3 = dr::tc3;
   alignas(64) CUtensorMap mq, mk, mv;
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
-  if (!make_map(&mq, bf, 2, q, p->B, p->T, p->H, p->dk, 64, tc::C, sw) ||
-      !make_map(&mk, bf, 2, k, p->B, p->T, p->H, p->dk, 64, tc::C, sw) ||
-      !make_map(&mv, bf, 2, v, p->B, p->T, p->H, p->dv, tc::VS, tc::C, sw))
+  const int mB = cu ? 1 : p->B;  // a packed batch is one [1, Ttot, H, d] array
+  if (!make_map(&mq, bf, 2, q, mB, p->T, p->H, p->dk, 64, tc::C, sw) ||
+      !make_map(&mk, bf, 2, k, mB, p->T, p->H, p->dk, 64, tc::C, sw) ||
+      !make_map(&mv, bf, 2, v, mB, p->T, p->H, p->dv, tc::VS, tc::C, sw))
     return DR_ERR_CUDA;
   tc::Params prm{p->T, p->H, p->dv, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v, p->beta_v_mode,
-                 S0, o, S_T, status, s_scale};
+                 S0, o, S_T, status, s_scale, cu};
   const bool chan_gates = p->alpha_mode == DR_CHANNEL || p->beta_k_mode != DR_SCALAR;
   auto kern = s_scale ? (chan_gates ? tc3::chunk_fwd_ring_kernel<IO, true, true>
                                     : tc3::chunk_fwd_ring_kernel<IO, false, true>)
@@ -285,10 +289,12 @@ dr_status decode_dispatch(const dr_problem *p, const void *q, const void *k, con
   return decode_launch<IO, 64, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
 }
 
-// Prefill with an optional write-side key scale (NULL: a = b).
-dr_status chunk_fwd_impl(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                         const float *beta_k, const float *beta_v, const float *s_scale, const float *S0, void *o,
-                         float *S_T, void *workspace, size_t workspace_bytes, void *stream) {
+// Prefill with an optional write-side key scale (NULL: a = b) and optional packed-sequence offsets
+// (NULL: a dense [B, T, H, d] batch).
+dr_status chunk_fwd_impl(const dr_problem *p, const int *cu, const void *q, const void *k, const void *v,
+                         const float *alpha, const float *beta_k, const float *beta_v, const float *s_scale,
+                         const float *S0, void *o, float *S_T, void *workspace, size_t workspace_bytes,
+                         void *stream) {
   dr_status s = check_common(p, false);
   if (s != DR_OK) return s;
   s = check_pointers(p, q, k, v, alpha, beta_k, beta_v, o);
@@ -309,15 +315,16 @@ dr_status chunk_fwd_impl(const dr_problem *p, const void *q, const void *k, cons
     return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
   }
   if (p->io_dtype == DR_F32)
-    return simt_dispatch<float>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+    return simt_dispatch<float>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
   const bool ring_shape = p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv == 2 * dr::tc::VS;
-  if (ring_shape && (s_scale || prefill_kernel() == kRing))
-    return tc_ring_launch(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
-  if (!s_scale && ring_shape && prefill_kernel() == kPair)
+  const bool plain = !s_scale && !cu;  // the older kernels take neither extension
+  if (ring_shape && (!plain || prefill_kernel() == kRing))
+    return tc_ring_launch(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+  if (plain && ring_shape && prefill_kernel() == kPair)
     return tc_pair_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
-  if (!s_scale && p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv % dr::tc::VS == 0)
+  if (plain && p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv % dr::tc::VS == 0)
     return tc_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
-  return simt_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+  return simt_dispatch<__nv_bfloat16>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
 }
 
 dr_status decode_step_impl(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
@@ -361,13 +368,25 @@ size_t dr_chunk_fwd_workspace(const dr_problem *p) {
 dr_status dr_chunk_fwd(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
                        const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
                        void *workspace, size_t workspace_bytes, void *stream) {
-  return chunk_fwd_impl(p, q, k, v, alpha, beta_k, beta_v, nullptr, S0, o, S_T, workspace, workspace_bytes, stream);
+  return chunk_fwd_impl(p, nullptr, q, k, v, alpha, beta_k, beta_v, nullptr, S0, o, S_T, workspace, workspace_bytes,
+                        stream);
 }
 
 dr_status dr_chunk_fwd_osdn(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
                             const float *beta_k, const float *beta_v, const float *s, const float *S0, void *o,
                             float *S_T, void *workspace, size_t workspace_bytes, void *stream) {
-  return chunk_fwd_impl(p, q, k, v, alpha, beta_k, beta_v, s, S0, o, S_T, workspace, workspace_bytes, stream);
+  return chunk_fwd_impl(p, nullptr, q, k, v, alpha, beta_k, beta_v, s, S0, o, S_T, workspace, workspace_bytes,
+                        stream);
+}
+
+dr_status dr_chunk_fwd_varlen(const dr_problem *p, const int *cu_seqlens, const void *q, const void *k,
+                              const void *v, const float *alpha, const float *beta_k, const float *beta_v,
+                              const float *s, const float *S0, void *o, float *S_T, void *workspace,
+                              size_t workspace_bytes, void *stream) {
+  if (!cu_seqlens) return DR_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return DR_ERR_ALIGNMENT;
+  return chunk_fwd_impl(p, cu_seqlens, q, k, v, alpha, beta_k, beta_v, s, S0, o, S_T, workspace,
+                        workspace_bytes, stream);
 }
 
 dr_status dr_decode_step(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
