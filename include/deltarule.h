@@ -181,6 +181,22 @@ DR_API dr_status dr_chunk_fwd_varlen(const dr_problem *p, const int *cu_seqlens,
                                      void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Affine state maps, for a sequence split into consecutive segments (NEXT-4
+ * of the build plan; the chunkwise form's linearity in the state, DeltaNet
+ * page step 7 / FG2-GDN page section 2).  A segment maps its initial state to
+ * its final state as S_out = M S_in + N: N is the segment's final state from a
+ * zero initial state (dr_chunk_fwd with S0 = NULL), and M (dk x dk) its final
+ * state when the write vectors are zero and S0 = I (dr_chunk_fwd with v = 0,
+ * beta_v = NULL and dv = dk).  This call applies such maps to n independent
+ * heads:  out_h = M_h S_h + N_h.
+ *   M   [n, dk, dk] fp32;  S [n, dk, dv] fp32 or NULL (zero);  N, out [n, dk, dv] fp32
+ *   dk in {64, 128}, dv a multiple of 32, n <= 65535; all 16-byte aligned device
+ *   pointers; out may be N but not S.  Asynchronous on `stream`.
+ */
+DR_API dr_status dr_state_map_apply(int n, int dk, int dv, const float *M, const float *S, const float *N,
+                                    float *out, void *stream);
+
+/*
  * dr_chunk_fwd for callers that cannot allocate device memory.  (The pages
  * have no counterpart; this is a deployment variant of dr_chunk_fwd.)  Some
  * hosts pre-plan every byte of device memory and give a kernel no workspace

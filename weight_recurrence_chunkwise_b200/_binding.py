@@ -40,7 +40,7 @@ _lib = None
 
 EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_chunk_fwd_osdn", "dr_chunk_fwd_varlen",
            "dr_chunk_fwd_noalloc", "dr_decode_step",
-           "dr_decode_step_osdn",
+           "dr_decode_step_osdn", "dr_state_map_apply",
            "dr_workspace_status", "dr_status_string", "dr_version", "dr_diag_umma_selftest",
            "dr_diag_tri_inverse")
 
@@ -65,6 +65,8 @@ def lib():
         L.dr_chunk_fwd_osdn.restype = ctypes.c_int
         L.dr_chunk_fwd_varlen.argtypes = [P] + [vp] * 11 + [vp, sz, vp]
         L.dr_chunk_fwd_varlen.restype = ctypes.c_int
+        L.dr_state_map_apply.argtypes = [ctypes.c_int] * 3 + [vp] * 5
+        L.dr_state_map_apply.restype = ctypes.c_int
         L.dr_decode_step_osdn.argtypes = [P] + [vp] * 9 + [vp]
         L.dr_decode_step_osdn.restype = ctypes.c_int
         L.dr_workspace_status.argtypes = [vp, vp]
@@ -258,6 +260,23 @@ def _decode_step(s, q, k, v, beta_k, S, alpha, beta_v, o, stream):
     if rc != DR_OK:
         raise DeltaRuleError(rc, name)
     return o
+
+
+def dr_state_map_apply(M, N, S=None, out=None, stream=None):
+    """out = M @ S + N per head (S None: zero).  M [..., dk, dk], S / N / out [..., dk, dv], fp32 CUDA."""
+    dk, dv = N.shape[-2], N.shape[-1]
+    n = N.numel() // (dk * dv)
+    if out is None:
+        out = torch.empty_like(N)
+    for name, t in (("M", M), ("N", N), ("S", S), ("out", out)):
+        if t is not None and (not t.is_cuda or not t.is_contiguous() or t.dtype != torch.float32):
+            raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor")
+    if M.numel() != n * dk * dk or (S is not None and S.shape != N.shape) or out.shape != N.shape:
+        raise ValueError("shapes: M [n, dk, dk], S / N / out [n, dk, dv]")
+    rc = lib().dr_state_map_apply(n, dk, dv, _ptr(M), _ptr(S), _ptr(N), _ptr(out), _stream(stream))
+    if rc != DR_OK:
+        raise DeltaRuleError(rc, "dr_state_map_apply")
+    return out
 
 
 def dr_workspace_status(workspace, stream=None) -> int:

@@ -17,6 +17,7 @@
 #include "chunk_tc3.cuh"
 #include "common.cuh"
 #include "decode.cuh"
+#include "state_map.cuh"
 #include "umma_selftest.cuh"
 
 namespace {
@@ -377,6 +378,23 @@ dr_status dr_chunk_fwd_osdn(const dr_problem *p, const void *q, const void *k, c
                             float *S_T, void *workspace, size_t workspace_bytes, void *stream) {
   return chunk_fwd_impl(p, nullptr, q, k, v, alpha, beta_k, beta_v, s, S0, o, S_T, workspace, workspace_bytes,
                         stream);
+}
+
+dr_status dr_state_map_apply(int n, int dk, int dv, const float *M, const float *S, const float *N, float *out,
+                             void *stream) {
+  if (n < 0 || (dk != 64 && dk != 128) || dv <= 0 || dv % 32 != 0) return DR_ERR_INVALID_ARG;
+  if (n == 0) return DR_OK;
+  if (!M || !N || !out) return DR_ERR_INVALID_ARG;
+  if (S && S == out) return DR_ERR_INVALID_ARG;  // S is read by other threads while out is written
+  if (!aligned16(M) || !aligned16(N) || !aligned16(out) || (S && !aligned16(S))) return DR_ERR_ALIGNMENT;
+  if (n > 65535) return DR_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid(dv / 32, n);
+  if (dk == 128)
+    dr::state_map_apply_kernel<128><<<grid, 256, 0, st>>>(dv, M, S, N, out);
+  else
+    dr::state_map_apply_kernel<64><<<grid, 256, 0, st>>>(dv, M, S, N, out);
+  return launch_status();
 }
 
 dr_status dr_chunk_fwd_varlen(const dr_problem *p, const int *cu_seqlens, const void *q, const void *k,
