@@ -265,6 +265,44 @@ def run_decode_only(args, dr, dev, st, ws):
     return 0
 
 
+def backward_bytes(p):
+    """Algorithmic HBM bytes of one backward: q, k, v, dout, gates, S0, dS_T read; fp32 gradients written."""
+    io = 2 if p.io == "bf16" else 4
+    gate = lambda m, w: {"none": 0, "scalar": 4, "channel": 4 * w}[m]
+    per_in = io * (2 * p.dk + 2 * p.dv) + gate(p.alpha, p.dk) + gate(p.beta_k, p.dk) + gate(p.beta_v, p.dv)
+    per_out = 4 * (2 * p.dk + p.dv) + gate(p.alpha, p.dk) + gate(p.beta_k, p.dk) + gate(p.beta_v, p.dv)
+    state = p.B * p.H * p.dk * p.dv * 4
+    return p.token_heads * (per_in + per_out) + 3 * state
+
+
+def run_backward(args, dr, p, x, dev, st, peaks, peaks_src):
+    """Profiling aid: the backward pass alone on one workload (warm-up, then timed launches)."""
+    g = torch.Generator().manual_seed(p.seed)
+    dout = torch.randn(x["v"].shape, generator=g).to(x["v"].dtype).to(dev)
+    S0 = torch.zeros((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=dev)
+    dST = torch.randn((p.B, p.H, p.dk, p.dv), generator=g).to(dev)
+    run = lambda: dr.dr_backward(x["q"], x["k"], x["v"], x["beta_k"], dout, alpha=x["alpha"], beta_v=x["beta_v"],
+                                 S0=S0, dS_T=dST, stream=st)
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        run()
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    byts = backward_bytes(p)
+    gbs = byts / (ms / 1e3) / 1e9
+    print(json.dumps({"backward": True, "workload": p.name, "ms": ms,
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                   "frac": gbs / peaks["hbm_gbs"], "peak_source": peaks_src,
+                                   "kernel": "delta_rule_bwd_kernel", "algorithmic_bytes_per_launch": byts}}),
+          flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- our arm
 def main():
     ap = argparse.ArgumentParser()
@@ -279,7 +317,9 @@ def main():
     ap.add_argument("--only-decode", action="store_true",
                     help="profiling aid: time only the decode workload")
     ap.add_argument("--config", default=WORKLOAD, choices=list(CONFIGS),
-                    help="with --only-prefill: the prefill workload to time (default: the headline one)")
+                    help="with --only-prefill / --backward: the workload to time (default: the headline one)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (dr_backward) on the --config workload instead")
     args = ap.parse_args()
     ws, rank, local = dist_env()
     if args.impl == "reference":
@@ -298,8 +338,10 @@ def main():
     st = torch.cuda.current_stream()
 
     # ---------------- prefill -> decode step workload (every rank its own seeded batch)
-    p = rank_problem(rank, args.config if args.only_prefill else WORKLOAD)
+    p = rank_problem(rank, args.config if (args.only_prefill or args.backward) else WORKLOAD)
     x = to_dev(make_inputs(p), dev)
+    if args.backward:
+        return run_backward(args, dr, p, x, dev, st, peaks, peaks_src)
     nxt = to_dev(make_inputs(p.replace(T=1, seed=p.seed + 500)), dev)  # the token after the prompt
     o = torch.empty_like(x["v"])
     S = torch.empty((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=dev)

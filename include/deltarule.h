@@ -197,6 +197,38 @@ DR_API dr_status dr_state_map_apply(int n, int dk, int dv, const float *M, const
                                     float *out, void *stream);
 
 /*
+ * Backward pass (NEXT-3 of the build plan): the gradients of
+ *   L = sum(dout (.) o) + sum(dS_T (.) S_T)
+ * with respect to every input of dr_chunk_fwd / dr_chunk_fwd_osdn, for the
+ * forward defined by the recurrence (DeltaNet page steps 3-6; FG2-GDN page
+ * section 2; OSDN summary "Method").  Reverse mode through
+ *   X = Diag(alpha_t) S_{t-1},  u = w_t - X^T b_t,  S_t = X + a_t u^T,  o_t = S_t^T q_t.
+ * The pass recomputes the forward itself (it keeps the state every 32 tokens in
+ * the workspace and re-derives the states in between), so it takes the
+ * forward's inputs, not its outputs.
+ *   inputs   as dr_chunk_fwd_osdn (s may be NULL); p->chunk is ignored
+ *   dout     [B,T,H,dv] in the I/O dtype;  dS_T [B,H,dk,dv] fp32 or NULL (zero)
+ *   outputs  fp32, caller owned, overwritten:
+ *            dq, dk [B,T,H,dk];  dv [B,T,H,dv];
+ *            dalpha, dbeta_k, dbeta_v, ds in the shape of alpha, beta_k, beta_v, s
+ *            (each non-NULL exactly when its input is given; dbeta_k always);
+ *            dS0 [B,H,dk,dv] or NULL (not wanted).  A gate's gradient at beta = 0
+ *            is reported as 0 (the square root has no derivative there).
+ *   workspace >= dr_backward_workspace(p) bytes, 16-byte aligned, device memory
+ *            (fp32 state checkpoints and per-head recomputation scratch).
+ * dk, dv in {64, 128}; fp32 or bf16 I/O.  Asynchronous on `stream`.  Errors as
+ * dr_chunk_fwd, plus DR_ERR_INVALID_ARG for a missing or extra gradient buffer.
+ */
+DR_API size_t dr_backward_workspace(const dr_problem *p);
+DR_API dr_status dr_backward(const dr_problem *p,
+                             const void *q, const void *k, const void *v,
+                             const float *alpha, const float *beta_k, const float *beta_v,
+                             const float *s, const float *S0, const void *dout, const float *dS_T,
+                             float *dq, float *dk, float *dv, float *dalpha, float *dbeta_k,
+                             float *dbeta_v, float *ds, float *dS0,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * dr_chunk_fwd for callers that cannot allocate device memory.  (The pages
  * have no counterpart; this is a deployment variant of dr_chunk_fwd.)  Some
  * hosts pre-plan every byte of device memory and give a kernel no workspace

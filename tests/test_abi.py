@@ -21,6 +21,18 @@ def _declared_symbols():
     return names
 
 
+def _declared_arity():
+    """Parameter count of every DR_API function, from the headers."""
+    out = {}
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", f)).read()
+            for name, params in re.findall(r"DR_API\s+[\w\s\*]+?\b(dr_\w+)\s*\(([^)]*)\)", txt):
+                params = params.strip()
+                out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
 @pytest.fixture(scope="module")
 def lib():
     from weight_recurrence_chunkwise_b200 import build
@@ -36,6 +48,14 @@ def test_every_declared_symbol_is_exported(lib):
     for n in names:
         assert hasattr(lib, n), f"{n} declared but not exported"
     assert set(B.EXPORTS) == names
+
+
+def test_binding_argument_counts_match_the_headers(lib):
+    """Every ctypes prototype the binding sets up has the declared number of parameters."""
+    arity = _declared_arity()
+    assert set(arity) == set(B.EXPORTS)
+    for name, n in arity.items():
+        assert len(getattr(lib, name).argtypes) == n, (name, len(getattr(lib, name).argtypes), n)
 
 
 def test_version_and_status_strings(lib):

@@ -40,7 +40,7 @@ _lib = None
 
 EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_chunk_fwd_osdn", "dr_chunk_fwd_varlen",
            "dr_chunk_fwd_noalloc", "dr_decode_step",
-           "dr_decode_step_osdn", "dr_state_map_apply",
+           "dr_decode_step_osdn", "dr_state_map_apply", "dr_backward_workspace", "dr_backward",
            "dr_workspace_status", "dr_status_string", "dr_version", "dr_diag_umma_selftest",
            "dr_diag_tri_inverse")
 
@@ -67,6 +67,10 @@ def lib():
         L.dr_chunk_fwd_varlen.restype = ctypes.c_int
         L.dr_state_map_apply.argtypes = [ctypes.c_int] * 3 + [vp] * 5
         L.dr_state_map_apply.restype = ctypes.c_int
+        L.dr_backward_workspace.argtypes = [P]
+        L.dr_backward_workspace.restype = sz
+        L.dr_backward.argtypes = [P] + [vp] * 18 + [vp, sz, vp]
+        L.dr_backward.restype = ctypes.c_int
         L.dr_decode_step_osdn.argtypes = [P] + [vp] * 9 + [vp]
         L.dr_decode_step_osdn.restype = ctypes.c_int
         L.dr_workspace_status.argtypes = [vp, vp]
@@ -277,6 +281,33 @@ def dr_state_map_apply(M, N, S=None, out=None, stream=None):
     if rc != DR_OK:
         raise DeltaRuleError(rc, "dr_state_map_apply")
     return out
+
+
+def dr_backward(q, k, v, beta_k, dout, alpha=None, beta_v=None, s=None, S0=None, dS_T=None, want_dS0=True,
+                workspace=None, stream=None):
+    """Gradients of sum(dout * o) + sum(dS_T * S_T) w.r.t. the forward's inputs (fp32 tensors).
+
+    Returns a dict with keys q, k, v, beta_k, alpha, beta_v, s, S0 (None where absent / not wanted).
+    """
+    p = make_problem(q, v, alpha, beta_k, beta_v, 64)
+    dev = q.device
+    f32 = lambda t: None if t is None else torch.empty(t.shape, dtype=torch.float32, device=dev)
+    g = {"q": f32(q), "k": f32(k), "v": f32(v), "alpha": f32(alpha), "beta_k": f32(beta_k), "beta_v": f32(beta_v),
+         "s": f32(s), "S0": torch.empty((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=dev) if want_dS0 else None}
+    _check_tensors(q.dtype, [("q", q), ("k", k), ("v", v), ("o", dout), ("alpha", alpha), ("beta_k", beta_k),
+                             ("beta_v", beta_v), ("s", s), ("S0", S0), ("S_T", dS_T)])
+    if s is not None and tuple(s.shape) != tuple(q.shape):
+        raise ValueError("s must have the shape of q / k")
+    need = int(lib().dr_backward_workspace(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    rc = lib().dr_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k), _ptr(beta_v),
+                           _ptr(s), _ptr(S0), _ptr(dout), _ptr(dS_T), _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]),
+                           _ptr(g["alpha"]), _ptr(g["beta_k"]), _ptr(g["beta_v"]), _ptr(g["s"]), _ptr(g["S0"]),
+                           _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if rc != DR_OK:
+        raise DeltaRuleError(rc, "dr_backward")
+    return g
 
 
 def dr_workspace_status(workspace, stream=None) -> int:

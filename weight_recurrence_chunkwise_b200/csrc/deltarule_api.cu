@@ -18,6 +18,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "state_map.cuh"
+#include "backward.cuh"
 #include "umma_selftest.cuh"
 
 namespace {
@@ -342,9 +343,71 @@ dr_status decode_step_impl(const dr_problem *p, const void *q, const void *k, co
   return decode_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
 }
 
+constexpr int kBwdSpan = 32;  // tokens between the backward pass's state checkpoints
+
+size_t bwd_workspace_bytes(const dr_problem *p) {
+  const size_t nck = (static_cast<size_t>(p->T) + kBwdSpan - 1) / kBwdSpan;
+  return sizeof(float) * static_cast<size_t>(p->B) * p->H * (nck + kBwdSpan) * p->dk * p->dv;
+}
+
+template <typename IO, int DK, int DV>
+dr_status bwd_launch(const dr::BwdParams &bp, int heads, cudaStream_t st) {
+  dr::delta_rule_bwd_kernel<IO, DK, DV, kBwdSpan><<<heads, 256, 0, st>>>(bp);
+  return launch_status();
+}
+
+template <typename IO>
+dr_status bwd_dispatch(const dr_problem *p, const dr::BwdParams &bp, cudaStream_t st) {
+  const int heads = p->B * p->H;
+  if (p->dk == 128 && p->dv == 128) return bwd_launch<IO, 128, 128>(bp, heads, st);
+  if (p->dk == 128 && p->dv == 64) return bwd_launch<IO, 128, 64>(bp, heads, st);
+  if (p->dk == 64 && p->dv == 128) return bwd_launch<IO, 64, 128>(bp, heads, st);
+  return bwd_launch<IO, 64, 64>(bp, heads, st);
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t dr_backward_workspace(const dr_problem *p) {
+  return check_common(p, false) == DR_OK ? bwd_workspace_bytes(p) : 0;
+}
+
+dr_status dr_backward(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                      const float *beta_k, const float *beta_v, const float *s, const float *S0, const void *dout,
+                      const float *dS_T, float *dq, float *dk, float *dv, float *dalpha, float *dbeta_k,
+                      float *dbeta_v, float *ds, float *dS0, void *workspace, size_t workspace_bytes,
+                      void *stream) {
+  dr_status st = check_common(p, false);
+  if (st != DR_OK) return st;
+  st = check_pointers(p, q, k, v, alpha, beta_k, beta_v, dout);
+  if (st != DR_OK) return st;
+  const bool need = p->T > 0;
+  if (need && (!dq || !dk || !dv || !dbeta_k)) return DR_ERR_INVALID_ARG;
+  if (need && ((dalpha == nullptr) != (alpha == nullptr))) return DR_ERR_INVALID_ARG;
+  if (need && ((dbeta_v == nullptr) != (beta_v == nullptr))) return DR_ERR_INVALID_ARG;
+  if (need && ((ds == nullptr) != (s == nullptr))) return DR_ERR_INVALID_ARG;
+  const void *ptrs[] = {s, S0, dS_T, dq, dk, dv, dalpha, dbeta_k, dbeta_v, ds, dS0, workspace};
+  for (const void *x : ptrs)
+    if (x && !aligned16(x)) return DR_ERR_ALIGNMENT;
+  if (static_cast<long long>(p->B) * p->H > 0x7fffffffLL) return DR_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const size_t state_bytes = sizeof(float) * size_t(p->B) * p->H * p->dk * p->dv;
+  if (p->T == 0) {  // nothing to differentiate but the identity S_T = S0
+    if (!dS0) return DR_OK;
+    const cudaError_t e = dS_T ? cudaMemcpyAsync(dS0, dS_T, state_bytes, cudaMemcpyDeviceToDevice, cs)
+                               : cudaMemsetAsync(dS0, 0, state_bytes, cs);
+    return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+  }
+  if (!workspace || workspace_bytes < bwd_workspace_bytes(p)) return DR_ERR_WORKSPACE;
+  float *ws = static_cast<float *>(workspace);
+  const size_t nck = (static_cast<size_t>(p->T) + kBwdSpan - 1) / kBwdSpan;
+  dr::BwdParams bp{p->T, p->H, q, k, v, dout, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v,
+                   p->beta_v_mode, s, S0, dS_T, dq, dk, dv, dalpha, dbeta_k, dbeta_v, ds, dS0, ws,
+                   ws + static_cast<size_t>(p->B) * p->H * nck * p->dk * p->dv};
+  if (p->io_dtype == DR_F32) return bwd_dispatch<float>(p, bp, cs);
+  return bwd_dispatch<__nv_bfloat16>(p, bp, cs);
+}
 
 int dr_version(void) { return 100; }
 
