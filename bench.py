@@ -204,9 +204,16 @@ def cpu_oracle_sample(p, seconds=12.0):
                                  S0=x["S0"], threads=threads)
     dt = time.perf_counter() - t0
     th = x["q"].shape[0] * x["q"].shape[1] * x["q"].shape[2]
+    # one thread on one whole head, for the per-core rate
+    x1 = {k: (None if t is None else (t[:1, :, :1] if k != "S0" else t[:1, :1])) for k, t in x.items()}
+    t1 = time.perf_counter()
+    oracle.delta_rule_sequential(x1["q"], x1["k"], x1["v"], x1["beta_k"], alpha=x1["alpha"], beta_v=x1["beta_v"],
+                                 S0=x1["S0"], threads=1)
+    dt1 = time.perf_counter() - t1
     return {"value": th / dt / 1e6, "unit": "Mtokens·heads/s", "cores": threads, "kind": "oracle",
+            "hardware_concurrency": os.cpu_count(), "single_thread_value": p.T / dt1 / 1e6,
             "sample": f"{x['q'].shape[0] * x['q'].shape[2]} whole heads x T={p.T} of the {p.name} workload, float64, "
-                      f"{threads} OpenMP threads, {dt:.2f} s"}
+                      f"{threads} OpenMP threads, {dt:.2f} s; single thread: one head, {dt1:.2f} s"}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -434,7 +441,37 @@ def main():
     dms = max_over_ranks(e0.elapsed_time(e1), ws, dev) / args.decode_steps
     dbytes = decode_bytes(DECODE.B, DECODE.H, DECODE.dk, DECODE.dv)
     dgbs = dbytes / (dms / 1e3) / 1e9
+
+    # the same chained steps captured in a CUDA graph (one pool cycle per graph) and replayed
+    cap = torch.cuda.Stream()
+    cap.wait_stream(st)
+
+    def dstep_on(i, stream):
+        j = i % DECODE.pool
+        dr.dr_decode_step(pool["q"][j], pool["k"][j], pool["v"][j], pool["beta_k"][j], S_dec, alpha=pool["alpha"][j],
+                          o=o_dec, stream=stream)
+
+    with torch.cuda.stream(cap):
+        for i in range(3):
+            dstep_on(i, cap)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cap):
+        for i in range(DECODE.pool):
+            dstep_on(i, cap)
+    reps = max(1, args.decode_steps // DECODE.pool)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0.record(st)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(st)
+    torch.cuda.synchronize()
+    dms_graph = max_over_ranks(e0.elapsed_time(e1), ws, dev) / (reps * DECODE.pool)
+    del graph
     decode = {"value": dgbs * ws, "unit": "GB/s", "ms_per_step": dms, "steps": args.decode_steps,
+              "graph": {"ms_per_step": dms_graph, "GB/s": dbytes / (dms_graph / 1e3) / 1e9 * ws,
+                        "steps": reps * DECODE.pool},
               "config": {"workload": DECODE.name, "B": DECODE.B, "H": DECODE.H, "dk": DECODE.dk, "dv": DECODE.dv,
                          "state_MiB": DECODE.B * DECODE.H * DECODE.dk * DECODE.dv * 4 / 2 ** 20},
               "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
