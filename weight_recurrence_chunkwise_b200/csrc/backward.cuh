@@ -12,15 +12,19 @@
 // then the chain rule through b = sqrt(beta_k) (.) k, a = s (.) b and
 // w = beta_v (.) v or sqrt(beta_k) (.) v.
 //
-// One CTA of 256 threads walks one (b, h).  It needs S_{t-1} at every step, so it keeps the
-// forward's state every CK tokens (checkpoints, in the workspace) and, for each span of CK tokens
-// from the last, recomputes the span's states into a per-head scratch and walks the span
-// backwards.  State, adjoint and scratch are fp32; each step is two cross-row reductions through
-// shared memory and four row reductions over the lanes of a warp.  Thread layout as in the decode
-// step: warp w owns rows w, w+8, ...; lane l owns DV/32 consecutive columns.
+// The value columns of S never mix, forward or backward (u_j, S[:, j] and G[:, j] involve column j
+// only), so one CTA of 256 threads walks one (b, h) and one slice of VSB value columns.  It needs
+// S_{t-1} at every step, so it keeps the forward's state every CK tokens (checkpoints, in the
+// workspace) and, for each span of CK tokens from the last, recomputes the span's states into a
+// per-(head, slice) scratch and walks the span backwards.  State, adjoint and scratch are fp32;
+// each step is two cross-row reductions through shared memory and four row reductions over the
+// lanes of a warp.  Thread layout as in the decode step: warp w owns rows w, w+8, ...; lane l owns
+// VSB/32 consecutive columns of the slice.  Per-row gradients (dq, dk, ds, dalpha, dbeta_k) sum
+// over the value columns, so each slice adds its part with atomics into outputs zeroed first;
+// per-column gradients (dv, dbeta_v) are written by their slice.
 //
-// This is a correct, memory- and latency-bound first implementation of the backward: two
-// sequential passes over T per head, with 2*CK*dk*dv*4 bytes of scratch traffic per span.
+// A correct, memory- and latency-bound implementation: two sequential passes over T per
+// (head, slice), with 2*CK*dk*VSB*4 bytes of scratch traffic per span.
 #pragma once
 #include "common.cuh"
 
@@ -41,14 +45,15 @@ struct BwdParams {
   float *dq, *dk, *dv;  // [B,T,H,d] fp32
   float *dalpha, *dbeta_k, *dbeta_v, *ds;  // gate shapes, fp32 (nullptr where the input is absent)
   float *dS0;           // [B,H,dk,dv] fp32 or nullptr
-  float *ckpt;          // [B*H][ceil(T/CK)][dk*dv]
-  float *scratch;       // [B*H][CK][dk*dv]
+  float *ckpt;          // [B*H][DVf/VSB][ceil(T/CK)][dk*VSB]
+  float *scratch;       // [B*H][DVf/VSB][CK][dk*VSB]
 };
 
-template <typename IO, int DK, int DV, int CK>
-__global__ void __launch_bounds__(256, 1) delta_rule_bwd_kernel(const BwdParams p) {
-  constexpr int NW = 8, RPW = DK / NW, CPL = DV / 32;
-  static_assert(DK % NW == 0 && DV % 32 == 0, "unsupported head dims");
+// DV: the slice width handled by one CTA (VSB); DVF: the full value width.
+template <typename IO, int DK, int DVF, int DV, int CK>
+__global__ void __launch_bounds__(256) delta_rule_bwd_kernel(const BwdParams p) {
+  constexpr int NW = 8, RPW = DK / NW, CPL = DV / 32, NSL = DVF / DV;
+  static_assert(DK % NW == 0 && DV % 32 == 0 && DVF % DV == 0, "unsupported head dims");
   __shared__ float s_al[DK], s_b[DK], s_ab[DK], s_a[DK], s_q[DK], s_k[DK], s_sc[DK], s_sb[DK];
   __shared__ float s_w[DV], s_do[DV], s_u[DV], s_du[DV], s_v[DV], s_wsc[DV], s_pv[DV];
   __shared__ float s_xdo[DK], s_da[DK], s_db[DK], s_dal[DK];
@@ -58,10 +63,12 @@ __global__ void __launch_bounds__(256, 1) delta_rule_bwd_kernel(const BwdParams 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = p.T, H = p.H;
   const size_t bh = blockIdx.x;  // b * H + h
+  const int slice = blockIdx.y, v0 = slice * DV;
   const size_t b = bh / H, h = bh % H;
   const int nck = (T + CK - 1) / CK;
-  float *ck = p.ckpt + bh * static_cast<size_t>(nck) * DK * DV;
-  float *scr = p.scratch + bh * static_cast<size_t>(CK) * DK * DV;
+  const size_t hs = bh * NSL + slice;  // (head, slice)
+  float *ck = p.ckpt + hs * static_cast<size_t>(nck) * DK * DV;
+  float *scr = p.scratch + hs * static_cast<size_t>(CK) * DK * DV;
   const bool sym = p.beta_v_mode == MODE_ABSENT;  // w = sqrt(beta_k) (.) v
 
   // per-token factors into shared memory (with_back: also q, do, v, k for the gradients)
@@ -85,14 +92,15 @@ __global__ void __launch_bounds__(256, 1) delta_rule_bwd_kernel(const BwdParams 
         s_k[tid] = kk;
       }
     } else if (tid - 128 < DV && tid >= 128) {
-      const int j = tid - 128;
-      const float vj = to_f32(static_cast<const IO *>(p.v)[th * DV + j]);
-      const float ws = sym ? sqrtf(gate_at(p.beta_k, p.beta_k_mode, th, DK, j)) : gate_at(p.beta_v, p.beta_v_mode, th, DV, j);
+      const int j = tid - 128, jg = v0 + j;  // local and full column index
+      const float vj = to_f32(static_cast<const IO *>(p.v)[th * DVF + jg]);
+      const float ws = sym ? sqrtf(gate_at(p.beta_k, p.beta_k_mode, th, DK, jg))
+                           : gate_at(p.beta_v, p.beta_v_mode, th, DVF, jg);
       s_wsc[j] = ws;
       s_w[j] = ws * vj;
       if (with_back) {
         s_v[j] = vj;
-        s_do[j] = to_f32(static_cast<const IO *>(p.dout)[th * DV + j]);
+        s_do[j] = to_f32(static_cast<const IO *>(p.dout)[th * DVF + jg]);
       }
     }
   };
@@ -139,25 +147,26 @@ __global__ void __launch_bounds__(256, 1) delta_rule_bwd_kernel(const BwdParams 
       for (int c = 0; c < CPL; ++c) S[r][c] = fmaf(ai, s_w[lane * CPL + c] - s_u[lane * CPL + c], S[r][c]);
     }
   };
-  auto store_state = [&](float *dst, const float (&S)[RPW][CPL]) {
+  // ld: row stride of the array (DV for the slice's checkpoints and scratch, DVF for S0, dS_T, dS0)
+  auto store_state = [&](float *dst, int ld, const float (&S)[RPW][CPL]) {
 #pragma unroll
     for (int r = 0; r < RPW; ++r)
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) dst[(warp + r * NW) * DV + lane * CPL + c] = S[r][c];
+      for (int c = 0; c < CPL; ++c) dst[(warp + r * NW) * ld + lane * CPL + c] = S[r][c];
   };
-  auto load_state = [&](const float *src, float (&S)[RPW][CPL]) {
+  auto load_state = [&](const float *src, int ld, float (&S)[RPW][CPL]) {
 #pragma unroll
     for (int r = 0; r < RPW; ++r)
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) S[r][c] = src ? src[(warp + r * NW) * DV + lane * CPL + c] : 0.f;
+      for (int c = 0; c < CPL; ++c) S[r][c] = src ? src[(warp + r * NW) * ld + lane * CPL + c] : 0.f;
   };
 
   float S[RPW][CPL];
-  const size_t sbase = bh * static_cast<size_t>(DK) * DV;
+  const size_t sbase = bh * static_cast<size_t>(DK) * DVF + v0;  // this slice of the full-width state
   // ---- pass 1: the forward, keeping the state before every CK-th token
-  load_state(p.S0 ? p.S0 + sbase : nullptr, S);
+  load_state(p.S0 ? p.S0 + sbase : nullptr, DVF, S);
   for (int t = 0; t < T; ++t) {
-    if (t % CK == 0) store_state(ck + static_cast<size_t>(t / CK) * DK * DV, S);
+    if (t % CK == 0) store_state(ck + static_cast<size_t>(t / CK) * DK * DV, DV, S);
     __syncthreads();
     load_token(t, false);
     __syncthreads();
@@ -166,13 +175,13 @@ __global__ void __launch_bounds__(256, 1) delta_rule_bwd_kernel(const BwdParams 
 
   // ---- pass 2: spans of CK tokens from the last, each recomputed then walked backwards
   float G[RPW][CPL];
-  load_state(p.dS_T ? p.dS_T + sbase : nullptr, G);
+  load_state(p.dS_T ? p.dS_T + sbase : nullptr, DVF, G);
   for (int c = nck - 1; c >= 0; --c) {
     const int t0 = c * CK, L = min(CK, T - t0);
     __syncthreads();  // the previous span's scratch reads are done
-    load_state(ck + static_cast<size_t>(c) * DK * DV, S);
+    load_state(ck + static_cast<size_t>(c) * DK * DV, DV, S);
     for (int i = 0; i < L; ++i) {
-      store_state(scr + static_cast<size_t>(i) * DK * DV, S);  // state before token t0 + i
+      store_state(scr + static_cast<size_t>(i) * DK * DV, DV, S);  // state before token t0 + i
       if (i + 1 == L) break;
       __syncthreads();
       load_token(t0 + i, false);
@@ -186,7 +195,7 @@ __global__ void __launch_bounds__(256, 1) delta_rule_bwd_kernel(const BwdParams 
       load_token(t, true);
       __syncthreads();  // also orders the scratch stores above before the loads below
       float Sp[RPW][CPL];  // S_{t-1}; X = D S_{t-1} is applied row by row where it is used
-      load_state(scr + static_cast<size_t>(i) * DK * DV, Sp);
+      load_state(scr + static_cast<size_t>(i) * DK * DV, DV, Sp);
       colsum(Sp, s_ab, s_u);  // s_u = X^T b
       if (tid < DV) s_u[tid] = s_w[tid] - s_u[tid];  // u = w - X^T b
       __syncthreads();
@@ -236,29 +245,32 @@ __global__ void __launch_bounds__(256, 1) delta_rule_bwd_kernel(const BwdParams 
         }
       }
       __syncthreads();
-      // per-token gradients
+      // per-token gradients.  Per-row ones sum over all value columns: each slice adds its part
+      // (outputs are zeroed before the launch); per-column ones belong to this slice alone.
       const float udo = s_udo;
       if (tid < DK) {
         const int i = tid;
         const float ai = s_a[i], sc = s_sc[i], sb = s_sb[i];
         const float dbt = s_db[i] + sc * s_da[i];  // through b, directly and through a = s (.) b
-        p.dq[th * DK + i] = s_xdo[i] + ai * udo;
-        p.dk[th * DK + i] = sb * dbt;
-        if (p.ds) p.ds[th * DK + i] = s_b[i] * s_da[i];
+        atomicAdd(&p.dq[th * DK + i], s_xdo[i] + ai * udo);
+        atomicAdd(&p.dk[th * DK + i], sb * dbt);
+        if (p.ds) atomicAdd(&p.ds[th * DK + i], s_b[i] * s_da[i]);
         const float dbeta = sb > 0.f ? 0.5f * s_k[i] * dbt / sb : 0.f;  // d sqrt(beta) / d beta
-        const float dsym = (sym && p.beta_k_mode == MODE_CHANNEL && sb > 0.f) ? 0.5f * s_v[i] * s_du[i] / sb : 0.f;
-        if (p.beta_k_mode == MODE_CHANNEL) p.dbeta_k[th * DK + i] = dbeta + dsym;
-        if (p.alpha_mode == MODE_CHANNEL) p.dalpha[th * DK + i] = s_dal[i];
+        if (p.beta_k_mode == MODE_CHANNEL) atomicAdd(&p.dbeta_k[th * DK + i], dbeta);
+        if (p.alpha_mode == MODE_CHANNEL) atomicAdd(&p.dalpha[th * DK + i], s_dal[i]);
         s_k[i] = dbeta;  // scalar-mode partials, summed below
       } else if (tid >= 128 && tid - 128 < DV) {
-        const int j = tid - 128;
+        const int j = tid - 128, jg = v0 + j;
         const float du = s_du[j];
-        p.dv[th * DV + j] = s_wsc[j] * du;
-        if (!sym && p.beta_v_mode == MODE_CHANNEL) p.dbeta_v[th * DV + j] = s_v[j] * du;
+        p.dv[th * DVF + jg] = s_wsc[j] * du;
+        if (!sym && p.beta_v_mode == MODE_CHANNEL) p.dbeta_v[th * DVF + jg] = s_v[j] * du;
+        // symmetric channel write w = sqrt(beta_k) (.) v (dk == dv): column jg is key channel jg
+        if (sym && p.beta_k_mode == MODE_CHANNEL && s_sb[jg] > 0.f)
+          atomicAdd(&p.dbeta_k[th * DK + jg], 0.5f * s_v[j] * du / s_sb[jg]);
         s_pv[j] = s_v[j] * du;  // scalar-mode partials
       }
       __syncthreads();
-      if (warp == 0) {  // scalar gates: sums over the channels
+      if (warp == 0) {  // scalar gates: sums over the channels (this slice's part of the columns)
         float sa = 0.f, sbk = 0.f, svv = 0.f;
         for (int i = lane; i < DK; i += 32) {
           sa += s_dal[i];
@@ -269,17 +281,17 @@ __global__ void __launch_bounds__(256, 1) delta_rule_bwd_kernel(const BwdParams 
         sbk = warp_sum(sbk);
         svv = warp_sum(svv);
         if (lane == 0) {
-          if (p.alpha_mode == MODE_SCALAR) p.dalpha[th] = sa;
+          if (p.alpha_mode == MODE_SCALAR) atomicAdd(&p.dalpha[th], sa);
           if (p.beta_k_mode == MODE_SCALAR) {
-            const float sb0 = s_sb[0];
-            p.dbeta_k[th] = sbk + ((sym && sb0 > 0.f) ? 0.5f * svv / sb0 : 0.f);  // + through w = sqrt(beta) v
+            const float sb0 = s_sb[0];  // + through w = sqrt(beta) v
+            atomicAdd(&p.dbeta_k[th], sbk + ((sym && sb0 > 0.f) ? 0.5f * svv / sb0 : 0.f));
           }
-          if (!sym && p.beta_v_mode == MODE_SCALAR) p.dbeta_v[th] = svv;
+          if (!sym && p.beta_v_mode == MODE_SCALAR) atomicAdd(&p.dbeta_v[th], svv);
         }
       }
     }
   }
-  if (p.dS0) store_state(p.dS0 + sbase, G);
+  if (p.dS0) store_state(p.dS0 + sbase, DVF, G);
 }
 
 }  // namespace dr

@@ -350,9 +350,11 @@ size_t bwd_workspace_bytes(const dr_problem *p) {
   return sizeof(float) * static_cast<size_t>(p->B) * p->H * (nck + kBwdSpan) * p->dk * p->dv;
 }
 
+constexpr int kBwdSlice = 32;  // value columns per CTA of the backward pass
+
 template <typename IO, int DK, int DV>
 dr_status bwd_launch(const dr::BwdParams &bp, int heads, cudaStream_t st) {
-  dr::delta_rule_bwd_kernel<IO, DK, DV, kBwdSpan><<<heads, 256, 0, st>>>(bp);
+  dr::delta_rule_bwd_kernel<IO, DK, DV, kBwdSlice, kBwdSpan><<<dim3(heads, DV / kBwdSlice), 256, 0, st>>>(bp);
   return launch_status();
 }
 
@@ -401,6 +403,16 @@ dr_status dr_backward(const dr_problem *p, const void *q, const void *k, const v
   }
   if (!workspace || workspace_bytes < bwd_workspace_bytes(p)) return DR_ERR_WORKSPACE;
   float *ws = static_cast<float *>(workspace);
+  {  // the per-key-channel gradients are sums over value-column slices, accumulated in place
+    const size_t tok = static_cast<size_t>(p->B) * p->T * p->H;
+    const size_t gk = tok * p->dk * sizeof(float);
+    auto gate_bytes = [&](int mode) { return mode == DR_CHANNEL ? gk : tok * sizeof(float); };
+    struct Z { void *ptr; size_t bytes; } zs[] = {
+        {dq, gk}, {dk, gk}, {ds, gk}, {dalpha, dalpha ? gate_bytes(p->alpha_mode) : 0},
+        {dbeta_k, gate_bytes(p->beta_k_mode)}, {dbeta_v, dbeta_v ? gate_bytes(p->beta_v_mode) : 0}};
+    for (const Z &z : zs)
+      if (z.ptr && cudaMemsetAsync(z.ptr, 0, z.bytes, cs) != cudaSuccess) return DR_ERR_CUDA;
+  }
   const size_t nck = (static_cast<size_t>(p->T) + kBwdSpan - 1) / kBwdSpan;
   dr::BwdParams bp{p->T, p->H, q, k, v, dout, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v,
                    p->beta_v_mode, s, S0, dS_T, dq, dk, dv, dalpha, dbeta_k, dbeta_v, ds, dS0, ws,
