@@ -203,7 +203,7 @@ DR_API dr_status dr_state_map_apply(int n, int dk, int dv, const float *M, const
  * forward defined by the recurrence (DeltaNet page steps 3-6; FG2-GDN page
  * section 2; OSDN summary "Method").  Reverse mode through
  *   X = Diag(alpha_t) S_{t-1},  u = w_t - X^T b_t,  S_t = X + a_t u^T,  o_t = S_t^T q_t.
- * The pass recomputes the forward itself (it keeps the state every 32 tokens in
+ * The pass recomputes the forward itself (it keeps the state every 16 tokens in
  * the workspace and re-derives the states in between), so it takes the
  * forward's inputs, not its outputs.
  *   inputs   as dr_chunk_fwd_osdn (s may be NULL); p->chunk is ignored

@@ -343,18 +343,20 @@ dr_status decode_step_impl(const dr_problem *p, const void *q, const void *k, co
   return decode_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
 }
 
-constexpr int kBwdSpan = 32;  // tokens between the backward pass's state checkpoints
+constexpr int kBwdSpan = 16;  // tokens between the backward pass's state checkpoints
 
 size_t bwd_workspace_bytes(const dr_problem *p) {
   const size_t nck = (static_cast<size_t>(p->T) + kBwdSpan - 1) / kBwdSpan;
   return sizeof(float) * static_cast<size_t>(p->B) * p->H * (nck + kBwdSpan) * p->dk * p->dv;
 }
 
-constexpr int kBwdSlice = 32;  // value columns per CTA of the backward pass
-
 template <typename IO, int DK, int DV>
 dr_status bwd_launch(const dr::BwdParams &bp, int heads, cudaStream_t st) {
-  dr::delta_rule_bwd_kernel<IO, DK, DV, kBwdSlice, kBwdSpan><<<dim3(heads, DV / kBwdSlice), 256, 0, st>>>(bp);
+  auto kern = dr::delta_rule_bwd_kernel<IO, DK, DV, kBwdSpan>;
+  constexpr int smem = dr::bwd_smem_bytes<DK, kBwdSpan>();
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return DR_ERR_CUDA;
+  kern<<<dim3(heads, DV / dr::kBwdCols), 256, smem, st>>>(bp);
   return launch_status();
 }
 
