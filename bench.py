@@ -62,10 +62,12 @@ def decode_bytes(B, H, dk, dv, io=2, alpha_ch=True, beta_ch=True):
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the ncu captures
 # summarised under profiles/, each valid only for the kernel sources it was taken on: the key is
-# a digest of every file under csrc/ (see csrc_digest), so any source change voids the number.
+# a digest of the kernel's own source files under csrc/ (see csrc_digest), so any change to them
+# voids the number, and the workload it was taken on, so other workloads report none.
+RING_SOURCES = ("chunk_tc3.cuh", "chunk_tc.cuh", "tri_inverse.cuh", "sm100.cuh", "common.cuh")
 MEASURED_TRAFFIC = {
-    "chunk_fwd_ring_kernel": ("5946d073e482", 248.945664e6, None),
-    "decode_step_kernel": ("f563c5e8b358", 1031.6032e6, "decode.cuh"),
+    ("chunk_fwd_ring_kernel", "gdn_bf16"): ("f96b31f64e46", 249.28128e6, RING_SOURCES),
+    ("decode_step_kernel", "decode_bf16"): ("381fd28fdea0", 1033.046016e6, ("decode.cuh",)),
 }
 
 # Prefill kernel the library runs for dk = dv = 128, chunk 64 (DR_PREFILL_KERNEL selects it).
@@ -77,24 +79,24 @@ def prefill_kernel_name():
 
 
 def csrc_digest(only=None):
-    """sha1 over the kernel sources (all of csrc/, or the one file `only`), in name order."""
+    """sha1 over the kernel sources (all of csrc/, or the files named in `only`), in name order."""
     import hashlib
 
     d = os.path.join(ROOT, "weight_recurrence_chunkwise_b200", "csrc")
     h = hashlib.sha1()
     for name in sorted(os.listdir(d)):
-        if only is not None and name != only:
+        if only is not None and name not in only:
             continue
         with open(os.path.join(d, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def measured_traffic(kernel):
+def measured_traffic(kernel, workload):
     """Bytes per launch from the committed ncu summary, or None once the kernel sources changed."""
-    if kernel not in MEASURED_TRAFFIC:
+    if (kernel, workload) not in MEASURED_TRAFFIC:
         return None
-    prefix, nbytes, only = MEASURED_TRAFFIC[kernel]
+    prefix, nbytes, only = MEASURED_TRAFFIC[(kernel, workload)]
     try:
         digest = csrc_digest(only)
     except OSError:
@@ -193,12 +195,13 @@ def to_dev(x, dev):
     return {k: (None if t is None else t.to(dev)) for k, t in x.items()}
 
 
-def cpu_oracle_sample(p, seconds=12.0):
-    """Time the float64 oracle on a bounded sample of the prefill workload (whole heads, all T)."""
+def cpu_oracle_sample(p):
+    """Time the float64 oracle on a bounded sample of the prefill workload (whole heads, all T):
+    about four heads per host thread, at most the whole batch (some 10-30 s of CPU work)."""
     import oracle
 
     threads = oracle.max_threads()
-    x = make_inputs(p.replace(B=max(1, min(p.B, threads // p.H))))
+    x = make_inputs(p.replace(B=max(1, min(p.B, -(-4 * threads // p.H)))))
     t0 = time.perf_counter()
     oracle.delta_rule_sequential(x["q"], x["k"], x["v"], x["beta_k"], alpha=x["alpha"], beta_v=x["beta_v"],
                                  S0=x["S0"], threads=threads)
@@ -404,7 +407,7 @@ def main():
     achieved_gbs = byts / (prefill_ms / 1e3) / 1e9
     t_roof_ms = max(byts / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops_sustained"] * 1e12)) * 1e3
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": measured_traffic(prefill_kernel_name()),
+                "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": measured_traffic(prefill_kernel_name(), p.name),
                 "peak_source": peaks_src,
                 "kernel": prefill_kernel_name(), "algorithmic_bytes_per_launch": byts,
                 "algorithmic_flops_per_launch": flops,
@@ -475,7 +478,7 @@ def main():
               "config": {"workload": DECODE.name, "B": DECODE.B, "H": DECODE.H, "dk": DECODE.dk, "dv": DECODE.dv,
                          "state_MiB": DECODE.B * DECODE.H * DECODE.dk * DECODE.dv * 4 / 2 ** 20},
               "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": dgbs / peaks["hbm_gbs"], "traffic": measured_traffic("decode_step_kernel"),
+                           "frac": dgbs / peaks["hbm_gbs"], "traffic": measured_traffic("decode_step_kernel", DECODE.name),
                            "peak_source": peaks_src,
                            "kernel": "decode_step_kernel", "algorithmic_bytes_per_launch": dbytes}}
     del S_dec, pool

@@ -77,3 +77,55 @@ def test_backward_without_final_state_gradient(dr):
     assert got["S0"] is None
     assert err(got["v"].cpu().numpy(), ref["v"].numpy()) <= 2e-4
     assert err(got["alpha"].cpu().numpy(), ref["alpha"].numpy()) <= 2e-4
+
+
+@pytest.mark.parametrize("base", ["gdn_bf16", "kda_bf16"])
+def test_backward_workload_full_size(dr, base):
+    """The backward at the workload's full size, in the launch configuration ``bench.py --backward``
+    times, checked two ways:
+
+    * Linearity, over the whole batch.  With the gates and keys fixed, o and S_T are linear in
+      (v, S0) jointly and o is linear in q, so for L = sum(do o) + sum(dS_T S_T)
+          <dv, v> + <dS0, S0> = L   and   <dq, q> = sum(do o),
+      with o and S_T from the forward kernel.  The forward's bf16 output rounding (2^-9 relative)
+      bounds the mismatch by 5e-3 of sum |do o| + sum |dS_T S_T|.
+    * One sampled head (the last (b, h), whose gradients depend on that head's inputs alone)
+      against the float64 reference, to the same 2e-4 of each gradient's RMS as the small cases
+      (GDN only: the reference needs about ten seconds per 4096 tokens).
+    """
+    p = problem(base, S0="normal")
+    x = make_inputs(p)
+    g = to_dev(x)
+    gen = torch.Generator().manual_seed(5)
+    do = torch.randn(x["v"].shape, generator=gen).to(x["v"].dtype)
+    dST = torch.randn((p.B, p.H, p.dk, p.dv), generator=gen)
+    do_d, dST_d = do.cuda(), dST.cuda()
+    got = dr.dr_backward(g["q"], g["k"], g["v"], g["beta_k"], do_d, alpha=g["alpha"], beta_v=g["beta_v"], s=g["s"],
+                         S0=g["S0"], dS_T=dST_d)
+    o, S_T = dr.dr_chunk_fwd(g["q"], g["k"], g["v"], g["beta_k"], alpha=g["alpha"], beta_v=g["beta_v"], S0=g["S0"],
+                             chunk=p.chunk)
+    torch.cuda.synchronize()
+    f64 = lambda t: t.double()
+    Lo = (f64(do_d) * f64(o)).sum()
+    LS = (f64(dST_d) * f64(S_T)).sum()
+    scale = float((f64(do_d) * f64(o)).abs().sum() + (f64(dST_d) * f64(S_T)).abs().sum())
+    lin_v = float((got["v"].double() * f64(g["v"])).sum() + (got["S0"].double() * f64(g["S0"])).sum())
+    lin_q = float((got["q"].double() * f64(g["q"])).sum())
+    assert abs(lin_v - float(Lo + LS)) <= 5e-3 * scale, (lin_v, float(Lo + LS), scale)
+    assert abs(lin_q - float(Lo)) <= 5e-3 * scale, (lin_q, float(Lo), scale)
+
+    if base != "gdn_bf16":
+        return
+    b, h = p.B - 1, p.H - 1
+    one = lambda t: None if t is None else t[b:b + 1, :, h:h + 1]
+    ref = ob.backward(one(x["q"]), one(x["k"]), one(x["v"]), one(x["beta_k"]), one(do), alpha=one(x["alpha"]),
+                      beta_v=one(x["beta_v"]), S0=x["S0"][b:b + 1, h:h + 1], s_scale=one(x["s"]),
+                      dS_T=dST[b:b + 1, h:h + 1])
+    pick = {"q": one, "k": one, "v": one, "beta_k": one, "alpha": one, "beta_v": one,
+            "S0": lambda t: t[b:b + 1, h:h + 1]}
+    names = {"q": "q", "k": "k", "v": "v", "beta_k": "beta_k", "alpha": "alpha", "beta_v": "beta_v", "S0": "S0"}
+    for mine, theirs in names.items():
+        if ref[theirs] is None:
+            continue
+        e = err(pick[mine](got[mine]).cpu().numpy(), ref[theirs].numpy())
+        assert e <= 2e-4, (mine, e)
