@@ -320,7 +320,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--decode-steps", type=int, default=1000,
+                    help="chained in-place decode steps timed (the decode workload is 1000 steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only-prefill", action="store_true",
                     help="profiling aid: time only the prefill step (no decode workload, e2e or CPU leg)")
@@ -483,37 +484,73 @@ def main():
                            "kernel": "decode_step_kernel", "algorithmic_bytes_per_launch": dbytes}}
     del S_dec, pool
 
-    # ---------------- end to end through the public API with host buffers (pinned), copies timed
+    # ---------------- end to end through the public API with host buffers (pinned), copies timed.
+    # Steps are pipelined over two buffer slots and three streams, as a caller streaming batches
+    # would: step i's host->device copies overlap step i-1's kernels and step i-2's device->host
+    # copies (PCIe carries both directions at once).  Every step still moves all its inputs in and
+    # all its results out inside the timed region.
     host = {k: (None if t is None else t.cpu().pin_memory()) for k, t in x.items()}
     host_n = {k: (None if t is None else t.cpu().pin_memory()) for k, t in nxt.items()}
-    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    S_h = torch.empty(S.shape, dtype=S.dtype).pin_memory()
-    o1_h = torch.empty(o1.shape, dtype=o1.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in list(host.values()) + list(host_n.values()) if t is not None)
-    d2h = o_h.numel() * o_h.element_size() + S_h.numel() * 4 + o1_h.numel() * o1_h.element_size()
+    d2h = o.numel() * o.element_size() + S.numel() * 4 + o1.numel() * o1.element_size()
     e2e_steps = max(3, min(10, n))
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    dev_like = lambda h: {k: (None if t is None else torch.empty(t.shape, dtype=t.dtype, device=dev))
+                          for k, t in h.items()}
+    slots = [{"g": dev_like(host), "gn": dev_like(host_n), "o": torch.empty_like(o), "S": torch.empty_like(S),
+              "o1": torch.empty_like(o1), "o_h": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
+              "S_h": torch.empty(S.shape, dtype=S.dtype).pin_memory(),
+              "o1_h": torch.empty(o1.shape, dtype=o1.dtype).pin_memory(),
+              "in": torch.cuda.Event(), "done": torch.cuda.Event(), "out": torch.cuda.Event()} for _ in range(2)]
+    for sl in slots:  # every event recorded once, so the first waits on it are satisfied
+        for e in ("in", "done", "out"):
+            sl[e].record(st)
 
-    def e2e_step():
-        g = {k: (None if t is None else t.to(dev, non_blocking=True)) for k, t in host.items()}
-        gn = {k: (None if t is None else t.to(dev, non_blocking=True)) for k, t in host_n.items()}
-        og, Sg = dr.dr_chunk_fwd(g["q"], g["k"], g["v"], g["beta_k"], alpha=g["alpha"], beta_v=g["beta_v"],
-                                 chunk=p.chunk, workspace=ws_buf, stream=st)
-        og1 = dr.dr_decode_step(gn["q"], gn["k"], gn["v"], gn["beta_k"], Sg, alpha=gn["alpha"], stream=st)
-        o_h.copy_(og, non_blocking=True)
-        S_h.copy_(Sg, non_blocking=True)
-        o1_h.copy_(og1, non_blocking=True)
+    def e2e_step(i):
+        sl = slots[i % 2]
+        s_in.wait_event(sl["done"])  # step i-2's kernels no longer read this slot's inputs
+        with torch.cuda.stream(s_in):
+            for src, dst in ((host, sl["g"]), (host_n, sl["gn"])):
+                for k, t in src.items():
+                    if t is not None:
+                        dst[k].copy_(t, non_blocking=True)
+        sl["in"].record(s_in)
+        st.wait_event(sl["in"])
+        st.wait_event(sl["out"])  # step i-2's results have been read back
+        g, gn = sl["g"], sl["gn"]
+        dr.dr_chunk_fwd(g["q"], g["k"], g["v"], g["beta_k"], alpha=g["alpha"], beta_v=g["beta_v"], chunk=p.chunk,
+                        o=sl["o"], S_T=sl["S"], workspace=ws_buf, stream=st)
+        dr.dr_decode_step(gn["q"], gn["k"], gn["v"], gn["beta_k"], sl["S"], alpha=gn["alpha"], o=sl["o1"], stream=st)
+        sl["done"].record(st)
+        s_out.wait_event(sl["done"])
+        with torch.cuda.stream(s_out):
+            sl["o_h"].copy_(sl["o"], non_blocking=True)
+            sl["S_h"].copy_(sl["S"], non_blocking=True)
+            sl["o1_h"].copy_(sl["o1"], non_blocking=True)
+        sl["out"].record(s_out)
 
-    e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier(ws)
     e0.record(st)
-    for _ in range(e2e_steps):
-        e2e_step()
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    st.wait_stream(s_in)
+    st.wait_stream(s_out)
     e1.record(st)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws, dev) / e2e_steps
+    # the last step's results, as read back, against the same step computed on the device alone
+    last = slots[(e2e_steps - 1) % 2]
+    if not (torch.equal(last["o_h"], o.cpu()) and torch.equal(last["o1_h"], o1.cpu())):
+        raise RuntimeError("end-to-end results differ from the device-resident run")
     e2e = {"value": tok_heads * ws / (e2e_ms / 1e3) / 1e6, "unit": "Mtokens·heads/s", "ms_per_step": e2e_ms,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+           "pipeline": "2 slots; copies in, kernels and copies out on three streams"}
+    del slots
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
