@@ -44,6 +44,21 @@ DR_API int dr_diag_umma_selftest(int N, int K, int a_mn, int b_mn, int bf16, con
  */
 DR_API int dr_diag_tri_inverse(const float *A, float *T, void *stream);
 
+/*
+ * The bounded waits of the prefill kernels, run out on purpose: every CTA waits
+ * on an mbarrier that nothing completes, through the prefill kernels' own wait
+ * helpers (cluster_scope = 0: one CTA, CTA-scope wait; cluster_scope != 0: a
+ * cluster of two CTAs, cluster-scope acquire).  Each wait gives up after
+ * limit_ns of wall time (0 < limit_ns <= 1e9, else DR_ERR_INVALID_ARG), sets the
+ * timeout bit of the status word in `workspace` (>= 256 bytes of device memory;
+ * dr_workspace_status then returns DR_ERR_TIMEOUT) and stores the nanoseconds
+ * it waited in waited_ns[cta] (device buffer of 2 entries, or NULL).  The
+ * kernel exits normally and the context stays usable.  Asynchronous on
+ * `stream`; returns a dr_status code for the launch.
+ */
+DR_API int dr_diag_wait_timeout(int cluster_scope, unsigned long long limit_ns, void *workspace,
+                                unsigned long long *waited_ns, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

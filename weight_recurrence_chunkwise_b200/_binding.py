@@ -42,7 +42,7 @@ EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_chunk_fwd_osdn", "dr_ch
            "dr_chunk_fwd_noalloc", "dr_decode_step",
            "dr_decode_step_osdn", "dr_state_map_apply", "dr_backward_workspace", "dr_backward",
            "dr_workspace_status", "dr_status_string", "dr_version", "dr_diag_umma_selftest",
-           "dr_diag_tri_inverse")
+           "dr_diag_tri_inverse", "dr_diag_wait_timeout")
 
 
 def lib():
@@ -83,6 +83,8 @@ def lib():
         L.dr_diag_umma_selftest.restype = ctypes.c_int
         L.dr_diag_tri_inverse.argtypes = [vp, vp, vp]
         L.dr_diag_tri_inverse.restype = ctypes.c_int
+        L.dr_diag_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_ulonglong, vp, vp, vp]
+        L.dr_diag_wait_timeout.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -338,3 +340,19 @@ def dr_diag_tri_inverse(A, stream=None):
     if rc != DR_OK:
         raise DeltaRuleError(rc, "dr_diag_tri_inverse")
     return T
+
+
+def dr_diag_wait_timeout(cluster_scope: bool, limit_ns: int, device=None, stream=None):
+    """Run the prefill kernels' bounded wait out on a barrier nothing completes.
+
+    Returns ``(status, waited_ns)``: the workspace status code (DR_ERR_TIMEOUT when the wait gave
+    up) and the nanoseconds each CTA waited (one CTA, or a cluster of two with ``cluster_scope``).
+    """
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    waited = torch.zeros(2, dtype=torch.int64, device=dev)
+    rc = lib().dr_diag_wait_timeout(int(bool(cluster_scope)), int(limit_ns), _ptr(ws), _ptr(waited), _stream(stream))
+    if rc != DR_OK:
+        raise DeltaRuleError(rc, "dr_diag_wait_timeout")
+    status = dr_workspace_status(ws, stream)
+    return status, [int(x) for x in waited[:2 if cluster_scope else 1].cpu()]

@@ -20,6 +20,7 @@
 #include "state_map.cuh"
 #include "backward.cuh"
 #include "umma_selftest.cuh"
+#include "wait_selftest.cuh"
 
 namespace {
 
@@ -566,6 +567,33 @@ int dr_diag_umma_selftest(int N, int K, int a_mn, int b_mn, int bf16, const void
   DR_SELFTEST_CASE(128, 128)
 #undef DR_SELFTEST_CASE
   return DR_ERR_UNSUPPORTED;
+}
+
+int dr_diag_wait_timeout(int cluster_scope, unsigned long long limit_ns, void *workspace,
+                         unsigned long long *waited_ns, void *stream) {
+  if (!workspace || limit_ns == 0 || limit_ns > 1000000000ull) return DR_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *status = static_cast<uint32_t *>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DR_ERR_CUDA;
+  const int sc = cluster_scope ? 1 : 0;
+  if (!sc) {
+    dr::wait_selftest_kernel<<<1, 32, 0, st>>>(0, limit_ns, status, waited_ns);
+    return launch_status();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(32, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, dr::wait_selftest_kernel, sc, limit_ns, status, waited_ns) != cudaSuccess)
+    return DR_ERR_CUDA;
+  return launch_status();
 }
 
 int dr_diag_tri_inverse(const float *A, float *T, void *stream) {
