@@ -177,9 +177,6 @@ __device__ __forceinline__ void inverse64(const __half *Ah, const __half *AhT, _
 
 // ------------------------------------------------------------------ layout-generic variant
 // Byte offset of element (r, c) of a 64 x 64 fp16 array.
-struct PaddedLayout {  // rows of LD halves
-  __device__ static uint32_t off(int r, int c) { return static_cast<uint32_t>((r * LD + c) * 2); }
-};
 struct Sw128Layout {  // 128-byte rows, 16-byte groups XOR-ed with (r & 7): a K-major MMA operand tile
   __device__ static uint32_t off(int r, int c) {
     return static_cast<uint32_t>(r * 128 + ((((c >> 3) ^ (r & 7))) << 4) + (c & 7) * 2);
@@ -277,148 +274,6 @@ __device__ __forceinline__ void inverse64_rows(const uint8_t *Ah, uint8_t *ThT, 
       }
     }
     sync();
-  }
-}
-
-// Flat variant with one group barrier.  With D = blockdiag((I + A_bb)^-1) and X = D A_off (A_off:
-// the blocks below the diagonal), I + A = D^-1 (I + X) and X^4 = 0, so
-//     T = (I - X + X^2 - X^3) D,   T_ij = S_ij D_j  (S = I - X + X^2 - X^3).
-// Warp i computes D_i and the X_ij of its block row alone; after one barrier (D_j^T and the
-// X_mj^T needed by other rows are exchanged through `scr`) it forms S_ij and T_ij.  Longest
-// dependent chain after the diagonal blocks: X_31 -> X^2_31 -> X^3_30 -> T_30.
-// Result as in inverse64_rows: warp i < 4 ends with Trow[d] = T_{i, i-d}.  `scr` (64 x 64 fp16 in
-// layout Lay) must not overlap Ah; Ah is not read after the barrier.
-template <class Lay, typename Sync>
-__device__ __forceinline__ void inverse64_flat(const uint8_t *Ah, uint8_t *scr, int warp, int lane, Frag (&Trow)[4],
-                                               Sync sync) {
-  Frag X[3];  // X_{i, i-1-e}: X[0] = X_{i,i-1}, X[1] = X_{i,i-2}, X[2] = X_{i,i-3}
-  if (warp < 4) {
-    const int b = warp;
-    const Frag N = load_frag_l<Lay>(Ah, b, b, lane);
-    const Frag Nt = load_frag_t_l<Lay>(Ah, b, b, lane);
-    const Frag N2 = mul(N, Nt), N2t = mul(Nt, N);
-    const Frag N4 = mul(N2, N2t), N4t = mul(N2t, N2);
-    const Frag N8t = mul(N4t, N4);
-    const Frag X1 = eye_plus(N, -1.f, lane);
-    const Frag Y1t = eye_plus(N2t, 1.f, lane);
-    const Frag P1 = mul(X1, Y1t);
-    const Frag Y2t = eye_plus(N4t, 1.f, lane);
-    const Frag P2 = mul(P1, Y2t);
-    const Frag Y3t = eye_plus(N8t, 1.f, lane);
-    Trow[0] = mul(P2, Y3t);  // D_b
-    if (b < 3) store_frag_l<Lay>(scr, b, b, mul(Y3t, P2), lane);  // D_b^T, for the rows below
-#pragma unroll
-    for (int e = 0; e < 3; ++e) {
-      if (e < b) {
-        const int j = b - 1 - e;
-        const Frag At = load_frag_t_l<Lay>(Ah, b, j, lane);  // F(A_bj^T)
-        X[e] = mul(Trow[0], At);                              // X_bj = D_b A_bj
-        if (b < 3) store_frag_l<Lay>(scr, j, b, mul(At, Trow[0]), lane);  // X_bj^T at block (j, b)
-      }
-    }
-  }
-  sync();
-  if (warp == 1) {
-    negate(X[0]);
-    Trow[1] = mul(X[0], load_frag_l<Lay>(scr, 0, 0, lane));  // T_10 = -X_10 D_0
-  } else if (warp == 2) {
-    Frag S20 = mul(X[0], load_frag_l<Lay>(scr, 0, 1, lane));  // X^2_20 = X_21 X_10
-#pragma unroll
-    for (int e = 0; e < 8; ++e) S20.v[e] -= X[1].v[e];
-    negate(X[0]);                                               // S_21 = -X_21
-    Trow[2] = mul(S20, load_frag_l<Lay>(scr, 0, 0, lane));
-    Trow[1] = mul(X[0], load_frag_l<Lay>(scr, 1, 1, lane));
-  } else if (warp == 3) {
-    const Frag X10t = load_frag_l<Lay>(scr, 0, 1, lane);
-    const Frag X2_31 = mul(X[0], load_frag_l<Lay>(scr, 1, 2, lane));  // X_32 X_21
-    Frag X2_30 = mul(X[1], X10t);                                       // X_31 X_10
-    mul_acc(X2_30, X[0], load_frag_l<Lay>(scr, 0, 2, lane));           //  + X_32 X_20
-    const Frag X3_30 = mul(X2_31, X10t);                                // X_32 X_21 X_10
-    Frag S30, S31;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      S30.v[e] = X2_30.v[e] - X[2].v[e] - X3_30.v[e];
-      S31.v[e] = X2_31.v[e] - X[1].v[e];
-    }
-    negate(X[0]);  // S_32
-    Trow[3] = mul(S30, load_frag_l<Lay>(scr, 0, 0, lane));
-    Trow[2] = mul(S31, load_frag_l<Lay>(scr, 1, 1, lane));
-    Trow[1] = mul(X[0], load_frag_l<Lay>(scr, 2, 2, lane));
-  }
-}
-
-// As inverse64_flat, with the diagonal blocks by forward substitution on the FMA pipe (fp32): the
-// warp MMAs share the SM's tensor cores with any tcgen05 work of the same CTA, so the fewer
-// dependent warp-MMA steps the chain has, the less it waits behind them.  Threads 0..63 each
-// solve one column j of one block b: (I + N_b) d = e_j.  `scr` receives D_b at block (b, b).
-template <class Lay, typename Sync>
-__device__ __forceinline__ void inverse64_subst(const uint8_t *Ah, uint8_t *scr, int warp, int lane, Frag (&Trow)[4],
-                                                Sync sync) {
-  if (warp < 2) {
-    const int t = warp * 32 + lane, b = t >> 4, j = t & 15;
-    float x[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int r = 16 * b + i;
-      const uint4 lo = *reinterpret_cast<const uint4 *>(Ah + Lay::off(r, 16 * b));
-      const uint4 hi = *reinterpret_cast<const uint4 *>(Ah + Lay::off(r, 16 * b + 8));
-      const __half2 *nl = reinterpret_cast<const __half2 *>(&lo);
-      const __half2 *nh = reinterpret_cast<const __half2 *>(&hi);
-      float acc = (i == j) ? 1.f : 0.f;
-#pragma unroll
-      for (int m = 0; m < i; ++m) {
-        const __half2 h2 = (m < 8) ? nl[m >> 1] : nh[(m - 8) >> 1];
-        const float n = (m & 1) ? __high2float(h2) : __low2float(h2);
-        acc = fmaf(-n, x[m], acc);
-      }
-      x[i] = acc;
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      *reinterpret_cast<__half *>(scr + Lay::off(16 * b + i, 16 * b + j)) = __float2half_rn(x[i]);
-  }
-  sync();
-  Frag X[3];  // X_{i, i-1-e}
-  if (warp < 4) {
-    const int b = warp;
-    Trow[0] = load_frag_l<Lay>(scr, b, b, lane);  // D_b
-#pragma unroll
-    for (int e = 0; e < 3; ++e) {
-      if (e < b) {
-        const int j = b - 1 - e;
-        const Frag At = load_frag_t_l<Lay>(Ah, b, j, lane);  // F(A_bj^T)
-        X[e] = mul(Trow[0], At);                              // X_bj = D_b A_bj
-        if (b < 3) store_frag_l<Lay>(scr, j, b, mul(At, Trow[0]), lane);  // X_bj^T at block (j, b)
-      }
-    }
-  }
-  sync();
-  if (warp == 1) {
-    negate(X[0]);
-    Trow[1] = mul(X[0], load_frag_t_l<Lay>(scr, 0, 0, lane));  // T_10 = -X_10 D_0
-  } else if (warp == 2) {
-    Frag S20 = mul(X[0], load_frag_l<Lay>(scr, 0, 1, lane));  // X^2_20 = X_21 X_10
-#pragma unroll
-    for (int e = 0; e < 8; ++e) S20.v[e] -= X[1].v[e];
-    negate(X[0]);
-    Trow[2] = mul(S20, load_frag_t_l<Lay>(scr, 0, 0, lane));
-    Trow[1] = mul(X[0], load_frag_t_l<Lay>(scr, 1, 1, lane));
-  } else if (warp == 3) {
-    const Frag X10t = load_frag_l<Lay>(scr, 0, 1, lane);
-    const Frag X2_31 = mul(X[0], load_frag_l<Lay>(scr, 1, 2, lane));
-    Frag X2_30 = mul(X[1], X10t);
-    mul_acc(X2_30, X[0], load_frag_l<Lay>(scr, 0, 2, lane));
-    const Frag X3_30 = mul(X2_31, X10t);
-    Frag S30, S31;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      S30.v[e] = X2_30.v[e] - X[2].v[e] - X3_30.v[e];
-      S31.v[e] = X2_31.v[e] - X[1].v[e];
-    }
-    negate(X[0]);
-    Trow[3] = mul(S30, load_frag_t_l<Lay>(scr, 0, 0, lane));
-    Trow[2] = mul(S31, load_frag_t_l<Lay>(scr, 1, 1, lane));
-    Trow[1] = mul(X[0], load_frag_t_l<Lay>(scr, 2, 2, lane));
   }
 }
 
