@@ -70,6 +70,12 @@ MEASURED_TRAFFIC = {
     ("decode_step_kernel", "decode_bf16"): ("381fd28fdea0", 1033.046016e6, ("decode.cuh",)),
 }
 
+# Decode kernel the library runs for the decode workload (more heads than SMs; DR_DECODE_KERNEL=classic
+# keeps one CTA per head).
+def decode_kernel_name():
+    return "decode_step_kernel" if os.environ.get("DR_DECODE_KERNEL") == "classic" else "decode_stream_kernel"
+
+
 # Prefill kernel the library runs for dk = dv = 128, chunk 64 (DR_PREFILL_KERNEL selects it).
 PREFILL_KERNELS = {"ring": "chunk_fwd_ring_kernel", "pair": "chunk_fwd_pair_kernel", "single": "chunk_fwd_tc_kernel"}
 
@@ -479,9 +485,9 @@ def main():
               "config": {"workload": DECODE.name, "B": DECODE.B, "H": DECODE.H, "dk": DECODE.dk, "dv": DECODE.dv,
                          "state_MiB": DECODE.B * DECODE.H * DECODE.dk * DECODE.dv * 4 / 2 ** 20},
               "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": dgbs / peaks["hbm_gbs"], "traffic": measured_traffic("decode_step_kernel", DECODE.name),
+                           "frac": dgbs / peaks["hbm_gbs"], "traffic": measured_traffic(decode_kernel_name(), DECODE.name),
                            "peak_source": peaks_src,
-                           "kernel": "decode_step_kernel", "algorithmic_bytes_per_launch": dbytes}}
+                           "kernel": decode_kernel_name(), "algorithmic_bytes_per_launch": dbytes}}
     del S_dec, pool
 
     # ---------------- end to end through the public API with host buffers (pinned), copies timed.

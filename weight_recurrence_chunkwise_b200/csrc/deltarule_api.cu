@@ -17,6 +17,7 @@
 #include "chunk_tc3.cuh"
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_stream.cuh"
 #include "state_map.cuh"
 #include "backward.cuh"
 #include "umma_selftest.cuh"
@@ -267,12 +268,43 @@ dr_status tc_ring_launch(const dr_problem *p, const int *cu, const void *q, cons
 }
 
 // ----------------------------------------------------------------- decode
+// DR_DECODE_KERNEL=classic keeps dk = dv = 128 on one CTA per head (for comparisons); the default
+// streams the states through a persistent kernel once there are more heads than SMs.
+bool decode_stream_enabled() {
+  static const bool on = [] {
+    const char *e = std::getenv("DR_DECODE_KERNEL");
+    return !(e && std::strcmp(e, "classic") == 0);
+  }();
+  return on;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
 template <typename IO, int DK, int DV>
 dr_status decode_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
                         const float *beta_k, const float *beta_v, const float *s_scale, float *S, void *o,
                         cudaStream_t st) {
   const long long heads = static_cast<long long>(p->B) * p->H;
   if (heads > 0x7fffffffLL) return DR_ERR_INVALID_ARG;
+  if constexpr (DK == 128 && DV == 128) {
+    const int sms = sm_count();
+    if (decode_stream_enabled() && sms > 0 && heads > sms) {
+      auto kern = dr::decode_stream_kernel<IO>;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(dr::kDecodeStreamSmem)) != cudaSuccess)
+        return DR_ERR_CUDA;
+      const long long grid = heads < 2LL * sms ? heads : 2LL * sms;  // two CTAs per SM
+      kern<<<static_cast<unsigned>(grid), 256, dr::kDecodeStreamSmem, st>>>(
+          static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v), alpha, p->alpha_mode,
+          beta_k, p->beta_k_mode, beta_v, p->beta_v_mode, s_scale, S, static_cast<IO *>(o), heads);
+      return launch_status();
+    }
+  }
   dr::decode_step_kernel<IO, DK, DV><<<static_cast<unsigned>(heads), 256, 0, st>>>(
       static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v), alpha, p->alpha_mode,
       beta_k, p->beta_k_mode, beta_v, p->beta_v_mode, s_scale, S, static_cast<IO *>(o));
