@@ -66,8 +66,8 @@ def decode_bytes(B, H, dk, dv, io=2, alpha_ch=True, beta_ch=True):
 # voids the number, and the workload it was taken on, so other workloads report none.
 RING_SOURCES = ("chunk_tc3.cuh", "chunk_tc.cuh", "tri_inverse.cuh", "sm100.cuh", "common.cuh")
 MEASURED_TRAFFIC = {
-    ("chunk_fwd_ring_kernel", "gdn_bf16"): ("f96b31f64e46", 249.28128e6, RING_SOURCES),
-    ("decode_step_kernel", "decode_bf16"): ("381fd28fdea0", 1033.046016e6, ("decode.cuh",)),
+    ("chunk_fwd_ring_kernel", "gdn_bf16"): ("f43247f89c6c", 249.243904e6, RING_SOURCES),
+    ("decode_stream_kernel", "decode_bf16"): ("f9a46a4cdf2e", 1032.60288e6, ("decode_stream.cuh", "common.cuh")),
 }
 
 # Decode kernel the library runs for the decode workload (more heads than SMs; DR_DECODE_KERNEL=classic
