@@ -1,12 +1,13 @@
-"""The streaming decode kernel (persistent, one CTA per SM, head states copied ahead through a ring
-of shared-memory stages) against the one-CTA-per-head kernel and the oracle.
+"""The dk = dv = 128 decode paths against the one-CTA-per-head kernel and the oracle: the streaming
+kernel (persistent, two CTAs per SM, the next head's state copied ahead into shared memory) for more
+heads than SMs, and four CTAs per head (32 value columns each) for fewer.
 
-The library picks the dk = dv = 128 decode kernel once per process (DR_DECODE_KERNEL=classic keeps
-one CTA per head; by default more heads than SMs stream), so each runs in a child process on the same
-inputs: the decode workload (all 8192 heads, four chained in-place steps) and head counts just above
-the SM count and not a multiple of it, in every gate mode and with OSDN's write-key scale.  The two
-kernels do the same operations in the same order, so their outputs and states must agree bit for
-bit; the small cases are also checked against the float64 oracle.
+The library picks the path once per process (DR_DECODE_KERNEL=classic keeps one CTA per head), so
+each runs in a child process on the same inputs: the decode workload (all 8192 heads, four chained
+in-place steps), head counts just above the SM count and not a multiple of it, and small batches,
+in every gate mode and with OSDN's write-key scale.  Every path does the same operations in the
+same order per value column, so outputs and states must agree bit for bit; the small cases are also
+checked against the float64 oracle.
 """
 import os
 import subprocess
@@ -25,6 +26,9 @@ SMALL = [
     (10, 30, "scalar", "scalar", "none", "none"),
     (3, 101, "channel", "scalar", "channel", "channel"),
     (7, 43, "none", "channel", "scalar", "none"),
+    (4, 16, "scalar", "scalar", "none", "none"),         # the handoff batch: 64 heads, split 4 ways
+    (2, 74, "channel", "channel", "channel", "channel"),  # 148 heads
+    (1, 1, "channel", "scalar", "none", "channel"),
 ]
 
 

@@ -12,9 +12,12 @@
 // decoupled beta^v for FG2-GDN+).
 //
 // Memory-bound: each head's fp32 state (dk*dv*4 bytes) is read once and
-// written once with 16-byte (or 8-byte) coalesced accesses held in registers;
-// the two reductions go through shared memory.  One CTA of 256 threads per
-// head: warp w owns rows w, w+8, ...; lane l owns DV/32 consecutive columns.
+// written once with coalesced accesses held in registers; the two reductions
+// go through shared memory.  One CTA of 256 threads per head and slice of
+// DVF/NSL value columns (NSL > 1 spreads a small batch over more SMs; a value
+// column's reductions, error and update involve that column alone, so the
+// slices are independent and compute exactly what one CTA would): warp w owns
+// rows w, w+8, ...; lane l owns DVF/(32 NSL) consecutive columns of the slice.
 #pragma once
 #include "common.cuh"
 
@@ -23,8 +26,9 @@ namespace dr {
 template <int CPL> struct VecF;
 template <> struct VecF<4> { using T = float4; };
 template <> struct VecF<2> { using T = float2; };
+template <> struct VecF<1> { using T = float; };
 
-template <typename IO, int DK, int DV>
+template <typename IO, int DK, int DVF, int NSL = 1>
 __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
                    const float *__restrict__ alpha, int alpha_mode, const float *__restrict__ beta_k,
@@ -32,24 +36,26 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
                    const float *__restrict__ s_scale, float *__restrict__ S, IO *__restrict__ o) {
   constexpr int NW = 8;
   constexpr int RPW = DK / NW;
+  constexpr int DV = DVF / NSL;  // value columns of this CTA's slice
   constexpr int CPL = DV / 32;
   using V = typename VecF<CPL>::T;
-  static_assert(DK % NW == 0 && DV % 64 == 0, "unsupported head dims");
+  static_assert(DK % NW == 0 && DVF % NSL == 0 && DV % 32 == 0 && CPL <= 4, "unsupported head dims");
 
   __shared__ float s_al[DK], s_b[DK], s_a[DK], s_q[DK], s_w[DV], s_u[DV];
   __shared__ float s_red_r[NW][DV], s_red_p[NW][DV];
   __shared__ float s_bq;
 
-  const size_t bh = blockIdx.x;  // token-head index b*H + h (T == 1)
+  const size_t bh = blockIdx.x / NSL;  // token-head index b*H + h (T == 1)
+  const int v0 = static_cast<int>(blockIdx.x % NSL) * DV;  // first value column of the slice
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  float *Sh = S + bh * DK * DV;
+  float *Sh = S + bh * DK * DVF + v0;
 
   // 1. issue the state loads first so they are in flight while the factors are formed
   float s[RPW][CPL];
 #pragma unroll
   for (int rr = 0; rr < RPW; ++rr) {
     const int i = warp + rr * NW;
-    V x = __ldcs(reinterpret_cast<const V *>(Sh + i * DV + lane * CPL));
+    V x = __ldcs(reinterpret_cast<const V *>(Sh + i * DVF + lane * CPL));
     const float *xf = reinterpret_cast<const float *>(&x);
 #pragma unroll
     for (int c = 0; c < CPL; ++c) s[rr][c] = xf[c];
@@ -65,10 +71,10 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
     s_al[tid] = gate_at(alpha, alpha_mode, bh, DK, tid);
   }
   if (tid >= 128 && tid - 128 < DV) {
-    const int j = tid - 128;
-    const float vj = to_f32(v[bh * DV + j]);
-    const float ws = (beta_v_mode != MODE_ABSENT) ? gate_at(beta_v, beta_v_mode, bh, DV, j)
-                                                  : sqrtf(gate_at(beta_k, beta_k_mode, bh, DK, j));
+    const int j = tid - 128, jg = v0 + j;
+    const float vj = to_f32(v[bh * DVF + jg]);
+    const float ws = (beta_v_mode != MODE_ABSENT) ? gate_at(beta_v, beta_v_mode, bh, DVF, jg)
+                                                  : sqrtf(gate_at(beta_k, beta_k_mode, bh, DK, jg));
     s_w[j] = ws * vj;
   }
   __syncthreads();
@@ -112,7 +118,7 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
     }
     const float u = s_w[tid] - rs;
     s_u[tid] = u;
-    o[bh * DV + tid] = from_f32<IO>(fmaf(u, s_bq, ps));
+    o[bh * DVF + v0 + tid] = from_f32<IO>(fmaf(u, s_bq, ps));
   }
   __syncthreads();
 
@@ -125,7 +131,7 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
     float *xf = reinterpret_cast<float *>(&x);
 #pragma unroll
     for (int c = 0; c < CPL; ++c) xf[c] = fmaf(ai, s_u[lane * CPL + c], s[rr][c]);
-    __stcs(reinterpret_cast<V *>(Sh + i * DV + lane * CPL), x);
+    __stcs(reinterpret_cast<V *>(Sh + i * DVF + lane * CPL), x);
   }
 }
 

@@ -269,7 +269,8 @@ dr_status tc_ring_launch(const dr_problem *p, const int *cu, const void *q, cons
 
 // ----------------------------------------------------------------- decode
 // DR_DECODE_KERNEL=classic keeps dk = dv = 128 on one CTA per head (for comparisons); the default
-// streams the states through a persistent kernel once there are more heads than SMs.
+// splits each head over four CTAs when there are no more heads than SMs, and streams the states
+// through a persistent kernel when there are more.
 bool decode_stream_enabled() {
   static const bool on = [] {
     const char *e = std::getenv("DR_DECODE_KERNEL");
@@ -293,6 +294,12 @@ dr_status decode_launch(const dr_problem *p, const void *q, const void *k, const
   if (heads > 0x7fffffffLL) return DR_ERR_INVALID_ARG;
   if constexpr (DK == 128 && DV == 128) {
     const int sms = sm_count();
+    if (decode_stream_enabled() && sms > 0 && heads <= sms) {  // small batch: 4 CTAs per head
+      dr::decode_step_kernel<IO, DK, DV, 4><<<static_cast<unsigned>(heads * 4), 256, 0, st>>>(
+          static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v), alpha, p->alpha_mode,
+          beta_k, p->beta_k_mode, beta_v, p->beta_v_mode, s_scale, S, static_cast<IO *>(o));
+      return launch_status();
+    }
     if (decode_stream_enabled() && sms > 0 && heads > sms) {
       auto kern = dr::decode_stream_kernel<IO>;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
