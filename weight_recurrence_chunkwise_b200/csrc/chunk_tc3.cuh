@@ -406,12 +406,25 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         uint8_t *pA = tAC + blk * 64 * 128 + (rgl * RGL) * 128 + inb;
         float amax = 0.f;
         float ga = h0, gb = h1;  // gamma_r of the current row, two key channels
+        // rows in batches of RB: a batch's raw k and q are read before any of its results are
+        // written back in place, so their shared-memory loads overlap instead of each waiting
+        // behind the previous row's stores
+        constexpr int RB = kScaled ? 1 : 4;  // the scaled variant has no registers to spare
 #pragma unroll
-        for (int jj = 0; jj < RGL; ++jj) {
+        for (int j0 = 0; j0 < RGL; j0 += RB) {
+        __nv_bfloat162 kraw[RB], qraw[RB];
+#pragma unroll
+        for (int jb = 0; jb < RB; ++jb) {
+          const int jj = j0 + jb;
           const uint32_t sw = ((ch ^ static_cast<uint32_t>(jj & 7)) << 4) + jj * 128;
-          const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(pB + sw);  // raw k
-          const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(pQ + sw);  // raw q
-          const float2 kf = __bfloat1622float2(k2), qf = __bfloat1622float2(q2);
+          kraw[jb] = *reinterpret_cast<const __nv_bfloat162 *>(pB + sw);  // raw k
+          qraw[jb] = *reinterpret_cast<const __nv_bfloat162 *>(pQ + sw);  // raw q
+        }
+#pragma unroll
+        for (int jb = 0; jb < RB; ++jb) {
+          const int jj = j0 + jb;
+          const uint32_t sw = ((ch ^ static_cast<uint32_t>(jj & 7)) << 4) + jj * 128;
+          const float2 kf = __bfloat1622float2(kraw[jb]), qf = __bfloat1622float2(qraw[jb]);
           float s0, s1;
           if (beta_scalar) {
             s0 = s1 = tc::sqrt_fast(pbe[2 * jj]);
@@ -433,6 +446,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           *reinterpret_cast<uint32_t *>(pQ + sw) = pack_f16x2(ga * qf.x, gb * qf.y);  // Qh (in place of q)
           *reinterpret_cast<uint32_t *>(pB + sw) = pack_f16x2(ga * b0, gb * b1);      // Bh (in place of k)
           *reinterpret_cast<uint32_t *>(pA + sw) = pack_f16x2(a0, a1);                // Ac
+        }
         }
         if (!(amax < kF16Max)) raise_status(p.status, STATUS_RANGE);
       }
