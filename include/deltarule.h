@@ -181,9 +181,9 @@ DR_API dr_status dr_chunk_fwd_varlen(const dr_problem *p, const int *cu_seqlens,
                                      void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * Affine state maps, for a sequence split into consecutive segments (NEXT-4
- * of the build plan; the chunkwise form's linearity in the state, DeltaNet
- * page step 7 / FG2-GDN page section 2).  A segment maps its initial state to
+ * Affine state maps, for a sequence split into consecutive segments (the
+ * chunkwise form's linearity in the state, DeltaNet page step 7 / FG2-GDN
+ * page section 2).  A segment maps its initial state to
  * its final state as S_out = M S_in + N: N is the segment's final state from a
  * zero initial state (dr_chunk_fwd with S0 = NULL), and M (dk x dk) its final
  * state when the write vectors are zero and S0 = I (dr_chunk_fwd with v = 0,
@@ -197,7 +197,7 @@ DR_API dr_status dr_state_map_apply(int n, int dk, int dv, const float *M, const
                                     float *out, void *stream);
 
 /*
- * Backward pass (NEXT-3 of the build plan): the gradients of
+ * Backward pass: the gradients of
  *   L = sum(dout (.) o) + sum(dS_T (.) S_T)
  * with respect to every input of dr_chunk_fwd / dr_chunk_fwd_osdn, for the
  * forward defined by the recurrence (DeltaNet page steps 3-6; FG2-GDN page

@@ -1,4 +1,4 @@
-"""Sequence-parallel prefill (NEXT-4) on the CPU: two gloo ranks, each holding one segment of T.
+"""Sequence-parallel prefill on the CPU: two gloo ranks, each holding one segment of T.
 
 The ranks run weight_recurrence_chunkwise_b200.seqpar with the float64 oracle standing in for the
 prefill kernel and a float64 product for the map composition, so the test checks the algebra and the
