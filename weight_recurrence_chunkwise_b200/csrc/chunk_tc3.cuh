@@ -639,26 +639,6 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         pws = __ldg((p.beta_v_mode == MODE_SCALAR ? p.beta_v : p.beta_k) + th);
       }
     };
-    // ph: phase bits, bit `bit` is this barrier's parity
-    auto wait_all = [&](uint64_t *bar, uint32_t &ph, int bit, bool cluster_scope) -> bool {
-      const uint32_t par = (ph >> bit) & 1u;
-      const bool ok = cluster_scope ? mbar_wait_cluster(bar, par, kWaitLimitNs) : mbar_wait(bar, par, kWaitLimitNs);
-      ph ^= 1u << bit;
-      const bool fail = bar_or(BAR_CHAIN, NT - NL, !ok);
-      if (fail && ct == 0) raise_status(p.status, STATUS_TIMEOUT);
-      return !fail;
-    };
-    auto wait_one = [&](uint64_t *bar, uint32_t &ph, int bit, bool cluster_scope) -> bool {
-      const uint32_t par = (ph >> bit) & 1u;
-      bool ok = true;
-      if (ct == 0)
-        ok = cluster_scope ? mbar_wait_cluster(bar, par, kWaitLimitNs) : mbar_wait(bar, par, kWaitLimitNs);
-      ph ^= 1u << bit;
-      const bool fail = bar_or(BAR_CHAIN, NT - NL, !ok);
-      tc_fence_after();
-      if (fail && ct == 0) raise_status(p.status, STATUS_TIMEOUT);
-      return !fail;
-    };
     // write vectors of the chunk whose raw v sits in Wr, in place (after bar_v)
     auto convert_wr = [&](int wL) {  // wL: valid rows of the chunk
       float sc[16];
@@ -741,15 +721,24 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint64_t dS = sdesc_sw128(sbase_addr + OFF_S, 128 * 128, 1024);
     const uint64_t dWr = sdesc_sw128(sbase_addr + OFF_WR, 64 * 128, 1024);
 
-    // Software pipeline: the write vectors of chunk c+1 are built at the end of chunk c (their v is
-    // requested as soon as the first MMA group of chunk c has read Wr), and the outputs of chunk c
-    // are stored while the first MMA group of chunk c+1 runs (D3 alternates between two column sets).
+    // Software pipeline: the write vectors of chunk c+1 are built while the second MMA group of
+    // chunk c runs (their v is requested as soon as the first MMA group of chunk c has read Wr, and
+    // the second group does not read Wr), and the outputs of chunk c are stored while the first MMA
+    // group of chunk c+1 runs (D3 alternates between two column sets).
     if (nchunks > 0) {
       if (ct == 0) {
         issue_v(0);
         for (int c = 1; c < 3 && c < nchunks; ++c) tma_prefetch_l2_4d(&tm_v, v0, h, tt0 + c * C, tb);
       }
       prefetch_ws(0);
+      const bool ok_v = mbar_wait(&bar_v, ph_v & 1u, kWaitLimitNs);
+      ph_v ^= 1u;
+      if (ok_v) convert_wr(min(C, T));
+      fence_async_smem();
+      if (bar_or(BAR_CHAIN, NT - NL, !ok_v)) {
+        if (ct == 0) raise_status(p.status, STATUS_TIMEOUT);
+        aborted = true;
+      }
     }
     // iteration c builds the write vectors of chunk c and runs its state pass; the extra last
     // iteration only stores the outputs of the final chunk
@@ -761,15 +750,11 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const uint32_t cD3 = col_d3(c);
       float gc = 0.f;
       if (run) {
-        // v of this chunk (TMA data: every thread waits), its write vectors, then the slot; one
-        // group barrier decides both waits and orders the conversion before the MMAs
-        const bool ok_v = mbar_wait(&bar_v, ph_v & 1u, kWaitLimitNs);
-        ph_v ^= 1u;
-        if (ok_v) convert_wr(min(C, T - c * C));
-        fence_async_smem();
+        // the slot (its write vectors were built during the previous chunk, or before the loop);
+        // the group barrier also orders that conversion before the MMAs
         const bool ok_f = mbar_wait_cluster(&bar_full[j], (ph_full >> j) & 1u, kWaitLimitNs);
         ph_full ^= 1u << j;
-        if (bar_or(BAR_CHAIN, NT - NL, !(ok_v && ok_f))) {
+        if (bar_or(BAR_CHAIN, NT - NL, !ok_f)) {
           if (ct == 0) raise_status(p.status, STATUS_TIMEOUT);
           aborted = true;
           break;
@@ -863,7 +848,26 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         __syncwarp();
       }
-      if (!wait_one(&bar_cmma, ph_mma, 0, false)) { aborted = true; break; }
+      // while group 2 runs: v of chunk c+1 (TMA data: every thread waits) into write vectors, in
+      // place in Wr; then group 2's completion.  One group barrier decides both waits.
+      {
+        bool ok = true;
+        if (c + 1 < nchunks) {
+          ok = mbar_wait(&bar_v, ph_v & 1u, kWaitLimitNs);
+          ph_v ^= 1u;
+          if (ok) convert_wr(min(C, T - (c + 1) * C));
+          fence_async_smem();
+        }
+        if (ct == 0) ok = mbar_wait(&bar_cmma, ph_mma & 1u, kWaitLimitNs) && ok;
+        ph_mma ^= 1u;
+        const bool fail = bar_or(BAR_CHAIN, NT - NL, !ok);
+        tc_fence_after();
+        if (fail) {
+          if (ct == 0) raise_status(p.status, STATUS_TIMEOUT);
+          aborted = true;
+          break;
+        }
+      }
       // this CTA is done with slot j: tell the CTA that produces chunk c+3 into it
       if (ct == 128) {
         if (((c + 3) & 1) == rank) mbar_arrive(&bar_free[j]);
