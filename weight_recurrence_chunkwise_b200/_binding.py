@@ -118,13 +118,39 @@ def make_problem(q, v, alpha, beta_k, beta_v, chunk=64) -> dr_problem:
                       _mode(beta_k, 3), _mode(beta_v, 3))
 
 
+def _check_shapes(q, v, named, state_batch=None):
+    """Every tensor's shape against q [B, T, H, dk] and v [B, T, H, dv], and its device against q's.
+
+    The library sizes every access from these dimensions, so a mismatched tensor is refused here,
+    before anything is launched.  ``state_batch``: the leading size of the states when it is not B
+    (a packed batch: the number of sequences).
+    """
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D: [B, T, H, d]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    SB = B if state_batch is None else state_batch
+    tok, st = (B, T, H), (SB, H, dk, dv)
+    want = {"k": [tok + (dk,)], "s": [tok + (dk,)], "v": [tok + (dv,)], "o": [tok + (dv,)],
+            "dout": [tok + (dv,)], "alpha": [tok, tok + (dk,)], "beta_k": [tok, tok + (dk,)],
+            "beta_v": [tok, tok + (dv,)], "S0": [st], "S_T": [st], "S": [st], "dS_T": [st]}
+    for name, t in named:
+        if t is None:
+            continue
+        if tuple(t.shape) not in want[name]:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}; expected "
+                             + " or ".join(str(w) for w in want[name]))
+        if t.device != q.device:
+            raise ValueError(f"{name} is on {t.device}, q on {q.device}")
+
+
 def _check_tensors(io_dtype, named):
     for name, t in named:
         if t is None:
             continue
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor")
-        want = io_dtype if name in ("q", "k", "v", "o") else torch.float32
+        want = io_dtype if name in ("q", "k", "v", "o", "dout") else torch.float32
         if t.dtype != want:
             raise TypeError(f"{name} must be {want}, got {t.dtype}")
 
@@ -159,6 +185,8 @@ def dr_chunk_fwd_varlen(q, k, v, beta_k, cu_seqlens, alpha=None, beta_v=None, s=
     n = cu_seqlens.numel() - 1
     if n < 1:
         raise ValueError("cu_seqlens needs at least two entries")
+    _check_shapes(q, v, [("k", k), ("v", v), ("o", o), ("alpha", alpha), ("beta_k", beta_k), ("beta_v", beta_v),
+                         ("s", s), ("S0", S0), ("S_T", S_T)], state_batch=n)
     p = make_problem(q, v, alpha, beta_k, beta_v, chunk)
     p.B = n
     dev = q.device
@@ -184,6 +212,8 @@ def dr_chunk_fwd_varlen(q, k, v, beta_k, cu_seqlens, alpha=None, beta_v=None, s=
 
 
 def _chunk_fwd(s, q, k, v, beta_k, alpha, beta_v, S0, chunk, o, S_T, workspace, stream, final_state):
+    _check_shapes(q, v, [("k", k), ("v", v), ("o", o), ("alpha", alpha), ("beta_k", beta_k), ("beta_v", beta_v),
+                         ("s", s), ("S0", S0), ("S_T", S_T)])
     p = make_problem(q, v, alpha, beta_k, beta_v, chunk)
     dev = q.device
     if o is None:
@@ -220,6 +250,8 @@ def dr_chunk_fwd_noalloc(q, k, v, beta_k, alpha=None, beta_v=None, S0=None, chun
     must be passed in by such callers (they are only allocated here when
     omitted, as a convenience for tests).  Returns ``(o, S_T)``.
     """
+    _check_shapes(q, v, [("k", k), ("v", v), ("o", o), ("alpha", alpha), ("beta_k", beta_k), ("beta_v", beta_v),
+                         ("S0", S0), ("S_T", S_T)])
     p = make_problem(q, v, alpha, beta_k, beta_v, chunk)
     if o is None:
         o = torch.empty(q.shape[:3] + (p.dv,), dtype=q.dtype, device=q.device)
@@ -248,6 +280,12 @@ def dr_decode_step_osdn(q, k, v, beta_k, S, s, alpha=None, beta_v=None, o=None, 
 
 
 def _decode_step(s, q, k, v, beta_k, S, alpha, beta_v, o, stream):
+    if q.dim() == 4 and q.shape[1] != 1:
+        raise ValueError("a decode step takes one token: q [B, 1, H, dk]")
+    _check_shapes(q, v, [("k", k), ("v", v), ("o", o), ("alpha", alpha), ("beta_k", beta_k), ("beta_v", beta_v),
+                         ("s", s), ("S", S)])
+    if S is None:
+        raise ValueError("S (the state to update in place) is required")
     p = make_problem(q, v, alpha, beta_k, beta_v, 0)
     if o is None:
         o = torch.empty(q.shape[:3] + (p.dv,), dtype=q.dtype, device=q.device)
@@ -291,12 +329,14 @@ def dr_backward(q, k, v, beta_k, dout, alpha=None, beta_v=None, s=None, S0=None,
 
     Returns a dict with keys q, k, v, beta_k, alpha, beta_v, s, S0 (None where absent / not wanted).
     """
+    _check_shapes(q, v, [("k", k), ("v", v), ("dout", dout), ("alpha", alpha), ("beta_k", beta_k),
+                         ("beta_v", beta_v), ("s", s), ("S0", S0), ("dS_T", dS_T)])
     p = make_problem(q, v, alpha, beta_k, beta_v, 64)
     dev = q.device
     f32 = lambda t: None if t is None else torch.empty(t.shape, dtype=torch.float32, device=dev)
     g = {"q": f32(q), "k": f32(k), "v": f32(v), "alpha": f32(alpha), "beta_k": f32(beta_k), "beta_v": f32(beta_v),
          "s": f32(s), "S0": torch.empty((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=dev) if want_dS0 else None}
-    _check_tensors(q.dtype, [("q", q), ("k", k), ("v", v), ("o", dout), ("alpha", alpha), ("beta_k", beta_k),
+    _check_tensors(q.dtype, [("q", q), ("k", k), ("v", v), ("dout", dout), ("alpha", alpha), ("beta_k", beta_k),
                              ("beta_v", beta_v), ("s", s), ("S0", S0), ("S_T", dS_T)])
     if s is not None and tuple(s.shape) != tuple(q.shape):
         raise ValueError("s must have the shape of q / k")
