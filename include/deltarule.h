@@ -37,7 +37,8 @@
  * Every pointer must be 16-byte aligned.
  *
  * Supported sizes: dk, dv in {64, 128}; chunk in {16, 32, 64}; T >= 0 (a
- * partial last chunk is handled); B, H >= 1.
+ * partial last chunk is handled); B, H >= 1; for the prefill B, H <= 65535
+ * (they index a launch grid's y and z), and for the decode B * H < 2^31.
  *
  * Ownership and threading: the caller owns every buffer; the library
  * allocates no device memory and keeps no state between calls.  All work is
@@ -73,7 +74,7 @@ extern "C" {
 typedef enum {
   DR_OK = 0,
   DR_ERR_INVALID_ARG = 1,   /* NULL required pointer, negative size, mode/shape mismatch */
-  DR_ERR_UNSUPPORTED = 2,   /* valid but not implemented: dk/dv/chunk outside the lists above */
+  DR_ERR_UNSUPPORTED = 2,   /* valid but not implemented: sizes outside the lists above */
   DR_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
   DR_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than dr_chunk_fwd_workspace() */
   DR_ERR_RANGE = 5,         /* device: cumulative decay inside a chunk below the factorised range */

@@ -86,6 +86,8 @@ def _chunk(lib, p, q=FAKE, alpha=FAKE, beta_v=None, ws=FAKE, ws_bytes=256):
     (dict(dk=96), B.DR_ERR_UNSUPPORTED),
     (dict(dv=256), B.DR_ERR_UNSUPPORTED),
     (dict(chunk=48), B.DR_ERR_UNSUPPORTED),
+    (dict(H=70000), B.DR_ERR_UNSUPPORTED),  # the prefill grids index H and B in y and z
+    (dict(B=65536), B.DR_ERR_UNSUPPORTED),
     (dict(chunk=0), B.DR_ERR_INVALID_ARG),
     (dict(io_dtype=7), B.DR_ERR_INVALID_ARG),
     (dict(beta_k_mode=B.DR_ABSENT), B.DR_ERR_INVALID_ARG),

@@ -56,6 +56,7 @@ dr_status check_common(const dr_problem *p, bool decode) {
   if (p->beta_v_mode == DR_ABSENT && p->beta_k_mode == DR_CHANNEL && p->dk != p->dv) return DR_ERR_INVALID_ARG;
   if ((p->dk != 64 && p->dk != 128) || (p->dv != 64 && p->dv != 128)) return DR_ERR_UNSUPPORTED;
   if (!decode && p->chunk != 16 && p->chunk != 32 && p->chunk != 64) return DR_ERR_UNSUPPORTED;
+  if (!decode && (p->B > 65535 || p->H > 65535)) return DR_ERR_UNSUPPORTED;  // launch grid y and z
   const double elems = double(p->B) * p->T * p->H * (p->dk > p->dv ? p->dk : p->dv);
   if (elems > 9.0e15) return DR_ERR_INVALID_ARG;
   return DR_OK;
