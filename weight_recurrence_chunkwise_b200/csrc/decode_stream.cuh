@@ -8,16 +8,16 @@
 // The step moves 128 KiB of fp32 state per head (read, then written in place) and does about one
 // flop per byte, so it is bound by HBM.  decode_step_kernel (one CTA per head, two per SM) has a
 // head's loads in flight only while that CTA waits on them, and none while it reduces and stores.
-// Here two CTAs per SM each walk heads blockIdx.x, blockIdx.x + gridDim.x, ...: as soon as a
-// thread has moved its 16 x 4 tile of the current head from shared memory into registers, it
-// copies its tile of the CTA's next head into the same place with 16-byte asynchronous copies
-// (cp.async, one commit group per head), so that load is in flight while the current head is
-// reduced, updated and stored from registers.  A thread reads back only the tile it copied itself,
-// so the stage needs no block barrier; the next head's per-row factors are loaded into registers
-// during the current head and published at its end.  One 64 KiB stage per CTA keeps two CTAs (16
-// warps) on each SM; a deeper ring with one CTA per SM was slower (its single CTA serialises every
-// head's reduce-update chain).  Tile layout as in decode_step_kernel: warp w owns rows w, w+8,
-// ...; lane l owns columns 4l..4l+3.
+// Here two CTAs per SM each walk heads blockIdx.x, blockIdx.x + gridDim.x, ...: once the CTA has
+// moved the current head from shared memory into registers (the first block barrier of the step
+// orders those reads before any overwrite), every thread copies its 16 x 4 tile of the CTA's next
+// head into the same place with 16-byte asynchronous copies (cp.async, one commit group per head),
+// so that load is in flight while the current head is reduced, updated and stored from registers.
+// A thread reads back only the tile it copied itself, so its wait_group is all the landing needs;
+// the next head's per-row factors are loaded into registers during the current head and published
+// at its end.  One 64 KiB stage per CTA keeps two CTAs (16 warps) on each SM; a deeper ring with
+// one CTA per SM was slower (its single CTA serialises every head's reduce-update chain).  Tile
+// layout as in decode_step_kernel: warp w owns rows w, w+8, ...; lane l owns columns 4l..4l+3.
 #pragma once
 #include "common.cuh"
 
@@ -115,8 +115,8 @@ decode_stream_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const I
     const long long bh_next = bh + G;
     Raw fn;
     if (bh_next < nheads) load_raw(bh_next, fn);
-    // this thread's tile of the current head has landed: into registers, then the stage takes the
-    // head NST ahead (one commit group per iteration, empty past the last head)
+    // this thread's tile of the current head has landed: into registers (the stage takes the head
+    // NST ahead once the block barrier below has ordered these reads before the copies)
     cp_async_wait_group<NST - 1>();
     float s[RPW][CPL];
     {
@@ -127,9 +127,6 @@ decode_stream_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const I
         s[rr][0] = x.x, s[rr][1] = x.y, s[rr][2] = x.z, s[rr][3] = x.w;
       }
     }
-    const long long bh_ahead = bh + NST * G;
-    if (bh_ahead < nheads) issue_state(bh_ahead, stg);
-    cp_async_commit_group();
     if (warp == 0) {
       float acc = 0.f;
       for (int i = lane; i < DK; i += 32) acc += s_a[buf][i] * s_q[buf][i];
@@ -158,6 +155,11 @@ decode_stream_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const I
       s_red_p[warp][lane * CPL + c] = p[c];
     }
     __syncthreads();
+    // every thread's reads of the stage are complete: copy in the head NST ahead (one commit group
+    // per iteration, empty past the last head)
+    const long long bh_ahead = bh + NST * G;
+    if (bh_ahead < nheads) issue_state(bh_ahead, stg);
+    cp_async_commit_group();
     // finish the reductions; error u and output o per value column
     if (tid < DV) {
       float rs = 0.f, ps = 0.f;
