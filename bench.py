@@ -66,8 +66,8 @@ def decode_bytes(B, H, dk, dv, io=2, alpha_ch=True, beta_ch=True):
 # voids the number, and the workload it was taken on, so other workloads report none.
 RING_SOURCES = ("chunk_tc3.cuh", "chunk_tc.cuh", "tri_inverse.cuh", "sm100.cuh", "common.cuh")
 MEASURED_TRAFFIC = {
-    ("chunk_fwd_ring_kernel", "gdn_bf16"): ("f43247f89c6c", 249.243904e6, RING_SOURCES),
-    ("decode_stream_kernel", "decode_bf16"): ("f9a46a4cdf2e", 1032.60288e6, ("decode_stream.cuh", "common.cuh")),
+    ("chunk_fwd_ring_kernel", "gdn_bf16"): ("f89185e36ba6", 250.54976e6, RING_SOURCES),
+    ("decode_stream_kernel", "decode_bf16"): ("6cb82d40c1fd", 1031.005696e6, ("decode_stream.cuh", "common.cuh")),
 }
 
 # Decode kernel the library runs for the decode workload (more heads than SMs; DR_DECODE_KERNEL=classic
