@@ -68,6 +68,7 @@ RING_SOURCES = ("chunk_tc3.cuh", "chunk_tc.cuh", "tri_inverse.cuh", "sm100.cuh",
 MEASURED_TRAFFIC = {
     ("chunk_fwd_ring_kernel", "gdn_bf16"): ("f89185e36ba6", 250.54976e6, RING_SOURCES),
     ("decode_stream_kernel", "decode_bf16"): ("6cb82d40c1fd", 1031.005696e6, ("decode_stream.cuh", "common.cuh")),
+    ("delta_rule_bwd_kernel", "gdn_bf16"): ("9a0d1d786d6e", 10536.615e6, ("backward.cuh", "common.cuh")),
 }
 
 # Decode kernel the library runs for the decode workload (more heads than SMs; DR_DECODE_KERNEL=classic
@@ -314,6 +315,7 @@ def run_backward(args, dr, p, x, dev, st, peaks, peaks_src):
     print(json.dumps({"backward": True, "workload": p.name, "ms": ms,
                       "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                    "frac": gbs / peaks["hbm_gbs"], "peak_source": peaks_src,
+                                   "traffic": measured_traffic("delta_rule_bwd_kernel", p.name),
                                    "kernel": "delta_rule_bwd_kernel", "algorithmic_bytes_per_launch": byts}}),
           flush=True)
     return 0
