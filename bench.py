@@ -331,6 +331,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1000,
                     help="chained in-place decode steps timed (the decode workload is 1000 steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--serial-steps", action="store_true",
+                    help="run each step's handoff decode after its prefill on one stream (no overlap of steps)")
     ap.add_argument("--only-prefill", action="store_true",
                     help="profiling aid: time only the prefill step (no decode workload, e2e or CPU leg)")
     ap.add_argument("--only-decode", action="store_true",
@@ -383,30 +385,48 @@ def main():
     assert dr.dr_workspace_status(ws_buf) == dr.DR_OK
 
     n = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    # Steps are pipelined unless --serial-steps: step i's handoff decode runs on a second stream
+    # beside step i+1's prefill (which leaves 20 of the 148 SMs free), with the final state
+    # double-buffered; the prefill's stream has the higher priority.  Every step still does all of
+    # its work inside the timed region.
+    pipelined = not (args.serial_steps or args.only_prefill)
+    pf = torch.cuda.Stream(device=dev, priority=-1) if pipelined else st
+    dec = torch.cuda.Stream(device=dev) if pipelined else st
+    S_buf = [S, torch.empty_like(S)] if pipelined else [S, S]
+    o1_buf = [o1, torch.empty_like(o1)] if pipelined else [o1, o1]
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    ev = [(mk(), mk(), mk(), mk()) for _ in range(n)]  # prefill start / end, decode start / end
     barrier(ws)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(st)
+        t_start, t_end = mk(), mk()
+        t_start.record(pf)
+        if dec is not pf:
+            dec.wait_event(t_start)
         for i in range(n):
-            ev[i][0].record(st)
+            j = i % 2
+            if pipelined and i >= 2:
+                pf.wait_event(ev[i - 2][3])  # the decode of step i-2 is done with S_buf[j]
+            ev[i][0].record(pf)
             dr.dr_chunk_fwd(x["q"], x["k"], x["v"], x["beta_k"], alpha=x["alpha"], beta_v=x["beta_v"], S0=None,
-                            chunk=p.chunk, o=o, S_T=S, workspace=ws_buf, stream=st)
-            ev[i][1].record(st)
+                            chunk=p.chunk, o=o, S_T=S_buf[j], workspace=ws_buf, stream=pf)
+            ev[i][1].record(pf)
+            if dec is not pf:
+                dec.wait_event(ev[i][1])
+            ev[i][2].record(dec)
             if not args.only_prefill:
-                dr.dr_decode_step(nxt["q"], nxt["k"], nxt["v"], nxt["beta_k"], S, alpha=nxt["alpha"], o=o1,
-                                  stream=st)
-            ev[i][2].record(st)
-        t_end.record(st)
+                dr.dr_decode_step(nxt["q"], nxt["k"], nxt["v"], nxt["beta_k"], S_buf[j], alpha=nxt["alpha"],
+                                  o=o1_buf[j], stream=dec)
+            ev[i][3].record(dec)
+        if dec is not pf:
+            pf.wait_stream(dec)
+        t_end.record(pf)
         torch.cuda.synchronize()
     barrier(ws)
     ms_total = max_over_ranks(t_start.elapsed_time(t_end), ws, dev)
     ms_step = ms_total / n
-    prefill_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
-    handoff_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    prefill_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    handoff_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
     tok_heads = p.B * p.H * (p.T + 1)
     value = tok_heads * ws / (ms_step / 1e3) / 1e6
 
@@ -575,8 +595,10 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": p.name, "B": p.B, "H": p.H, "T": p.T, "dk": p.dk, "dv": p.dv, "chunk": p.chunk,
                    "step": "chunkwise prefill of T tokens + one decode step per (b,h)", "parallelism": f"dp{ws}",
-                   "l2": "inputs (275 MB per rank) larger than the 126 MB L2; no flush between steps"},
-        "prefill_ms": prefill_ms, "handoff_decode_ms": handoff_ms,
+                   "l2": "inputs (275 MB per rank) larger than the 126 MB L2; no flush between steps",
+                   "pipeline": ("step i's handoff decode on a second stream beside step i+1's prefill"
+                                if pipelined else "serial: prefill, then its handoff decode, on one stream")},
+        "prefill_ms": prefill_ms, "handoff_decode_ms": handoff_ms, "step_serial_ms": prefill_ms + handoff_ms,
         "roofline": roofline, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
         "gpu_launches": 2 * n, "clocks": clk.summary(),
     }
