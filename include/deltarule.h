@@ -244,20 +244,34 @@ DR_API dr_status dr_backward(const dr_problem *p,
  * DR_ERR_WORKSPACE before anything is enqueued.  The call allocates nothing
  * (no cudaMalloc, no cudaFree, no allocating library routine).
  * Device and set-up: the GPU used is the current device, which must be the
- * device of `stream`.  The first call on each device looks up the array's
- * device address (cudaGetSymbolAddress) and caches it; make that first call
- * before any stream capture.
+ * device of `stream` and the device that holds q; a q on another device is
+ * refused with DR_ERR_INVALID_ARG.  The first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress) and caches it for the
+ * life of the process; make that first call before any stream capture, and
+ * after the last cudaDeviceReset of that device (a reset reloads the library's
+ * device code, and the cached address would then be stale).
  * Sharing: every call on a device uses the same array, which keeps the last
  * call's contents; each call clears the status word on its own stream before
  * its kernel runs.  Calls whose work overlaps on the GPU (several streams, or
  * several host threads) race on that word, so its device-side status is only
- * meaningful for calls that do not overlap; the array is not readable
- * through dr_workspace_status.
+ * meaningful for calls that do not overlap.  Read it with dr_noalloc_status().
  */
 DR_API dr_status dr_chunk_fwd_noalloc(const dr_problem *p,
                                       const void *q, const void *k, const void *v,
                                       const float *alpha, const float *beta_k, const float *beta_v,
                                       const float *S0, void *o, float *S_T, void *stream);
+
+/*
+ * Device status of the last dr_chunk_fwd_noalloc call on the current device
+ * (the pages have no counterpart): synchronises `stream`, then reads the
+ * status word from the library's static array and returns DR_OK,
+ * DR_ERR_RANGE (a chunk's cumulative decay left the factorised range) or
+ * DR_ERR_TIMEOUT (a bounded device wait expired).  Allocates nothing.
+ * Returns DR_ERR_INVALID_ARG if dr_chunk_fwd_noalloc has not run on the
+ * current device yet, DR_ERR_CUDA if the copy fails.  Like the entry point,
+ * it reports the last call only when calls do not overlap on the GPU.
+ */
+DR_API dr_status dr_noalloc_status(void *stream);
 
 /*
  * Synchronises `stream`, then reads the status word a previous dr_chunk_fwd

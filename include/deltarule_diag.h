@@ -1,13 +1,17 @@
 /*
  * deltarule_diag.h -- diagnostic entry points of libdeltarule (not part of the
- * operation itself; the pages have no counterpart).  They exercise the
- * tensor-core building blocks of the prefill kernel in isolation so that a
- * layout or descriptor fault is found before it hides inside the full kernel.
+ * operation itself; the pages have no counterpart).  They run a named kernel
+ * in place of the library's choice, so that the kernels can be compared on the
+ * same problem, exercise the tensor-core building blocks of the prefill kernel
+ * in isolation so that a layout or descriptor fault is found before it hides
+ * inside the full kernel, and run the kernels' bounded waits out on purpose.
  */
 #ifndef DELTARULE_DIAG_H
 #define DELTARULE_DIAG_H
 
 #include <stddef.h>
+
+#include "deltarule.h"
 
 #ifndef DR_API
 #if defined(__GNUC__)
@@ -20,6 +24,41 @@
 #ifdef __cplusplus
 extern "C" {
 #endif
+
+/*
+ * dr_chunk_fwd through a named kernel instead of the library's choice, so
+ * that the kernels can be compared with one another on the same problem:
+ *   variant 0  the library's choice (what dr_chunk_fwd runs)
+ *   variant 1  the tensor-core kernel with one CTA per 64-column value slice
+ *              (bf16 I/O, dk = 128, chunk 64, dv a multiple of 64); the
+ *              library's choice for such shapes when dv != 128
+ *   variant 2  the CUDA-core kernel (every supported shape; the library's
+ *              choice for fp32 I/O and for chunk 16 and 32)
+ * Arguments, layouts, ownership and errors are those of dr_chunk_fwd; a
+ * variant that cannot take the problem returns DR_ERR_UNSUPPORTED before
+ * anything is enqueued.  Every variant computes the same operation.
+ */
+DR_API int dr_diag_chunk_fwd_variant(int variant, const dr_problem *p, const void *q, const void *k,
+                                     const void *v, const float *alpha, const float *beta_k,
+                                     const float *beta_v, const float *S0, void *o, float *S_T,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * dr_decode_step (s == NULL) or dr_decode_step_osdn (s != NULL) through a
+ * named kernel:
+ *   variant 0  the library's choice
+ *   variant 1  one CTA per head
+ *   variant 2  four CTAs per head, 32 value columns each (dk = dv = 128)
+ *   variant 3  the persistent streaming kernel, two CTAs per SM, the next
+ *              head's state copied ahead into shared memory (dk = dv = 128)
+ * All variants perform the same operations in the same order per value
+ * column, so they give the same bits.  Arguments and errors as in
+ * dr_decode_step; an unsupported variant returns DR_ERR_UNSUPPORTED.
+ */
+DR_API int dr_diag_decode_step_variant(int variant, const dr_problem *p, const void *q, const void *k,
+                                       const void *v, const float *alpha, const float *beta_k,
+                                       const float *beta_v, const float *s, float *S, void *o,
+                                       void *stream);
 
 /*
  * D[128 x N] = A[128 x K] * B[K x N] on one CTA through tcgen05.mma (16-bit

@@ -1,20 +1,16 @@
-"""GPU parity of each tensor-core prefill kernel for dk = dv = 128, chunk 64.
+"""GPU parity of every prefill kernel on the same problems, for dk = dv = 128 and chunk 64.
 
-The library picks its kernel once per process from DR_PREFILL_KERNEL (ring: default, two CTAs
-and three factor slots; pair: two CTAs and two slots; single: one CTA per value slice), so each
-variant runs in a child process.  Cases cover ragged lengths, one to many chunks (the slot ring
-wraps several times), scalar and channel gates, and the symmetric and separate write strengths.
+The library's choice (dr_chunk_fwd) and the other kernels, named through
+dr_diag_chunk_fwd_variant (include/deltarule_diag.h): the tensor-core kernel with one CTA per
+64-column value slice, and the CUDA-core kernel.  Cases cover ragged lengths, one to many chunks
+(the factor-slot ring wraps several times), scalar and channel gates, and the symmetric and
+separate write strengths; each result is checked against the float64 oracle.
 """
-import os
-import subprocess
-import sys
 import zlib
 
 import pytest
 
 pytestmark = pytest.mark.gpu
-
-ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 CASES = [
     # (T, alpha, beta_k, beta_v, S0)
@@ -30,39 +26,39 @@ CASES = [
 ]
 
 
-def _run_cases():
-    import numpy as np  # noqa: F401
-    import torch
-
-    sys.path.insert(0, ROOT)
-    import weight_recurrence_chunkwise_b200 as dr
-    from synth import make_inputs, problem
-    from tests.test_gpu_parity import check, ref_prefill, run_prefill
-
-    dr.lib()
-    for case in CASES:
-        T, a, bk, bv, s0 = case
-        p = problem("kda_bf16", B=1, H=3, T=T, dk=128, dv=128, chunk=64, io="bf16", alpha=a, beta_k=bk,
-                    beta_v=bv, S0=s0, seed=zlib.crc32(repr(case).encode()) % 1000)
-        x = make_inputs(p)
-        o, S_T = run_prefill(dr, x, 64)
-        ref_o, ref_S = ref_prefill(x)
-        e_o, e_S = check(p, o, S_T, ref_o, ref_S)
-        print(f"{os.environ.get('DR_PREFILL_KERNEL', 'ring')} {case}: err_o={e_o:.2e} err_S={e_S:.2e}")
-    assert torch.cuda.is_available()
-
-
-@pytest.mark.parametrize("variant", ["ring", "pair", "single"])
+@pytest.mark.parametrize("variant", ["default", "single", "simt"])
 def test_prefill_kernel_variant(variant):
     import torch
 
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    env = dict(os.environ, DR_PREFILL_KERNEL=variant)
-    r = subprocess.run([sys.executable, os.path.abspath(__file__)], env=env, cwd=ROOT, capture_output=True,
-                       text=True, timeout=600)
-    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-4000:]
+    import weight_recurrence_chunkwise_b200 as dr
+    from synth import make_inputs, problem
+    from tests.test_gpu_parity import check, ref_prefill
+
+    for case in CASES:
+        T, a, bk, bv, s0 = case
+        p = problem("kda_bf16", B=1, H=3, T=T, dk=128, dv=128, chunk=64, io="bf16", alpha=a, beta_k=bk,
+                    beta_v=bv, S0=s0, seed=zlib.crc32(repr(case).encode()) % 1000)
+        x = make_inputs(p)
+        g = {n: (None if t is None else t.cuda()) for n, t in x.items()}
+        o, S_T = dr.dr_diag_chunk_fwd_variant(variant, g["q"], g["k"], g["v"], g["beta_k"], alpha=g["alpha"],
+                                              beta_v=g["beta_v"], S0=g["S0"], chunk=64)
+        torch.cuda.synchronize()
+        ref_o, ref_S = ref_prefill(x)
+        check(p, o.cpu(), S_T.cpu(), ref_o, ref_S)
 
 
-if __name__ == "__main__":
-    _run_cases()
+def test_unsupported_variant_is_refused():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import weight_recurrence_chunkwise_b200 as dr
+    from synth import make_inputs, problem
+
+    p = problem("deltanet_f32", B=1, H=1, T=64)  # fp32 I/O: no tensor-core kernel
+    g = {n: (None if t is None else t.cuda()) for n, t in make_inputs(p).items()}
+    with pytest.raises(dr.DeltaRuleError) as e:
+        dr.dr_diag_chunk_fwd_variant("single", g["q"], g["k"], g["v"], g["beta_k"], alpha=g["alpha"], chunk=64)
+    assert e.value.code == dr.DR_ERR_UNSUPPORTED

@@ -41,8 +41,12 @@ _lib = None
 EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_chunk_fwd_osdn", "dr_chunk_fwd_varlen",
            "dr_chunk_fwd_noalloc", "dr_decode_step",
            "dr_decode_step_osdn", "dr_state_map_apply", "dr_backward_workspace", "dr_backward",
-           "dr_workspace_status", "dr_status_string", "dr_version", "dr_diag_umma_selftest",
-           "dr_diag_tri_inverse", "dr_diag_wait_timeout")
+           "dr_workspace_status", "dr_noalloc_status", "dr_status_string", "dr_version", "dr_diag_umma_selftest",
+           "dr_diag_tri_inverse", "dr_diag_wait_timeout", "dr_diag_chunk_fwd_variant", "dr_diag_decode_step_variant")
+
+# kernels of dr_diag_chunk_fwd_variant / dr_diag_decode_step_variant (include/deltarule_diag.h)
+PREFILL_VARIANTS = {"default": 0, "single": 1, "simt": 2}
+DECODE_VARIANTS = {"default": 0, "per_head": 1, "split4": 2, "stream": 3}
 
 
 def lib():
@@ -75,6 +79,8 @@ def lib():
         L.dr_decode_step_osdn.restype = ctypes.c_int
         L.dr_workspace_status.argtypes = [vp, vp]
         L.dr_workspace_status.restype = ctypes.c_int
+        L.dr_noalloc_status.argtypes = [vp]
+        L.dr_noalloc_status.restype = ctypes.c_int
         L.dr_status_string.argtypes = [ctypes.c_int]
         L.dr_status_string.restype = ctypes.c_char_p
         L.dr_version.argtypes = []
@@ -85,6 +91,10 @@ def lib():
         L.dr_diag_tri_inverse.restype = ctypes.c_int
         L.dr_diag_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_ulonglong, vp, vp, vp]
         L.dr_diag_wait_timeout.restype = ctypes.c_int
+        L.dr_diag_chunk_fwd_variant.argtypes = [ctypes.c_int, P] + [vp] * 9 + [vp, sz, vp]
+        L.dr_diag_chunk_fwd_variant.restype = ctypes.c_int
+        L.dr_diag_decode_step_variant.argtypes = [ctypes.c_int, P] + [vp] * 9 + [vp]
+        L.dr_diag_decode_step_variant.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -97,10 +107,30 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
+def _stream(stream, device):
+    """The raw handle of ``stream``, else of ``device``'s current stream; a stream of another device
+    than the data's is refused (its kernels would run on one GPU with another GPU's pointers)."""
+    device = _dev(device)
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(device):
+    """``device`` as a CUDA device with an index (a bare "cuda" is the current device)."""
+    device = torch.device(device)
+    if device.type != "cuda":
+        raise ValueError(f"expected a CUDA device, got {device}")
+    return device if device.index is not None else torch.device("cuda", torch.cuda.current_device())
+
+
+def _call(name, device, *args):
+    """Call library function ``name`` with ``device`` current: the library launches on, and looks up
+    per-device state of, the current device."""
+    with torch.cuda.device(_dev(device)):
+        return getattr(lib(), name)(*args)
 
 
 def _mode(x, scalar_ndim):
@@ -165,6 +195,13 @@ def dr_chunk_fwd(q, k, v, beta_k, alpha=None, beta_v=None, S0=None, chunk=64, o=
     return _chunk_fwd(None, q, k, v, beta_k, alpha, beta_v, S0, chunk, o, S_T, workspace, stream, final_state)
 
 
+def dr_diag_chunk_fwd_variant(variant, q, k, v, beta_k, alpha=None, beta_v=None, S0=None, chunk=64, o=None,
+                              S_T=None, workspace=None, stream=None):
+    """dr_chunk_fwd through a named kernel (``PREFILL_VARIANTS``) instead of the library's choice."""
+    return _chunk_fwd(None, q, k, v, beta_k, alpha, beta_v, S0, chunk, o, S_T, workspace, stream, True,
+                      variant=PREFILL_VARIANTS[variant])
+
+
 def dr_chunk_fwd_osdn(q, k, v, beta_k, s, alpha=None, beta_v=None, S0=None, chunk=64, o=None, S_T=None,
                       workspace=None, stream=None, final_state=True):
     """Chunkwise prefill with OSDN's write-side key scale ``s`` [B, T, H, dk] (write key a = s * b)."""
@@ -203,15 +240,17 @@ def dr_chunk_fwd_varlen(q, k, v, beta_k, cu_seqlens, alpha=None, beta_v=None, s=
     need = workspace_bytes(p)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    rc = lib().dr_chunk_fwd_varlen(ctypes.byref(p), _ptr(cu_seqlens), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
-                                   _ptr(beta_k), _ptr(beta_v), _ptr(s), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
-                                   ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if cu_seqlens.device != dev:
+        raise ValueError(f"cu_seqlens is on {cu_seqlens.device}, q on {dev}")
+    rc = _call("dr_chunk_fwd_varlen", dev, ctypes.byref(p), _ptr(cu_seqlens), _ptr(q), _ptr(k), _ptr(v),
+               _ptr(alpha), _ptr(beta_k), _ptr(beta_v), _ptr(s), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+               ctypes.c_size_t(workspace.numel()), _stream(stream, dev))
     if rc != DR_OK:
         raise DeltaRuleError(rc, "dr_chunk_fwd_varlen")
     return o, S_T
 
 
-def _chunk_fwd(s, q, k, v, beta_k, alpha, beta_v, S0, chunk, o, S_T, workspace, stream, final_state):
+def _chunk_fwd(s, q, k, v, beta_k, alpha, beta_v, S0, chunk, o, S_T, workspace, stream, final_state, variant=None):
     _check_shapes(q, v, [("k", k), ("v", v), ("o", o), ("alpha", alpha), ("beta_k", beta_k), ("beta_v", beta_v),
                          ("s", s), ("S0", S0), ("S_T", S_T)])
     p = make_problem(q, v, alpha, beta_k, beta_v, chunk)
@@ -227,15 +266,22 @@ def _chunk_fwd(s, q, k, v, beta_k, alpha, beta_v, S0, chunk, o, S_T, workspace, 
     need = workspace_bytes(p)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    if s is None:
-        rc = lib().dr_chunk_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
-                                _ptr(beta_v), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
-                                ctypes.c_size_t(workspace.numel()), _stream(stream))
+    elif workspace.device != dev:
+        raise ValueError(f"workspace is on {workspace.device}, q on {dev}")
+    if variant is not None:
+        rc = _call("dr_diag_chunk_fwd_variant", dev, int(variant), ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                   _ptr(alpha), _ptr(beta_k), _ptr(beta_v), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+                   ctypes.c_size_t(workspace.numel()), _stream(stream, dev))
+        name = "dr_diag_chunk_fwd_variant"
+    elif s is None:
+        rc = _call("dr_chunk_fwd", dev, ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
+                   _ptr(beta_v), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+                   ctypes.c_size_t(workspace.numel()), _stream(stream, dev))
         name = "dr_chunk_fwd"
     else:
-        rc = lib().dr_chunk_fwd_osdn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
-                                     _ptr(beta_v), _ptr(s), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
-                                     ctypes.c_size_t(workspace.numel()), _stream(stream))
+        rc = _call("dr_chunk_fwd_osdn", dev, ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                   _ptr(beta_k), _ptr(beta_v), _ptr(s), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+                   ctypes.c_size_t(workspace.numel()), _stream(stream, dev))
         name = "dr_chunk_fwd_osdn"
     if rc != DR_OK:
         raise DeltaRuleError(rc, name)
@@ -259,8 +305,9 @@ def dr_chunk_fwd_noalloc(q, k, v, beta_k, alpha=None, beta_v=None, S0=None, chun
         S_T = torch.empty((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=q.device)
     _check_tensors(q.dtype, [("q", q), ("k", k), ("v", v), ("o", o), ("alpha", alpha),
                              ("beta_k", beta_k), ("beta_v", beta_v), ("S0", S0), ("S_T", S_T)])
-    rc = lib().dr_chunk_fwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
-                                    _ptr(beta_v), _ptr(S0), _ptr(o), _ptr(S_T), _stream(stream))
+    dev = q.device
+    rc = _call("dr_chunk_fwd_noalloc", dev, ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+               _ptr(beta_k), _ptr(beta_v), _ptr(S0), _ptr(o), _ptr(S_T), _stream(stream, dev))
     if rc != DR_OK:
         raise DeltaRuleError(rc, "dr_chunk_fwd_noalloc")
     return o, S_T
@@ -279,7 +326,12 @@ def dr_decode_step_osdn(q, k, v, beta_k, S, s, alpha=None, beta_v=None, o=None, 
     return _decode_step(s, q, k, v, beta_k, S, alpha, beta_v, o, stream)
 
 
-def _decode_step(s, q, k, v, beta_k, S, alpha, beta_v, o, stream):
+def dr_diag_decode_step_variant(variant, q, k, v, beta_k, S, alpha=None, beta_v=None, s=None, o=None, stream=None):
+    """dr_decode_step (or its OSDN form when ``s`` is given) through a named kernel (``DECODE_VARIANTS``)."""
+    return _decode_step(s, q, k, v, beta_k, S, alpha, beta_v, o, stream, variant=DECODE_VARIANTS[variant])
+
+
+def _decode_step(s, q, k, v, beta_k, S, alpha, beta_v, o, stream, variant=None):
     if q.dim() == 4 and q.shape[1] != 1:
         raise ValueError("a decode step takes one token: q [B, 1, H, dk]")
     _check_shapes(q, v, [("k", k), ("v", v), ("o", o), ("alpha", alpha), ("beta_k", beta_k), ("beta_v", beta_v),
@@ -287,19 +339,24 @@ def _decode_step(s, q, k, v, beta_k, S, alpha, beta_v, o, stream):
     if S is None:
         raise ValueError("S (the state to update in place) is required")
     p = make_problem(q, v, alpha, beta_k, beta_v, 0)
+    dev = q.device
     if o is None:
         o = torch.empty(q.shape[:3] + (p.dv,), dtype=q.dtype, device=q.device)
     _check_tensors(q.dtype, [("q", q), ("k", k), ("v", v), ("o", o), ("alpha", alpha),
                              ("beta_k", beta_k), ("beta_v", beta_v), ("s", s), ("S", S)])
     if s is not None and tuple(s.shape) != tuple(q.shape):
         raise ValueError("s must have the shape of q / k: [B, 1, H, dk]")
-    if s is None:
-        rc = lib().dr_decode_step(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
-                                  _ptr(beta_v), _ptr(S), _ptr(o), _stream(stream))
+    if variant is not None:
+        rc = _call("dr_diag_decode_step_variant", dev, int(variant), ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+                   _ptr(alpha), _ptr(beta_k), _ptr(beta_v), _ptr(s), _ptr(S), _ptr(o), _stream(stream, dev))
+        name = "dr_diag_decode_step_variant"
+    elif s is None:
+        rc = _call("dr_decode_step", dev, ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                   _ptr(beta_k), _ptr(beta_v), _ptr(S), _ptr(o), _stream(stream, dev))
         name = "dr_decode_step"
     else:
-        rc = lib().dr_decode_step_osdn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
-                                       _ptr(beta_v), _ptr(s), _ptr(S), _ptr(o), _stream(stream))
+        rc = _call("dr_decode_step_osdn", dev, ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                   _ptr(beta_k), _ptr(beta_v), _ptr(s), _ptr(S), _ptr(o), _stream(stream, dev))
         name = "dr_decode_step_osdn"
     if rc != DR_OK:
         raise DeltaRuleError(rc, name)
@@ -317,7 +374,11 @@ def dr_state_map_apply(M, N, S=None, out=None, stream=None):
             raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor")
     if M.numel() != n * dk * dk or (S is not None and S.shape != N.shape) or out.shape != N.shape:
         raise ValueError("shapes: M [n, dk, dk], S / N / out [n, dk, dv]")
-    rc = lib().dr_state_map_apply(n, dk, dv, _ptr(M), _ptr(S), _ptr(N), _ptr(out), _stream(stream))
+    dev = N.device
+    for name, t in (("M", M), ("S", S), ("out", out)):
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, N on {dev}")
+    rc = _call("dr_state_map_apply", dev, n, dk, dv, _ptr(M), _ptr(S), _ptr(N), _ptr(out), _stream(stream, dev))
     if rc != DR_OK:
         raise DeltaRuleError(rc, "dr_state_map_apply")
     return out
@@ -343,17 +404,25 @@ def dr_backward(q, k, v, beta_k, dout, alpha=None, beta_v=None, s=None, S0=None,
     need = int(lib().dr_backward_workspace(ctypes.byref(p)))
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    rc = lib().dr_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k), _ptr(beta_v),
-                           _ptr(s), _ptr(S0), _ptr(dout), _ptr(dS_T), _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]),
-                           _ptr(g["alpha"]), _ptr(g["beta_k"]), _ptr(g["beta_v"]), _ptr(g["s"]), _ptr(g["S0"]),
-                           _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    rc = _call("dr_backward", dev, ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
+               _ptr(beta_v), _ptr(s), _ptr(S0), _ptr(dout), _ptr(dS_T), _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]),
+               _ptr(g["alpha"]), _ptr(g["beta_k"]), _ptr(g["beta_v"]), _ptr(g["s"]), _ptr(g["S0"]),
+               _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream, dev))
     if rc != DR_OK:
         raise DeltaRuleError(rc, "dr_backward")
     return g
 
 
 def dr_workspace_status(workspace, stream=None) -> int:
-    return int(lib().dr_workspace_status(_ptr(workspace), _stream(stream)))
+    dev = workspace.device
+    return int(_call("dr_workspace_status", dev, _ptr(workspace), _stream(stream, dev)))
+
+
+def dr_noalloc_status(device=None, stream=None) -> int:
+    """Status word of the last dr_chunk_fwd_noalloc call on ``device`` (default: the current device),
+    read after synchronising the stream: DR_OK, DR_ERR_RANGE or DR_ERR_TIMEOUT."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return int(_call("dr_noalloc_status", dev, _stream(stream, dev)))
 
 
 def dr_diag_umma_selftest(A, B, a_mn: bool, b_mn: bool, stream=None):
@@ -363,8 +432,9 @@ def dr_diag_umma_selftest(A, B, a_mn: bool, b_mn: bool, stream=None):
         raise TypeError("A and B must both be bf16 or both fp16")
     D = torch.empty((A.shape[0], N), dtype=torch.float32, device=A.device)
     ws = torch.zeros(256, dtype=torch.uint8, device=A.device)
-    rc = lib().dr_diag_umma_selftest(N, K, int(a_mn), int(b_mn), int(A.dtype == torch.bfloat16), _ptr(A), _ptr(B), _ptr(D), _ptr(ws),
-                                     _stream(stream))
+    dev = A.device
+    rc = _call("dr_diag_umma_selftest", dev, N, K, int(a_mn), int(b_mn), int(A.dtype == torch.bfloat16), _ptr(A),
+               _ptr(B), _ptr(D), _ptr(ws), _stream(stream, dev))
     if rc != DR_OK:
         raise DeltaRuleError(rc, "dr_diag_umma_selftest")
     return D, dr_workspace_status(ws, stream)
@@ -376,7 +446,7 @@ def dr_diag_tri_inverse(A, stream=None):
         raise ValueError("A must be a 64 x 64 fp32 CUDA tensor")
     A = A.contiguous()
     T = torch.zeros_like(A)
-    rc = lib().dr_diag_tri_inverse(_ptr(A), _ptr(T), _stream(stream))
+    rc = _call("dr_diag_tri_inverse", A.device, _ptr(A), _ptr(T), _stream(stream, A.device))
     if rc != DR_OK:
         raise DeltaRuleError(rc, "dr_diag_tri_inverse")
     return T
@@ -391,7 +461,8 @@ def dr_diag_wait_timeout(cluster_scope: bool, limit_ns: int, device=None, stream
     dev = torch.device("cuda") if device is None else torch.device(device)
     ws = torch.zeros(256, dtype=torch.uint8, device=dev)
     waited = torch.zeros(2, dtype=torch.int64, device=dev)
-    rc = lib().dr_diag_wait_timeout(int(bool(cluster_scope)), int(limit_ns), _ptr(ws), _ptr(waited), _stream(stream))
+    rc = _call("dr_diag_wait_timeout", ws.device, int(bool(cluster_scope)), int(limit_ns), _ptr(ws), _ptr(waited),
+               _stream(stream, ws.device))
     if rc != DR_OK:
         raise DeltaRuleError(rc, "dr_diag_wait_timeout")
     status = dr_workspace_status(ws, stream)

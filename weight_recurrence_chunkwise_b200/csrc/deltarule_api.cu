@@ -13,7 +13,6 @@
 #include "../../include/deltarule_diag.h"
 #include "chunk_simt.cuh"
 #include "chunk_tc.cuh"
-#include "chunk_tc2.cuh"
 #include "chunk_tc3.cuh"
 #include "common.cuh"
 #include "decode.cuh"
@@ -27,19 +26,11 @@ namespace {
 
 constexpr size_t kWorkspaceBytes = 256;  // status word, padded to an allocation granule
 
-// Tensor-core prefill kernel for dk = dv = 128, chunk 64: the two-CTA kernel with a three-slot
-// ring by default; DR_PREFILL_KERNEL=pair selects the two-slot two-CTA kernel and
-// DR_PREFILL_KERNEL=single the one-CTA-per-value-slice kernel (same results; for comparison).
-enum PrefillKernel { kRing, kPair, kSingle };
-PrefillKernel prefill_kernel() {
-  static const PrefillKernel k = [] {
-    const char *e = std::getenv("DR_PREFILL_KERNEL");
-    if (e && std::strcmp(e, "pair") == 0) return kPair;
-    if (e && std::strcmp(e, "single") == 0) return kSingle;
-    return kRing;
-  }();
-  return k;
-}
+// Prefill kernel variants (the library's choice is kDefault; the others are reachable only through
+// dr_diag_chunk_fwd_variant, for comparisons).
+enum PrefillVariant { kPrefillDefault = 0, kPrefillSingle = 1, kPrefillSimt = 2 };
+// Decode kernel variants, likewise (dr_diag_decode_step_variant).
+enum DecodeVariant { kDecodeDefault = 0, kDecodePerHead = 1, kDecodeSplit4 = 2, kDecodeStream = 3 };
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -181,52 +172,6 @@ dr_status tc_launch(const dr_problem *p, const void *q, const void *k, const voi
   return launch_status();
 }
 
-// Two-CTA cluster per (b, h): the value slices 0..63 and 64..127 share the chunk-local factors.
-dr_status tc_pair_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                         const float *beta_k, const float *beta_v, const float *S0, void *o, float *S_T,
-                         uint32_t *status, cudaStream_t st) {
-  using IO = __nv_bfloat16;
-  namespace tc = dr::tc;
-  namespace tc2 = dr::tc2;
-  alignas(64) CUtensorMap mq, mk, mv, mb;
-  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
-  if (!make_map(&mq, bf, 2, q, p->B, p->T, p->H, p->dk, tc::DK, tc::C) ||
-      !make_map(&mk, bf, 2, k, p->B, p->T, p->H, p->dk, 64, tc::C, sw) ||
-      !make_map(&mv, bf, 2, v, p->B, p->T, p->H, p->dv, tc::VS, tc::C, sw))
-    return DR_ERR_CUDA;
-  const bool bv = p->beta_v_mode == DR_CHANNEL;
-  const bool sym = p->beta_v_mode == DR_ABSENT && p->beta_k_mode == DR_CHANNEL;
-  if (bv || sym) {
-    if (!make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, bv ? static_cast<const void *>(beta_v) : beta_k, p->B,
-                  p->T, p->H, bv ? p->dv : p->dk, tc::VS, tc::C))
-      return DR_ERR_CUDA;
-  } else {
-    mb = mv;  // unused by the kernel in this mode
-  }
-  tc::Params prm{p->T, p->H, p->dv, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v, p->beta_v_mode,
-                 S0, o, S_T, status};
-  auto kern = tc2::chunk_fwd_pair_kernel<IO>;
-  constexpr size_t smem = tc2::SMEM_BYTES;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-      cudaSuccess)
-    return DR_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2, p->H, p->B);
-  cfg.blockDim = dim3(tc2::NT, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mb, prm) != cudaSuccess) return DR_ERR_CUDA;
-  return launch_status();
-}
-
 dr_status tc_ring_launch(const dr_problem *p, const int *cu, const void *q, const void *k, const void *v,
                          const float *alpha, const float *beta_k, const float *beta_v, const float *s_scale,
                          const float *S0, void *o, float *S_T, uint32_t *status, cudaStream_t st) {
@@ -269,17 +214,6 @@ dr_status tc_ring_launch(const dr_problem *p, const int *cu, const void *q, cons
 }
 
 // ----------------------------------------------------------------- decode
-// DR_DECODE_KERNEL=classic keeps dk = dv = 128 on one CTA per head (for comparisons); the default
-// splits each head over four CTAs when there are no more heads than SMs, and streams the states
-// through a persistent kernel when there are more.
-bool decode_stream_enabled() {
-  static const bool on = [] {
-    const char *e = std::getenv("DR_DECODE_KERNEL");
-    return !(e && std::strcmp(e, "classic") == 0);
-  }();
-  return on;
-}
-
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -290,18 +224,23 @@ int sm_count() {
 template <typename IO, int DK, int DV>
 dr_status decode_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
                         const float *beta_k, const float *beta_v, const float *s_scale, float *S, void *o,
-                        cudaStream_t st) {
+                        int variant, cudaStream_t st) {
   const long long heads = static_cast<long long>(p->B) * p->H;
   if (heads > 0x7fffffffLL) return DR_ERR_INVALID_ARG;
+  // dk = dv = 128: four CTAs per head (32 value columns each) when there are no more heads than SMs,
+  // else the persistent streaming kernel; other head sizes, one CTA per head
   if constexpr (DK == 128 && DV == 128) {
     const int sms = sm_count();
-    if (decode_stream_enabled() && sms > 0 && heads <= sms) {  // small batch: 4 CTAs per head
+    if (variant == kDecodeDefault) variant = sms <= 0 ? kDecodePerHead : (heads <= sms ? kDecodeSplit4 : kDecodeStream);
+    if (variant == kDecodeSplit4) {
+      if (heads * 4 > 0x7fffffffLL) return DR_ERR_UNSUPPORTED;
       dr::decode_step_kernel<IO, DK, DV, 4><<<static_cast<unsigned>(heads * 4), 256, 0, st>>>(
           static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v), alpha, p->alpha_mode,
           beta_k, p->beta_k_mode, beta_v, p->beta_v_mode, s_scale, S, static_cast<IO *>(o));
       return launch_status();
     }
-    if (decode_stream_enabled() && sms > 0 && heads > sms) {
+    if (variant == kDecodeStream) {
+      if (sms <= 0) return DR_ERR_CUDA;
       auto kern = dr::decode_stream_kernel<IO>;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(dr::kDecodeStreamSmem)) != cudaSuccess)
@@ -312,6 +251,8 @@ dr_status decode_launch(const dr_problem *p, const void *q, const void *k, const
           beta_k, p->beta_k_mode, beta_v, p->beta_v_mode, s_scale, S, static_cast<IO *>(o), heads);
       return launch_status();
     }
+  } else {
+    if (variant == kDecodeSplit4 || variant == kDecodeStream) return DR_ERR_UNSUPPORTED;
   }
   dr::decode_step_kernel<IO, DK, DV><<<static_cast<unsigned>(heads), 256, 0, st>>>(
       static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v), alpha, p->alpha_mode,
@@ -322,14 +263,14 @@ dr_status decode_launch(const dr_problem *p, const void *q, const void *k, const
 template <typename IO>
 dr_status decode_dispatch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
                           const float *beta_k, const float *beta_v, const float *s_scale, float *S, void *o,
-                          cudaStream_t st) {
+                          int variant, cudaStream_t st) {
   if (p->dk == 128 && p->dv == 128)
-    return decode_launch<IO, 128, 128>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
+    return decode_launch<IO, 128, 128>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, variant, st);
   if (p->dk == 128 && p->dv == 64)
-    return decode_launch<IO, 128, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
+    return decode_launch<IO, 128, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, variant, st);
   if (p->dk == 64 && p->dv == 128)
-    return decode_launch<IO, 64, 128>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
-  return decode_launch<IO, 64, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
+    return decode_launch<IO, 64, 128>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, variant, st);
+  return decode_launch<IO, 64, 64>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, variant, st);
 }
 
 // Prefill with an optional write-side key scale (NULL: a = b) and optional packed-sequence offsets
@@ -337,7 +278,7 @@ dr_status decode_dispatch(const dr_problem *p, const void *q, const void *k, con
 dr_status chunk_fwd_impl(const dr_problem *p, const int *cu, const void *q, const void *k, const void *v,
                          const float *alpha, const float *beta_k, const float *beta_v, const float *s_scale,
                          const float *S0, void *o, float *S_T, void *workspace, size_t workspace_bytes,
-                         void *stream) {
+                         void *stream, int variant = kPrefillDefault) {
   dr_status s = check_common(p, false);
   if (s != DR_OK) return s;
   s = check_pointers(p, q, k, v, alpha, beta_k, beta_v, o);
@@ -348,6 +289,12 @@ dr_status chunk_fwd_impl(const dr_problem *p, const int *cu, const void *q, cons
   if (!aligned16(workspace)) return DR_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t *status = static_cast<uint32_t *>(workspace);
+  // a variant that cannot take the problem is refused before anything is enqueued
+  const bool tc_shape = p->io_dtype == DR_BF16 && p->dk == dr::tc::DK && p->chunk == dr::tc::C;
+  const bool ring_shape = tc_shape && p->dv == 2 * dr::tc::VS;
+  const bool plain = !s_scale && !cu;  // the one-CTA-per-slice kernel takes neither extension
+  if (variant == kPrefillSingle && !(plain && tc_shape && p->dv % dr::tc::VS == 0)) return DR_ERR_UNSUPPORTED;
+  if (variant != kPrefillDefault && variant != kPrefillSingle && variant != kPrefillSimt) return DR_ERR_UNSUPPORTED;
   if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DR_ERR_CUDA;
   const size_t state_bytes = sizeof(float) * size_t(p->B) * p->H * p->dk * p->dv;
   if (p->T == 0) {  // nothing to scan: the final state is the initial state
@@ -359,29 +306,29 @@ dr_status chunk_fwd_impl(const dr_problem *p, const int *cu, const void *q, cons
   }
   if (p->io_dtype == DR_F32)
     return simt_dispatch<float>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
-  const bool ring_shape = p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv == 2 * dr::tc::VS;
-  const bool plain = !s_scale && !cu;  // the older kernels take neither extension
-  if (ring_shape && (!plain || prefill_kernel() == kRing))
+  if (variant == kPrefillSimt)
+    return simt_dispatch<__nv_bfloat16>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
+  if (variant == kPrefillDefault && ring_shape)
     return tc_ring_launch(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
-  if (plain && ring_shape && prefill_kernel() == kPair)
-    return tc_pair_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
-  if (plain && p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv % dr::tc::VS == 0)
+  if (plain && tc_shape && p->dv % dr::tc::VS == 0)
     return tc_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
   return simt_dispatch<__nv_bfloat16>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
 }
 
 dr_status decode_step_impl(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
                            const float *beta_k, const float *beta_v, const float *s_scale, float *S, void *o,
-                           void *stream) {
+                           void *stream, int variant = kDecodeDefault) {
   dr_status s = check_common(p, true);
   if (s != DR_OK) return s;
   s = check_pointers(p, q, k, v, alpha, beta_k, beta_v, o);
   if (s != DR_OK) return s;
   if (!S) return DR_ERR_INVALID_ARG;
   if (!aligned16(S) || (s_scale && !aligned16(s_scale))) return DR_ERR_ALIGNMENT;
+  if (variant < kDecodeDefault || variant > kDecodeStream) return DR_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (p->io_dtype == DR_F32) return decode_dispatch<float>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
-  return decode_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, st);
+  if (p->io_dtype == DR_F32)
+    return decode_dispatch<float>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, variant, st);
+  return decode_dispatch<__nv_bfloat16>(p, q, k, v, alpha, beta_k, beta_v, s_scale, S, o, variant, st);
 }
 
 constexpr int kBwdSpan = 16;  // tokens between the backward pass's state checkpoints
@@ -560,6 +507,14 @@ dr_status dr_chunk_fwd_noalloc(const dr_problem *p, const void *q, const void *k
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return DR_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return DR_ERR_UNSUPPORTED;
+  if (q) {  // the array used is the current device's: the data must live there too
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, q) != cudaSuccess) {
+      cudaGetLastError();
+      return DR_ERR_INVALID_ARG;
+    }
+    if (a.type == cudaMemoryTypeDevice && a.device != dev) return DR_ERR_INVALID_ARG;
+  }
   void *scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_static_mu);
@@ -574,6 +529,19 @@ dr_status dr_chunk_fwd_noalloc(const dr_problem *p, const void *q, const void *k
   return dr_chunk_fwd(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, scratch, kStaticScratchBytes, stream);
 }
 
+dr_status dr_noalloc_status(void *stream) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DR_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DR_ERR_UNSUPPORTED;
+  void *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    scratch = g_static_addr[dev];
+  }
+  if (!scratch) return DR_ERR_INVALID_ARG;  // no no-alloc call on this device yet
+  return dr_workspace_status(scratch, stream);
+}
+
 dr_status dr_workspace_status(const void *workspace, void *stream) {
   if (!workspace) return DR_ERR_WORKSPACE;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DR_ERR_CUDA;
@@ -582,6 +550,19 @@ dr_status dr_workspace_status(const void *workspace, void *stream) {
   if (w & dr::STATUS_TIMEOUT) return DR_ERR_TIMEOUT;
   if (w & dr::STATUS_RANGE) return DR_ERR_RANGE;
   return DR_OK;
+}
+
+int dr_diag_chunk_fwd_variant(int variant, const dr_problem *p, const void *q, const void *k, const void *v,
+                              const float *alpha, const float *beta_k, const float *beta_v, const float *S0, void *o,
+                              float *S_T, void *workspace, size_t workspace_bytes, void *stream) {
+  return chunk_fwd_impl(p, nullptr, q, k, v, alpha, beta_k, beta_v, nullptr, S0, o, S_T, workspace, workspace_bytes,
+                        stream, variant);
+}
+
+int dr_diag_decode_step_variant(int variant, const dr_problem *p, const void *q, const void *k, const void *v,
+                                const float *alpha, const float *beta_k, const float *beta_v, const float *s,
+                                float *S, void *o, void *stream) {
+  return decode_step_impl(p, q, k, v, alpha, beta_k, beta_v, s, S, o, stream, variant);
 }
 
 int dr_diag_umma_selftest(int N, int K, int a_mn, int b_mn, int bf16, const void *A, const void *B, float *D,
