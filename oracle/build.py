@@ -12,13 +12,13 @@ SRC = os.path.join(HERE, "dr_oracle.c")
 LIB = os.path.join(HERE, "libdr_oracle.so")
 
 
-def build(force: bool = False, out: str = LIB, extra_flags=()) -> str:
-    """Build ``libdr_oracle.so`` next to its source; return its path."""
-    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(SRC):
+def build(force: bool = False, out: str = LIB, extra_flags=(), src: str = SRC) -> str:
+    """Build ``libdr_oracle.so`` next to its source (or ``src`` into ``out``); return its path."""
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
         return out
     # -ffp-contract=off: every product and sum rounds as written (no fused multiply-add).
     cmd = ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
-           *extra_flags, SRC, "-o", out + ".tmp", "-lm"]
+           *extra_flags, src, "-o", out + ".tmp", "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(out + ".tmp", out)
     return out

@@ -57,13 +57,6 @@
 #include <omp.h>
 #endif
 
-/* DRO_MUTANT selects a deliberately wrong variant, compiled only by the
- * mutation test (tests/test_oracle_mutants.py) to show that the pins reject
- * it.  The default build is DRO_MUTANT == 0: the recurrence as written. */
-#ifndef DRO_MUTANT
-#define DRO_MUTANT 0
-#endif
-
 #define DRO_ABSENT 0
 #define DRO_SCALAR 1
 #define DRO_CHANNEL 2
@@ -103,17 +96,14 @@ static int check_args(const dro_args *a) {
 static void token_vectors(const dro_args *a, size_t th, double *bv, double *av, double *wv) {
   const int dk = a->dk, dv = a->dv;
   for (int i = 0; i < dk; ++i) {
-    double bk = sqrt(gate(a->beta_k, a->beta_k_mode, th, dk, i)) * a->k[th * dk + i];
-    if (DRO_MUTANT == 1) bk = gate(a->beta_k, a->beta_k_mode, th, dk, i) * a->k[th * dk + i];
+    const double bk = sqrt(gate(a->beta_k, a->beta_k_mode, th, dk, i)) * a->k[th * dk + i];
     bv[i] = bk;
     av[i] = a->s_scale ? a->s_scale[th * dk + i] * bk : bk;
-    if (DRO_MUTANT == 2 && a->s_scale) { bv[i] = av[i]; av[i] = bk; }
   }
   for (int j = 0; j < dv; ++j) {
-    double vj = a->v[th * dv + j];
+    const double vj = a->v[th * dv + j];
     if (a->beta_v_mode != DRO_ABSENT)
-      wv[j] = (DRO_MUTANT == 3 ? sqrt(gate(a->beta_v, a->beta_v_mode, th, dv, j))
-                               : gate(a->beta_v, a->beta_v_mode, th, dv, j)) * vj;
+      wv[j] = gate(a->beta_v, a->beta_v_mode, th, dv, j) * vj;
     else
       wv[j] = sqrt(gate(a->beta_k, a->beta_k_mode, th, dk, j)) * vj;
   }
@@ -136,49 +126,25 @@ static void sequential_head(const dro_args *a, int b, int h) {
   for (int t = 0; t < T; ++t) {
     const size_t th = ((size_t)b * T + t) * H + h;
     token_vectors(a, th, bv, av, wv);
-    if (DRO_MUTANT == 4) { /* wrong: output read before the update */
-      for (int j = 0; j < dv; ++j) {
-        double acc = 0.0;
-        for (int i = 0; i < dk; ++i) acc += S[i * dv + j] * a->q[th * dk + i];
-        a->o[th * dv + j] = acc;
-      }
-    }
     /* decay first: S <- Diag(alpha_t) S */
-    if (DRO_MUTANT != 5) {
-      for (int i = 0; i < dk; ++i) {
-        double al = gate(a->alpha, a->alpha_mode, th, dk, i);
-        for (int j = 0; j < dv; ++j) S[i * dv + j] *= al;
-      }
+    for (int i = 0; i < dk; ++i) {
+      const double al = gate(a->alpha, a->alpha_mode, th, dk, i);
+      for (int j = 0; j < dv; ++j) S[i * dv + j] *= al;
     }
     /* read with the erase key and form the error: u = w - (D S)^T b */
     for (int j = 0; j < dv; ++j) {
       double r = 0.0;
-      for (int i = 0; i < dk; ++i)
-        r += (DRO_MUTANT == 6 && dk == dv ? S[j * dv + i] : S[i * dv + j]) * bv[i];
-      u[j] = (DRO_MUTANT == 7) ? wv[j] + r : wv[j] - r;
+      for (int i = 0; i < dk; ++i) r += S[i * dv + j] * bv[i];
+      u[j] = wv[j] - r;
     }
     /* rank-1 write: S <- D S + a u^T  ==  (I - a b^T) D S + a w^T */
     for (int i = 0; i < dk; ++i)
       for (int j = 0; j < dv; ++j) S[i * dv + j] += av[i] * u[j];
-    if (DRO_MUTANT == 5) { /* wrong: decay applied after the erase and write */
-      for (int i = 0; i < dk; ++i) {
-        double al = gate(a->alpha, a->alpha_mode, th, dk, i);
-        for (int j = 0; j < dv; ++j) S[i * dv + j] *= al;
-      }
-    }
-    if (DRO_MUTANT == 8 && dk == dv) { /* wrong: channel decay on the value dimension */
-      for (int i = 0; i < dk; ++i)
-        for (int j = 0; j < dv; ++j)
-          S[i * dv + j] *= gate(a->alpha, a->alpha_mode, th, dk, j) / gate(a->alpha, a->alpha_mode, th, dk, i);
-    }
     /* output from the updated state: o_t = S_t^T q_t */
-    if (DRO_MUTANT != 4) {
-      for (int j = 0; j < dv; ++j) {
-        double acc = 0.0;
-        for (int i = 0; i < dk; ++i)
-          acc += (DRO_MUTANT == 9 && dk == dv ? S[j * dv + i] : S[i * dv + j]) * a->q[th * dk + i];
-        a->o[th * dv + j] = acc;
-      }
+    for (int j = 0; j < dv; ++j) {
+      double acc = 0.0;
+      for (int i = 0; i < dk; ++i) acc += S[i * dv + j] * a->q[th * dk + i];
+      a->o[th * dv + j] = acc;
     }
   }
   if (a->ST) memcpy(a->ST + sh, S, sizeof(double) * dk * dv);
