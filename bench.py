@@ -336,6 +336,47 @@ def run_backward(args, dr, p, x, dev, st, peaks, peaks_src):
     return 0
 
 
+def run_seqpar_cost(args, dr, p, dev, st):
+    """Profiling aid: per-rank device time of a sequence split over n ranks (the map pass -- two
+    prefills of the segment --, the composition of the earlier maps, and the rerun of the segment)
+    against the unsplit prefill, each measured alone on this GPU.  The all-gather of the maps is not
+    included (8 MiB per rank for 64 heads)."""
+    from weight_recurrence_chunkwise_b200 import seqpar
+
+    x = to_dev(make_inputs(p), dev)
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = mk(), mk()
+        e0.record(st)
+        for _ in range(args.steps):
+            fn()
+        e1.record(st)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    run = lambda g: dr.dr_chunk_fwd(g["q"], g["k"], g["v"], g["beta_k"], alpha=g["alpha"], beta_v=g["beta_v"],
+                                    S0=g["S0"], chunk=p.chunk, stream=st)
+    out = {"seqpar_cost": True, "workload": p.name, "T": p.T, "unsplit_ms": timed(lambda: run(x)), "ranks": {}}
+    for n in (2, 4, 8):
+        L = p.T // n
+        seg = {k: (None if t is None else (t[:, :L].contiguous() if k != "S0" else t)) for k, t in x.items()}
+        maps = [seqpar.segment_map(seg["q"], seg["k"], seg["v"], seg["beta_k"], alpha=seg["alpha"],
+                                   beta_v=seg["beta_v"], chunk=p.chunk)] * (n - 1)
+        t_map = timed(lambda: seqpar.segment_map(seg["q"], seg["k"], seg["v"], seg["beta_k"], alpha=seg["alpha"],
+                                                 beta_v=seg["beta_v"], chunk=p.chunk))
+        t_compose = timed(lambda: seqpar.compose(maps, seg["S0"]))
+        t_rerun = timed(lambda: run(seg))
+        rank_ms = t_map + t_compose + t_rerun
+        out["ranks"][n] = {"segment_T": L, "map_ms": t_map, "compose_ms": t_compose, "rerun_ms": t_rerun,
+                           "rank_ms": rank_ms, "speedup_vs_unsplit": out["unsplit_ms"] / rank_ms}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- our arm
 def prefill_roofline(p, ms, peaks, peaks_src, with_S0=False):
     """Roofline of one prefill launch: HBM-bound on algorithmic counts (SURVEY-style work model)."""
@@ -407,6 +448,9 @@ def main():
                     help="with --only-prefill / --backward: the workload to time (default: the headline one)")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (dr_backward) on the --config workload instead")
+    ap.add_argument("--seqpar-cost", action="store_true",
+                    help="time one rank's work of a sequence-parallel prefill of the --config workload split "
+                         "over 2, 4 and 8 ranks (on this one GPU) beside the unsplit prefill")
     args = ap.parse_args()
     ws, rank, local = dist_env()
     if args.impl == "reference":
@@ -429,6 +473,8 @@ def main():
     if args.backward:
         p = rank_problem(rank, args.config)
         return run_backward(args, dr, p, to_dev(make_inputs(p), dev), dev, st, peaks, peaks_src)
+    if args.seqpar_cost:
+        return run_seqpar_cost(args, dr, rank_problem(rank, args.config), dev, st)
     if args.only_prefill:
         line = time_prefill_workload(dr, rank_problem(rank, args.config), dev, st, args.steps, args.warmup, ws,
                                      peaks, peaks_src)

@@ -50,6 +50,19 @@ def compose(maps, S0=None, apply=_cuda_apply):
     return S
 
 
+def _all_gather(x, group):
+    """Every rank's copy of `x`, in rank order.  Over NCCL the device tensors are exchanged directly;
+    a gloo group (CPU ranks, or ranks sharing one GPU in tests) exchanges through host copies."""
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    staged = x.is_cuda and dist.get_backend(group) == "gloo"
+    src = x.detach().cpu() if staged else x.contiguous()
+    out = [torch.empty_like(src) for _ in range(world)]
+    dist.all_gather(out, src, group=group)
+    return [t.to(x.device) for t in out] if staged else out
+
+
 def seqpar_chunk_fwd(q, k, v, beta_k, alpha=None, beta_v=None, s=None, S0=None, chunk=64, group=None,
                      prefill=_cuda_prefill, apply=_cuda_apply):
     """Prefill of this rank's segment of a sequence split along T over the ranks of `group`.
@@ -62,11 +75,7 @@ def seqpar_chunk_fwd(q, k, v, beta_k, alpha=None, beta_v=None, s=None, S0=None, 
 
     rank, world = dist.get_rank(group), dist.get_world_size(group)
     M, N = segment_map(q, k, v, beta_k, alpha=alpha, beta_v=beta_v, s=s, chunk=chunk, prefill=prefill)
-    Ms = [torch.empty_like(M) for _ in range(world)]
-    Ns = [torch.empty_like(N) for _ in range(world)]
-    dist.all_gather(Ms, M.contiguous(), group=group)
-    dist.all_gather(Ns, N.contiguous(), group=group)
-    maps = list(zip(Ms, Ns))
+    maps = list(zip(_all_gather(M, group), _all_gather(N, group)))
     S_in = compose(maps[:rank], S0, apply)
     o, S_seg = prefill(q, k, v, beta_k, alpha=alpha, beta_v=beta_v, s=s, S0=S_in, chunk=chunk)
     # this segment's own final state is exact; the later segments' maps carry it to the end
