@@ -75,13 +75,17 @@ DR_API int dr_diag_umma_selftest(int N, int K, int a_mn, int b_mn, int bf16, con
 
 /*
  * T = (I + A)^-1 for the strictly lower-triangular part of a 64 x 64 matrix A
- * (the UT transform of one chunk), computed by the warp-MMA routine of the
- * prefill kernel (fp16 operands, fp32 accumulation).  A: row-major fp32 device
- * buffer (its diagonal and upper part are ignored); T: row-major fp32 device
- * buffer that the caller zeroes first (only the lower blocks are written).
- * Returns a dr_status code.
+ * (the UT transform of one chunk), computed by one of the prefill kernels'
+ * warp-MMA routines (fp16 operands, fp32 accumulation):
+ *   variant 0  the ring prefill's (operands in its swizzled tile layout,
+ *              result kept in registers)
+ *   variant 1  the one-CTA prefill's (padded row-major arrays)
+ * A: row-major fp32 device buffer (its diagonal and upper part are ignored);
+ * T: row-major fp32 device buffer that the caller zeroes first (only the lower
+ * blocks are written).  Returns a dr_status code (DR_ERR_INVALID_ARG for an
+ * unknown variant).
  */
-DR_API int dr_diag_tri_inverse(const float *A, float *T, void *stream);
+DR_API int dr_diag_tri_inverse(int variant, const float *A, float *T, void *stream);
 
 /*
  * The bounded waits of the prefill kernels, run out on purpose: every CTA waits

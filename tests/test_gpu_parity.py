@@ -102,18 +102,21 @@ def _unit_lower_case(seed, scale):
     return torch.tril(scale * torch.randn(64, 64, generator=g, dtype=torch.float64), -1)
 
 
+@pytest.mark.parametrize("variant", [0, 1])
 @pytest.mark.parametrize("seed,scale", [(0, 0.05), (1, 0.15), (2, 0.3)])
-def test_tri_inverse_building_block(dr, seed, scale):
-    """The warp-MMA UT-transform inverse against a float64 matrix inverse."""
+def test_tri_inverse_building_block(dr, seed, scale, variant):
+    """The warp-MMA UT-transform inverse (the ring prefill's, and the one-CTA prefill's) against a
+    float64 matrix inverse."""
     A = _unit_lower_case(seed, scale)
     ref = torch.linalg.inv(torch.eye(64, dtype=torch.float64) + A)
-    T = dr.dr_diag_tri_inverse(A.float().cuda()).double().cpu()
+    T = dr.dr_diag_tri_inverse(A.float().cuda(), variant=variant).double().cpu()
     assert torch.equal(torch.triu(T, 1), torch.zeros_like(T))          # lower triangular
     assert torch.allclose(torch.diagonal(T), torch.ones(64, dtype=torch.float64), atol=1e-6)
     assert float((T - ref).abs().max() / ref.abs().max()) <= 5e-3
 
 
-def test_tri_inverse_on_key_gram_matrix(dr):
+@pytest.mark.parametrize("variant", [0, 1])
+def test_tri_inverse_on_key_gram_matrix(dr, variant):
     """A shaped like a real chunk: A_ij = sqrt(b_i b_j) k_i . k_j (unit keys, strengths in (0,1))."""
     g = torch.Generator().manual_seed(7)
     k = torch.nn.functional.normalize(torch.randn(64, 128, generator=g, dtype=torch.float64), dim=-1)
@@ -121,7 +124,7 @@ def test_tri_inverse_on_key_gram_matrix(dr):
     kb = k * beta.sqrt()[:, None]
     A = torch.tril(kb @ kb.T, -1)
     ref = torch.linalg.inv(torch.eye(64, dtype=torch.float64) + A)
-    T = dr.dr_diag_tri_inverse(A.float().cuda()).double().cpu()
+    T = dr.dr_diag_tri_inverse(A.float().cuda(), variant=variant).double().cpu()
     assert float((T - ref).abs().max() / ref.abs().max()) <= 5e-3
 
 

@@ -87,7 +87,7 @@ def lib():
         L.dr_version.restype = ctypes.c_int
         L.dr_diag_umma_selftest.argtypes = [ctypes.c_int] * 5 + [vp, vp, vp, vp, vp]
         L.dr_diag_umma_selftest.restype = ctypes.c_int
-        L.dr_diag_tri_inverse.argtypes = [vp, vp, vp]
+        L.dr_diag_tri_inverse.argtypes = [ctypes.c_int, vp, vp, vp]
         L.dr_diag_tri_inverse.restype = ctypes.c_int
         L.dr_diag_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_ulonglong, vp, vp, vp]
         L.dr_diag_wait_timeout.restype = ctypes.c_int
@@ -440,13 +440,14 @@ def dr_diag_umma_selftest(A, B, a_mn: bool, b_mn: bool, stream=None):
     return D, dr_workspace_status(ws, stream)
 
 
-def dr_diag_tri_inverse(A, stream=None):
-    """(I + strictly-lower(A))^-1 for a 64 x 64 fp32 CUDA tensor, via the prefill's warp-MMA routine."""
+def dr_diag_tri_inverse(A, stream=None, variant=0):
+    """(I + strictly-lower(A))^-1 for a 64 x 64 fp32 CUDA tensor, via a prefill kernel's warp-MMA routine
+    (variant 0: the ring prefill's, 1: the one-CTA prefill's)."""
     if A.shape != (64, 64) or A.dtype != torch.float32 or not A.is_cuda:
         raise ValueError("A must be a 64 x 64 fp32 CUDA tensor")
     A = A.contiguous()
     T = torch.zeros_like(A)
-    rc = _call("dr_diag_tri_inverse", A.device, _ptr(A), _ptr(T), _stream(stream, A.device))
+    rc = _call("dr_diag_tri_inverse", A.device, int(variant), _ptr(A), _ptr(T), _stream(stream, A.device))
     if rc != DR_OK:
         raise DeltaRuleError(rc, "dr_diag_tri_inverse")
     return T

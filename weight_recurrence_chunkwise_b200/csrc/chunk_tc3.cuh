@@ -8,7 +8,7 @@
 //                 T = (I + strictly-lower(Bh Ac^T))^-1, W = T Bh
 //   state pass:   U0 = T Wr, U = U0 - W S, O = Qh S + P U, S <- Diag(gamma_C)(S + Ac^T U)
 //
-// Work split (as in chunk_tc2.cuh): CTA r of the pair runs the state pass for value columns
+// Work split: CTA r of the pair runs the state pass for value columns
 // 64r..64r+63 over every chunk (chain role, warps 8..15), and builds the chunk-local factors of
 // the chunks c with c % 2 == r (local role, warps 0..7), which it writes into slot c % 3 of both
 // CTAs (its own by plain stores, the peer's by DSMEM bulk copies).
@@ -48,7 +48,7 @@ using tc::Params;
 constexpr int NT = 512;  // threads
 constexpr int NL = 256;  // local role: threads 0..255
 constexpr int BAR_LOCAL = 1, BAR_CHAIN = 2, BAR_INV = 3;  // BAR_INV: warps 0..3 in the UT inverse
-constexpr int RGL = 16;  // rows per local elementwise thread in the channel-gate K1
+constexpr int RGL = 8;   // channel-gate K1: rows per local thread (8 row groups x 32 groups of 4 channels)
 constexpr int NSLOT = 3;
 
 // slot layout (bytes from the slot base); every tile 1024-aligned
@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(NT, 1)
 chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_qk, bar_lmma, bar_cmma, bar_v;
+  __shared__ uint64_t bar_qk, bar_lmma, bar_cmma, bar_out, bar_v;
   __shared__ uint64_t bar_full[NSLOT], bar_free[NSLOT], bar_land[NSLOT];
   __shared__ uint32_t tmem_base_sh;
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -136,6 +136,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     mbar_init(&bar_qk, 1);
     mbar_init(&bar_lmma, 1);
     mbar_init(&bar_cmma, 1);
+    mbar_init(&bar_out, 1);
     mbar_init(&bar_v, 1);
     for (int j = 0; j < NSLOT; ++j) {
       mbar_init(&bar_full[j], 1);
@@ -167,13 +168,13 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // the TMA loads, L2 prefetches and DSMEM copies and tracks the free[] phases.
     constexpr int kIo = 128;
     uint32_t ph_free = 0;  // bit j: parity of the next wait on free[j] (ltid kIo only)
-    const int kp = ltid & 63, rgl = ltid >> 6, c0 = 2 * kp;
+    const int rgl = ltid >> 5, c0 = 4 * (ltid & 31);  // channel-gate K1: rows 8 rgl.., channels c0..c0+3
     const int quarter = warp & 3, half = warp >> 2;  // warps 0..7
     constexpr bool gates_scalar = !kChanGates;
     float *sGate = reinterpret_cast<float *>(sm + OFF_GS);  // [0..63] alpha, [64..127] beta_k
-    float pal[2 * RGL], pbe[2 * RGL];                        // channel-gate K1: this thread's gates
+    float pal[4 * RGL], pbe[4 * RGL];                        // channel-gate K1: this thread's gates
 #pragma unroll
-    for (int i = 0; i < 2 * RGL; ++i) pal[i] = pbe[i] = 1.f;
+    for (int i = 0; i < 4 * RGL; ++i) pal[i] = pbe[i] = 1.f;
 
     auto issue_qk = [&](int c) {  // raw q and k of chunk c, in place into slot c % 3
       const int t0 = c * C;
@@ -217,21 +218,25 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const int t0 = c * C, L = min(C, T - t0);
       const size_t thb = (tok0 + t0) * H + h;
 #pragma unroll
-      for (int j = 0; j < RGL; ++j) {
+      for (int j = 0; j < RGL; ++j) {  // 16-byte loads: four channels of a row per request
         const size_t th = thb + static_cast<size_t>(min(rgl * RGL + j, L - 1)) * H;
         if (p.alpha_mode == MODE_CHANNEL) {
-          const float2 a = __ldg(reinterpret_cast<const float2 *>(p.alpha + th * DK + c0));
-          pal[2 * j] = a.x;
-          pal[2 * j + 1] = a.y;
+          const float4 a = __ldg(reinterpret_cast<const float4 *>(p.alpha + th * DK + c0));
+          pal[4 * j] = a.x;
+          pal[4 * j + 1] = a.y;
+          pal[4 * j + 2] = a.z;
+          pal[4 * j + 3] = a.w;
         } else if (p.alpha_mode == MODE_SCALAR) {
-          pal[2 * j] = __ldg(p.alpha + th);
+          pal[4 * j] = __ldg(p.alpha + th);
         }
         if (p.beta_k_mode == MODE_CHANNEL) {
-          const float2 bt = __ldg(reinterpret_cast<const float2 *>(p.beta_k + th * DK + c0));
-          pbe[2 * j] = bt.x;
-          pbe[2 * j + 1] = bt.y;
+          const float4 bt = __ldg(reinterpret_cast<const float4 *>(p.beta_k + th * DK + c0));
+          pbe[4 * j] = bt.x;
+          pbe[4 * j + 1] = bt.y;
+          pbe[4 * j + 2] = bt.z;
+          pbe[4 * j + 3] = bt.w;
         } else {
-          pbe[2 * j] = __ldg(p.beta_k + th);
+          pbe[4 * j] = __ldg(p.beta_k + th);
         }
       }
     };
@@ -364,89 +369,108 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         if (!(amax < kF16Max)) raise_status(p.status, STATUS_RANGE);
       } else {
-        float *sPX = reinterpret_cast<float *>(tTP);  // row-group gate products, 4 x 128 fp32
+        float *sPX = reinterpret_cast<float *>(tTP);  // row-group gate products, 8 x 128 fp32
 #pragma unroll
         for (int jj = 0; jj < RGL; ++jj) {
           const bool valid = rgl * RGL + jj < L;
-          if (p.alpha_mode != MODE_CHANNEL) pal[2 * jj + 1] = pal[2 * jj];
-          if (p.alpha_mode == MODE_ABSENT || !valid) pal[2 * jj] = pal[2 * jj + 1] = 1.f;
-          if (p.beta_k_mode != MODE_CHANNEL) pbe[2 * jj + 1] = pbe[2 * jj];
-          if (!valid) pbe[2 * jj] = pbe[2 * jj + 1] = 0.f;
-        }
-        float p0 = 1.f, p1 = 1.f;  // gate product of my row group
 #pragma unroll
-        for (int jj = 0; jj < RGL; ++jj) {
-          p0 *= pal[2 * jj];
-          p1 *= pal[2 * jj + 1];
-        }
-        *reinterpret_cast<float2 *>(sPX + rgl * 128 + c0) = make_float2(p0, p1);
-        bar_sync(BAR_LOCAL, NL);
-        float h0 = 1.f, h1 = 1.f, t0a = 1.f, t1a = 1.f;  // products of the groups before / after mine
+          for (int e = 1; e < 4; ++e) {
+            if (p.alpha_mode != MODE_CHANNEL) pal[4 * jj + e] = pal[4 * jj];
+            if (p.beta_k_mode != MODE_CHANNEL) pbe[4 * jj + e] = pbe[4 * jj];
+          }
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float2 x = *reinterpret_cast<const float2 *>(sPX + g * 128 + c0);
-          if (g < rgl) {
-            h0 *= x.x;
-            h1 *= x.y;
-          } else if (g > rgl) {
-            t0a *= x.x;
-            t1a *= x.y;
+          for (int e = 0; e < 4; ++e) {
+            if (p.alpha_mode == MODE_ABSENT || !valid) pal[4 * jj + e] = 1.f;
+            if (!valid) pbe[4 * jj + e] = 0.f;
           }
         }
-        if (rgl == 0) {
-          const float g0 = h0 * p0 * t0a, g1 = h1 * p1 * t1a;
-          *reinterpret_cast<float2 *>(sGC + c0) = make_float2(g0, g1);
-          if (!(fminf(g0, g1) >= kMinChunkDecayF16)) raise_status(p.status, STATUS_RANGE);
+        float pg[4] = {1.f, 1.f, 1.f, 1.f};  // gate product of my row group
+#pragma unroll
+        for (int jj = 0; jj < RGL; ++jj)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pg[e] *= pal[4 * jj + e];
+        *reinterpret_cast<float4 *>(sPX + rgl * 128 + c0) = make_float4(pg[0], pg[1], pg[2], pg[3]);
+        bar_sync(BAR_LOCAL, NL);
+        float gr[4] = {1.f, 1.f, 1.f, 1.f};  // gamma_r of the current row: starts at the groups before mine
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          if (g < rgl) {
+            const float4 x = *reinterpret_cast<const float4 *>(sPX + g * 128 + c0);
+            gr[0] *= x.x;
+            gr[1] *= x.y;
+            gr[2] *= x.z;
+            gr[3] *= x.w;
+          }
+        }
+        if (rgl == 7) {  // the last group: gamma_C = (groups before) x (my group)
+          const float4 gC = make_float4(gr[0] * pg[0], gr[1] * pg[1], gr[2] * pg[2], gr[3] * pg[3]);
+          *reinterpret_cast<float4 *>(sGC + c0) = gC;
+          if (!(fminf(fminf(gC.x, gC.y), fminf(gC.z, gC.w)) >= kMinChunkDecayF16)) raise_status(p.status, STATUS_RANGE);
         }
         const bool beta_scalar = p.beta_k_mode == MODE_SCALAR;
-        const uint32_t blk = static_cast<uint32_t>(kp >> 5), ch = static_cast<uint32_t>((kp & 31) >> 2);
-        const uint32_t inb = static_cast<uint32_t>((kp & 3) * 4);
+        // element (row, c0..c0+3): 8 bytes inside one 16-byte group of the swizzled row; rows of my
+        // group are 8 rgl + jj, so the swizzle of row jj is (group ^ jj)
+        const uint32_t blk = static_cast<uint32_t>(c0 >> 6), grp = static_cast<uint32_t>((c0 & 63) >> 3);
+        const uint32_t inb = static_cast<uint32_t>((c0 & 7) * 2);
         uint8_t *pQ = X + blk * SX_CB + (64 + rgl * RGL) * 128 + inb;
         uint8_t *pB = X + blk * SX_CB + (rgl * RGL) * 128 + inb;
         uint8_t *pA = tAC + blk * 64 * 128 + (rgl * RGL) * 128 + inb;
         float amax = 0.f;
-        float ga = h0, gb = h1;  // gamma_r of the current row, two key channels
         // rows in batches of RB: a batch's raw k and q are read before any of its results are
-        // written back in place, so their shared-memory loads overlap instead of each waiting
-        // behind the previous row's stores
+        // written back in place, so their shared-memory loads overlap
         constexpr int RB = kScaled ? 1 : 4;  // the scaled variant has no registers to spare
 #pragma unroll
         for (int j0 = 0; j0 < RGL; j0 += RB) {
-        __nv_bfloat162 kraw[RB], qraw[RB];
+          uint2 kraw[RB], qraw[RB];
 #pragma unroll
-        for (int jb = 0; jb < RB; ++jb) {
-          const int jj = j0 + jb;
-          const uint32_t sw = ((ch ^ static_cast<uint32_t>(jj & 7)) << 4) + jj * 128;
-          kraw[jb] = *reinterpret_cast<const __nv_bfloat162 *>(pB + sw);  // raw k
-          qraw[jb] = *reinterpret_cast<const __nv_bfloat162 *>(pQ + sw);  // raw q
-        }
+          for (int jb = 0; jb < RB; ++jb) {
+            const int jj = j0 + jb;
+            const uint32_t sw = ((grp ^ static_cast<uint32_t>(jj & 7)) << 4) + jj * 128;
+            kraw[jb] = *reinterpret_cast<const uint2 *>(pB + sw);  // raw k
+            qraw[jb] = *reinterpret_cast<const uint2 *>(pQ + sw);  // raw q
+          }
 #pragma unroll
-        for (int jb = 0; jb < RB; ++jb) {
-          const int jj = j0 + jb;
-          const uint32_t sw = ((ch ^ static_cast<uint32_t>(jj & 7)) << 4) + jj * 128;
-          const float2 kf = __bfloat1622float2(kraw[jb]), qf = __bfloat1622float2(qraw[jb]);
-          float s0, s1;
-          if (beta_scalar) {
-            s0 = s1 = tc::sqrt_fast(pbe[2 * jj]);
-          } else {
-            s0 = tc::sqrt_fast(pbe[2 * jj]);
-            s1 = tc::sqrt_fast(pbe[2 * jj + 1]);
+          for (int jb = 0; jb < RB; ++jb) {
+            const int jj = j0 + jb;
+            const uint32_t sw = ((grp ^ static_cast<uint32_t>(jj & 7)) << 4) + jj * 128;
+            const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kraw[jb]);
+            const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qraw[jb]);
+            float kf[4], qf[4];
+            {
+              const float2 k01 = __bfloat1622float2(k2[0]), k23 = __bfloat1622float2(k2[1]);
+              const float2 q01 = __bfloat1622float2(q2[0]), q23 = __bfloat1622float2(q2[1]);
+              kf[0] = k01.x; kf[1] = k01.y; kf[2] = k23.x; kf[3] = k23.y;
+              qf[0] = q01.x; qf[1] = q01.y; qf[2] = q23.x; qf[3] = q23.y;
+            }
+            float sc[4] = {1.f, 1.f, 1.f, 1.f};
+            if constexpr (kScaled) {
+              const size_t th = (tok0 + t0 + min(rgl * RGL + jj, L - 1)) * H + h;
+              const float4 x = __ldg(reinterpret_cast<const float4 *>(p.s + th * DK + c0));
+              sc[0] = x.x; sc[1] = x.y; sc[2] = x.z; sc[3] = x.w;
+            }
+            float sb[4];
+            if (beta_scalar) {
+              sb[0] = sb[1] = sb[2] = sb[3] = tc::sqrt_fast(pbe[4 * jj]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) sb[e] = tc::sqrt_fast(pbe[4 * jj + e]);
+            }
+            float oq[4], ob[4], oa[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              gr[e] *= pal[4 * jj + e];
+              const float bv = sb[e] * kf[e];
+              float av = bv * __fdividef(1.f, gr[e]);  // a / gamma_r
+              if constexpr (kScaled) av *= sc[e];
+              amax = fmaxf(amax, fabsf(av));
+              oq[e] = gr[e] * qf[e];
+              ob[e] = gr[e] * bv;
+              oa[e] = av;
+            }
+            *reinterpret_cast<uint2 *>(pQ + sw) = make_uint2(pack_f16x2(oq[0], oq[1]), pack_f16x2(oq[2], oq[3]));
+            *reinterpret_cast<uint2 *>(pB + sw) = make_uint2(pack_f16x2(ob[0], ob[1]), pack_f16x2(ob[2], ob[3]));
+            *reinterpret_cast<uint2 *>(pA + sw) = make_uint2(pack_f16x2(oa[0], oa[1]), pack_f16x2(oa[2], oa[3]));
           }
-          ga *= pal[2 * jj];
-          gb *= pal[2 * jj + 1];
-          const float b0 = s0 * kf.x, b1 = s1 * kf.y;
-          float a0 = b0 * __fdividef(1.f, ga), a1 = b1 * __fdividef(1.f, gb);  // a / gamma_r
-          if constexpr (kScaled) {
-            const size_t th = (tok0 + t0 + min(rgl * RGL + jj, L - 1)) * H + h;
-            const float2 sc = __ldg(reinterpret_cast<const float2 *>(p.s + th * DK + c0));
-            a0 *= sc.x;
-            a1 *= sc.y;
-          }
-          amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
-          *reinterpret_cast<uint32_t *>(pQ + sw) = pack_f16x2(ga * qf.x, gb * qf.y);  // Qh (in place of q)
-          *reinterpret_cast<uint32_t *>(pB + sw) = pack_f16x2(ga * b0, gb * b1);      // Bh (in place of k)
-          *reinterpret_cast<uint32_t *>(pA + sw) = pack_f16x2(a0, a1);                // Ac
-        }
         }
         if (!(amax < kF16Max)) raise_status(p.status, STATUS_RANGE);
       }
@@ -604,7 +628,8 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const int cw = warp - 8;
     const int quarter = cw & 3, half = cw >> 2;
     const int trow = quarter * 32 + lane;
-    uint32_t ph_v = 0, ph_mma = 0;
+    uint32_t ph_v = 0, ph_mma = 0, ph_out = 0;
+    int u0_ready = -1;  // elected issuing thread: the chunk whose U0 is already issued
     uint32_t ph_full = 0, ph_land = 0;  // bit j: parity of the next wait on full[j] / land[j]
     bool aborted = false;
     const size_t sbase = (static_cast<size_t>(b) * H + h) * DK * DV;
@@ -637,6 +662,20 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
       } else {
         pws = __ldg((p.beta_v_mode == MODE_SCALAR ? p.beta_v : p.beta_k) + th);
+      }
+    };
+    // separate write strengths beta_v of chunk c into L2, ahead of prefetch_ws: this CTA's value
+    // columns of each row (two 128-byte lines per row), or one value per row if scalar.  (Symmetric
+    // writes read beta_k, whose rows the local roles already bring into L2.)
+    auto prefetch_ws_l2 = [&](int c) {
+      if (p.beta_v_mode == MODE_ABSENT) return;
+      const int t0 = c * C, L = min(C, T - t0);
+      const bool chan = p.beta_v_mode == MODE_CHANNEL;
+      if (ct < (chan ? 2 * C : C)) {
+        const int row = min(chan ? (ct >> 1) : ct, L - 1);
+        const size_t th = (tok0 + t0 + row) * H + h;
+        const float *a = chan ? p.beta_v + th * DV + v0 + (ct & 1) * 32 : p.beta_v + th;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
       }
     };
     // write vectors of the chunk whose raw v sits in Wr, in place (after bar_v)
@@ -720,6 +759,14 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     }
     const uint64_t dS = sdesc_sw128(sbase_addr + OFF_S, 128 * 128, 1024);
     const uint64_t dWr = sdesc_sw128(sbase_addr + OFF_WR, 64 * 128, 1024);
+    // U0 = [T; P] Wr of the chunk in the slot at `slot_addr` (elected issuing thread only)
+    auto issue_u0 = [&](uint32_t slot_addr) {
+      const uint64_t dTP = sdesc_sw128(slot_addr + STP, 16, 1024);
+      const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk)
+        umma_f16(tmem + COL_U0, kstep(dTP, 128, kk), mstep(dWr, kk), id3, kk > 0);
+    };
 
     // Software pipeline: the write vectors of chunk c+1 are built while the second MMA group of
     // chunk c runs (their v is requested as soon as the first MMA group of chunk c has read Wr, and
@@ -730,6 +777,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         issue_v(0);
         for (int c = 1; c < 3 && c < nchunks; ++c) tma_prefetch_l2_4d(&tm_v, v0, h, tt0 + c * C, tb);
       }
+      for (int c = 1; c < 3 && c < nchunks; ++c) prefetch_ws_l2(c);
       prefetch_ws(0);
       const bool ok_v = mbar_wait(&bar_v, ph_v & 1u, kWaitLimitNs);
       ph_v ^= 1u;
@@ -765,15 +813,14 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         gc = reinterpret_cast<const float *>(sm + gc_off(j))[trow];
 
         // ------------------------------------------------------------ U0 = [T;P] Wr,  D3 = [-W; Qh] S
+        // (U0 does not depend on S: it is usually issued at the end of the previous iteration, as
+        // soon as this chunk's slot and write vectors were ready, which leaves D3 alone here)
         if (cw == 0) {
           if (elect_one()) {
             tc_fence_after();
-            const uint64_t dTP = sdesc_sw128(xaddr + STP, 16, 1024);
             const uint64_t dX = sdesc_sw128(xaddr + SX, 16, 1024);
             const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
-#pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-              umma_f16(tmem + COL_U0, kstep(dTP, 128, kk), mstep(dWr, kk), id3, kk > 0);
+            if (u0_ready != c) issue_u0(xaddr);
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
               umma_f16(tmem + cD3, kstep(dX, 128, kk), mstep(dS, kk), id3, kk > 0);
@@ -806,6 +853,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (c + 1 < nchunks) issue_v(c + 1);  // Wr is free
         if (c + 3 < nchunks) tma_prefetch_l2_4d(&tm_v, v0, h, tt0 + (c + 3) * C, tb);
       }
+      if (c + 3 < nchunks) prefetch_ws_l2(c + 3);
       if (c + 1 < nchunks) prefetch_ws(c + 1);
 
       // -------------------------------------------------------------- E3: U = U0 - W S -> X rows 0..63
@@ -842,9 +890,10 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           const uint32_t id3 = idesc_f16_f32(128, VS, false, true);
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + COL_D4, mstep(dAcM, kk), mstep(dU, kk), id4, kk > 0);
+          umma_commit(&bar_cmma);  // the state update waits for Ac^T U alone
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + cD3, kstep(dTP, 128, kk), mstep(dU, kk), id3, 1u);
-          umma_commit(&bar_cmma);
+          umma_commit(&bar_out);   // the outputs and the slot's release wait for this
         }
         __syncwarp();
       }
@@ -868,32 +917,64 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           break;
         }
       }
-      // this CTA is done with slot j: tell the CTA that produces chunk c+3 into it
-      if (ct == 128) {
+      // U0 of the next chunk, if its slot is already full (its write vectors were just built)
+      if (cw == 0 && c + 1 < nchunks) {
+        if (elect_one()) {
+          const int j1 = (c + 1) % NSLOT;
+          if (mbar_test_cluster(&bar_full[j1], (ph_full >> j1) & 1u)) {
+            tc_fence_after();
+            issue_u0(sbase_addr + slot_off(j1));
+            u0_ready = c + 1;
+          }
+        }
+        __syncwarp();
+      }
+
+      // this CTA is done with slot j once the outputs' MMAs are too: tell the CTA that produces
+      // chunk c+3 into it -- now if they are done already, else after E4
+      auto release_slot = [&] {
         if (((c + 3) & 1) == rank) mbar_arrive(&bar_free[j]);
         else mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&bar_free[j]), static_cast<uint32_t>(peer)));
+      };
+      bool released = false;
+      if (ct == 128 && mbar_test_cluster(&bar_out, ph_out & 1u)) {
+        release_slot();
+        released = true;
       }
 
       // -------------------------------------------------------------- E4: S <- Diag(gamma_C) (S + Ac^T U)
       {
         float mx = 0.f;
+        float ds[32];
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D4 + half * 32), *reinterpret_cast<float(*)[16]>(ds));
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D4 + half * 32 + 16), *reinterpret_cast<float(*)[16]>(ds + 16));
+        tmem_ld_wait();
 #pragma unroll
-        for (int jj = 0; jj < 32; jj += 16) {
-          float ds[16];
-          tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D4 + half * 32 + jj), ds);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            Sreg[jj + i] = gc * (Sreg[jj + i] + ds[i]);
-            mx = fmaxf(mx, fabsf(Sreg[jj + i]));
-          }
-          tc::st_h16x16(tS, trow, half * 32 + jj, 128, Sreg + jj);
+        for (int i = 0; i < 32; ++i) {
+          Sreg[i] = gc * (Sreg[i] + ds[i]);
+          mx = fmaxf(mx, fabsf(Sreg[i]));
         }
+        tc::st_h16x16(tS, trow, half * 32, 128, Sreg);
+        tc::st_h16x16(tS, trow, half * 32 + 16, 128, Sreg + 16);
         if (!(mx < kF16Max)) raise_status(p.status, STATUS_RANGE);
       }
       fence_async_smem();
       tc_fence_before();
-      bar_sync(BAR_CHAIN, NT - NL);
+      {
+        bool ok = true;
+        if (ct == 128 && !released) {
+          ok = mbar_wait(&bar_out, ph_out & 1u, kWaitLimitNs);
+          if (ok) release_slot();
+        }
+        ph_out ^= 1u;
+        const bool fail = bar_or(BAR_CHAIN, NT - NL, !ok);
+        tc_fence_after();
+        if (fail) {
+          if (ct == 128) raise_status(p.status, STATUS_TIMEOUT);
+          aborted = true;
+          break;
+        }
+      }
     }
     if (!aborted && p.S_T) {
       float *dst = p.S_T + sbase + static_cast<size_t>(trow) * DV + v0 + half * 32;

@@ -617,9 +617,12 @@ int dr_diag_wait_timeout(int cluster_scope, unsigned long long limit_ns, void *w
   return launch_status();
 }
 
-int dr_diag_tri_inverse(const float *A, float *T, void *stream) {
-  if (!A || !T) return DR_ERR_INVALID_ARG;
-  dr::tri_selftest_kernel<<<1, 128, 0, static_cast<cudaStream_t>(stream)>>>(A, T);
+int dr_diag_tri_inverse(int variant, const float *A, float *T, void *stream) {
+  if (!A || !T || variant < 0 || variant > 1) return DR_ERR_INVALID_ARG;
+  if (cudaFuncSetAttribute(dr::tri_selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(dr::kTriSelftestSmem)) != cudaSuccess)
+    return DR_ERR_CUDA;
+  dr::tri_selftest_kernel<<<1, 128, dr::kTriSelftestSmem, static_cast<cudaStream_t>(stream)>>>(variant, A, T);
   return launch_status();
 }
 

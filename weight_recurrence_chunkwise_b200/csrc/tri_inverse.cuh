@@ -6,8 +6,8 @@
 // one warp on register fragments, which suits these tiny dependent products
 // far better than a round trip through tensor memory.
 //
-//  * Diagonal blocks (warps 0..3, one block each): for N = A_bb strictly lower
-//    (N^16 = 0),  (I + N)^-1 = (I - N)(I + N^2)(I + N^4)(I + N^8).
+//  * Diagonal blocks (one warp each): for N = A_bb strictly lower (N^16 = 0),
+//    (I + N)^-1 = (I - N)(I + N^2)(I + N^4)(I + N^8).
 //  * Off-diagonal blocks, by distance d = i - j = 1, 2, 3 (warp i computes
 //    block (i, j)):  T_ij = -T_ii * sum_{m=j}^{i-1} A_im T_mj.
 //

@@ -81,17 +81,18 @@ umma_selftest_kernel(const uint16_t *__restrict__ A, const uint16_t *__restrict_
 // T = (I + A)^-1 for the strictly lower part of a 64 x 64 fp32 matrix A (row-major),
 // through the same warp-MMA routine the prefill kernel uses.  T (row-major fp32)
 // must be zeroed by the caller: only its lower blocks are written.  128 threads.
-__global__ void __launch_bounds__(128) tri_selftest_kernel(const float *__restrict__ A, float *__restrict__ Tout) {
-  __shared__ __align__(16) __half Ah[64 * tri::LD], AhT[64 * tri::LD], ThT[64 * tri::LD];
+// T = (I + A)^-1 of a 64 x 64 A by one of the prefill kernels' routines, for tests.
+//   variant 0: the ring prefill's (inverse64_rows on the swizzled 128-byte-row tile layout);
+//   variant 1: the one-CTA prefill's (inverse64 on padded row-major arrays).
+// 128 threads; dynamic shared memory kTriSelftestSmem.
+constexpr size_t kTriSelftestSmem =
+    1024 + (3 * 64 * tri::LD * 2 > 128 * 128 ? 3 * 64 * tri::LD * 2 : 128 * 128);  // the larger variant
+__global__ void __launch_bounds__(128) tri_selftest_kernel(int variant, const float *__restrict__ A,
+                                                           float *__restrict__ Tout) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < 64 * 64; e += blockDim.x) {
-    const int r = e / 64, c = e % 64;
-    const __half a = __float2half_rn(c < r ? A[e] : 0.f);
-    Ah[r * tri::LD + c] = a;
-    AhT[c * tri::LD + r] = a;
-  }
-  __syncthreads();
-  tri::inverse64(Ah, AhT, ThT, warp, lane, [&](int bi, int bj, const tri::Frag &F, int ln) {
+  auto put = [&](int bi, int bj, const tri::Frag &F, int ln) {
     const int row = 16 * bi + (ln >> 2), col = 16 * bj + 2 * (ln & 3);
     Tout[row * 64 + col] = F.v[0];
     Tout[row * 64 + col + 1] = F.v[1];
@@ -101,7 +102,30 @@ __global__ void __launch_bounds__(128) tri_selftest_kernel(const float *__restri
     Tout[row * 64 + col + 9] = F.v[5];
     Tout[(row + 8) * 64 + col + 8] = F.v[6];
     Tout[(row + 8) * 64 + col + 9] = F.v[7];
-  }, [] { __syncthreads(); });
+  };
+  if (variant == 1) {
+    __half *Ah = reinterpret_cast<__half *>(sm), *AhT = Ah + 64 * tri::LD, *ThT = AhT + 64 * tri::LD;
+    for (int e = tid; e < 64 * 64; e += blockDim.x) {
+      const int r = e / 64, c = e % 64;
+      const __half a = __float2half_rn(c < r ? A[e] : 0.f);
+      Ah[r * tri::LD + c] = a;
+      AhT[c * tri::LD + r] = a;
+    }
+    __syncthreads();
+    tri::inverse64(Ah, AhT, ThT, warp, lane, put, [] { __syncthreads(); });
+    return;
+  }
+  uint8_t *TP = sm;  // rows 0..63: A; rows 64..127: T^T scratch (one 128-row tile of 128-byte rows)
+  for (int e = tid; e < 64 * 64; e += blockDim.x) {
+    const int r = e / 64, c = e % 64;
+    *reinterpret_cast<__half *>(TP + tri::Sw128Layout::off(r, c)) = __float2half_rn(c < r ? A[e] : 0.f);
+  }
+  __syncthreads();
+  tri::Frag Trow[4];
+  tri::inverse64_rows<tri::Sw128Layout>(TP, TP + 64 * 128, warp, lane, Trow, [] { __syncthreads(); });
+#pragma unroll
+  for (int d = 0; d < 4; ++d)
+    if (d <= warp) put(warp, warp - d, Trow[d], lane);
 }
 
 }  // namespace dr
