@@ -308,71 +308,37 @@ def backward_bytes(p):
 
 
 def run_backward(args, dr, p, x, dev, st, peaks, peaks_src):
-    """Profiling aid: the backward pass alone on one workload (warm-up, then timed launches)."""
+    """Profiling aid: the backward pass alone on one workload (warm-up, then timed launches), through
+    the library's choice of kernel and, for comparison, the token-sequential kernel."""
     g = torch.Generator().manual_seed(p.seed)
     dout = torch.randn(x["v"].shape, generator=g).to(x["v"].dtype).to(dev)
     S0 = torch.zeros((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=dev)
     dST = torch.randn((p.B, p.H, p.dk, p.dv), generator=g).to(dev)
-    run = lambda: dr.dr_backward(x["q"], x["k"], x["v"], x["beta_k"], dout, alpha=x["alpha"], beta_v=x["beta_v"],
-                                 S0=S0, dS_T=dST, stream=st)
-    for _ in range(args.warmup):
-        run()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(st)
-    for _ in range(args.steps):
-        run()
-    e1.record(st)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
-    byts = backward_bytes(p)
-    gbs = byts / (ms / 1e3) / 1e9
-    print(json.dumps({"backward": True, "workload": p.name, "ms": ms,
-                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                   "frac": gbs / peaks["hbm_gbs"], "peak_source": peaks_src,
-                                   "traffic": measured_traffic("delta_rule_bwd_kernel", p.name),
-                                   "kernel": "delta_rule_bwd_kernel", "algorithmic_bytes_per_launch": byts}}),
-          flush=True)
-    return 0
-
-
-def run_seqpar_cost(args, dr, p, dev, st):
-    """Profiling aid: per-rank device time of a sequence split over n ranks (the map pass -- two
-    prefills of the segment --, the composition of the earlier maps, and the rerun of the segment)
-    against the unsplit prefill, each measured alone on this GPU.  The all-gather of the maps is not
-    included (8 MiB per rank for 64 heads)."""
-    from weight_recurrence_chunkwise_b200 import seqpar
-
-    x = to_dev(make_inputs(p), dev)
-    mk = lambda: torch.cuda.Event(enable_timing=True)
-
-    def timed(fn):
+    chunk_path = p.io == "bf16" and p.dk == 128 and p.dv == 128
+    out = {"backward": True, "workload": p.name}
+    for variant in (["default", "sequential"] if chunk_path else ["default"]):
+        run = lambda: dr.dr_diag_backward_variant(variant, x["q"], x["k"], x["v"], x["beta_k"], dout,
+                                                  alpha=x["alpha"], beta_v=x["beta_v"], S0=S0, dS_T=dST, stream=st)
         for _ in range(args.warmup):
-            fn()
+            run()
         torch.cuda.synchronize()
-        e0, e1 = mk(), mk()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(st)
         for _ in range(args.steps):
-            fn()
+            run()
         e1.record(st)
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / args.steps
-
-    run = lambda g: dr.dr_chunk_fwd(g["q"], g["k"], g["v"], g["beta_k"], alpha=g["alpha"], beta_v=g["beta_v"],
-                                    S0=g["S0"], chunk=p.chunk, stream=st)
-    out = {"seqpar_cost": True, "workload": p.name, "T": p.T, "unsplit_ms": timed(lambda: run(x)), "ranks": {}}
-    for n in (2, 4, 8):
-        L = p.T // n
-        seg = {k: (None if t is None else (t[:, :L].contiguous() if k != "S0" else t)) for k, t in x.items()}
-        maps = [seqpar.segment_map(seg["q"], seg["k"], seg["v"], seg["beta_k"], alpha=seg["alpha"],
-                                   beta_v=seg["beta_v"], chunk=p.chunk)] * (n - 1)
-        t_map = timed(lambda: seqpar.segment_map(seg["q"], seg["k"], seg["v"], seg["beta_k"], alpha=seg["alpha"],
-                                                 beta_v=seg["beta_v"], chunk=p.chunk))
-        t_compose = timed(lambda: seqpar.compose(maps, seg["S0"]))
-        t_rerun = timed(lambda: run(seg))
-        rank_ms = t_map + t_compose + t_rerun
-        out["ranks"][n] = {"segment_T": L, "map_ms": t_map, "compose_ms": t_compose, "rerun_ms": t_rerun,
-                           "rank_ms": rank_ms, "speedup_vs_unsplit": out["unsplit_ms"] / rank_ms}
+        ms = e0.elapsed_time(e1) / args.steps
+        byts = backward_bytes(p)
+        gbs = byts / (ms / 1e3) / 1e9
+        chunked = variant == "default" and chunk_path
+        kern = "chunk_fwd_ring_kernel (states) + chunk_bwd_kernel" if chunked else "delta_rule_bwd_kernel"
+        out["sequential" if variant == "sequential" else "ms_kernel"] = kern
+        out[variant] = {"ms": ms, "kernel": kern,
+                        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": gbs / peaks["hbm_gbs"], "peak_source": peaks_src,
+                                     "traffic": None if chunked else measured_traffic("delta_rule_bwd_kernel", p.name),
+                                     "algorithmic_bytes_per_launch": byts}}
     print(json.dumps(out), flush=True)
     return 0
 

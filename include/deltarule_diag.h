@@ -61,6 +61,28 @@ DR_API int dr_diag_decode_step_variant(int variant, const dr_problem *p, const v
                                        void *stream);
 
 /*
+ * dr_backward through a named kernel instead of the library's choice:
+ *   variant 0  the library's choice (what dr_backward runs)
+ *   variant 1  the token-sequential kernel (fp32 arithmetic throughout; every
+ *              supported shape; the library's choice for fp32 I/O and for
+ *              head sizes other than dk = dv = 128)
+ *   variant 2  the chunkwise kernel on the tensor cores (bf16 I/O, dk = dv =
+ *              128): a forward pass that keeps the state at the start of every
+ *              chunk, then the chunks from the last to the first
+ * Arguments, layouts and errors are those of dr_backward; the workspace must
+ * hold dr_diag_backward_workspace(variant, p) bytes.  An unsupported variant
+ * returns DR_ERR_UNSUPPORTED before anything is enqueued.
+ */
+DR_API size_t dr_diag_backward_workspace(int variant, const dr_problem *p);
+DR_API int dr_diag_backward_variant(int variant, const dr_problem *p, const void *q, const void *k,
+                                    const void *v, const float *alpha, const float *beta_k,
+                                    const float *beta_v, const float *s, const float *S0,
+                                    const void *dout, const float *dS_T, float *dq, float *dk,
+                                    float *dv, float *dalpha, float *dbeta_k, float *dbeta_v,
+                                    float *ds, float *dS0, void *workspace, size_t workspace_bytes,
+                                    void *stream);
+
+/*
  * D[128 x N] = A[128 x K] * B[K x N] on one CTA through tcgen05.mma (16-bit
  * inputs: bf16 if bf16 != 0, else fp16; fp32 accumulate), with A staged
  * K-major (a_mn = 0) or MN-major (a_mn = 1)

@@ -14,12 +14,13 @@ from ._binding import (DR_ABSENT, DR_BF16, DR_CHANNEL, DR_ERR_ALIGNMENT, DR_ERR_
                        dr_chunk_fwd, dr_chunk_fwd_noalloc, dr_chunk_fwd_osdn, dr_chunk_fwd_varlen, dr_decode_step,
                        dr_decode_step_osdn, dr_diag_tri_inverse, dr_diag_wait_timeout, dr_state_map_apply, dr_backward,
                        dr_diag_umma_selftest, dr_diag_chunk_fwd_variant, dr_diag_decode_step_variant,
-                       dr_problem, PREFILL_VARIANTS, DECODE_VARIANTS,
+                       dr_diag_backward_variant, dr_problem, PREFILL_VARIANTS, DECODE_VARIANTS, BACKWARD_VARIANTS,
                        dr_noalloc_status, dr_workspace_status, lib, make_problem, status_string, workspace_bytes)
 
 __all__ = [
     "dr_chunk_fwd", "dr_chunk_fwd_noalloc", "dr_chunk_fwd_osdn", "dr_chunk_fwd_varlen", "dr_decode_step", "dr_decode_step_osdn", "dr_state_map_apply", "dr_backward", "dr_workspace_status", "dr_noalloc_status", "dr_diag_umma_selftest", "dr_diag_tri_inverse", "dr_diag_wait_timeout", "dr_diag_chunk_fwd_variant",
-    "dr_diag_decode_step_variant", "PREFILL_VARIANTS", "DECODE_VARIANTS", "dr_problem",
+    "dr_diag_decode_step_variant", "dr_diag_backward_variant", "PREFILL_VARIANTS", "DECODE_VARIANTS",
+    "BACKWARD_VARIANTS", "dr_problem",
     "DeltaRuleError", "lib", "make_problem", "status_string", "workspace_bytes", "EXPORTS", "LIB_PATH",
     "DR_OK", "DR_ERR_INVALID_ARG", "DR_ERR_UNSUPPORTED", "DR_ERR_ALIGNMENT", "DR_ERR_WORKSPACE",
     "DR_ERR_RANGE", "DR_ERR_TIMEOUT", "DR_ERR_CUDA", "DR_F32", "DR_BF16", "DR_ABSENT", "DR_SCALAR",

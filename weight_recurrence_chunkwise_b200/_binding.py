@@ -42,11 +42,13 @@ EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_chunk_fwd_osdn", "dr_ch
            "dr_chunk_fwd_noalloc", "dr_decode_step",
            "dr_decode_step_osdn", "dr_state_map_apply", "dr_backward_workspace", "dr_backward",
            "dr_workspace_status", "dr_noalloc_status", "dr_status_string", "dr_version", "dr_diag_umma_selftest",
-           "dr_diag_tri_inverse", "dr_diag_wait_timeout", "dr_diag_chunk_fwd_variant", "dr_diag_decode_step_variant")
+           "dr_diag_tri_inverse", "dr_diag_wait_timeout", "dr_diag_chunk_fwd_variant", "dr_diag_decode_step_variant",
+           "dr_diag_backward_workspace", "dr_diag_backward_variant")
 
 # kernels of dr_diag_chunk_fwd_variant / dr_diag_decode_step_variant (include/deltarule_diag.h)
 PREFILL_VARIANTS = {"default": 0, "single": 1, "simt": 2}
 DECODE_VARIANTS = {"default": 0, "per_head": 1, "split4": 2, "stream": 3}
+BACKWARD_VARIANTS = {"default": 0, "sequential": 1, "chunk": 2}
 
 
 def lib():
@@ -95,6 +97,10 @@ def lib():
         L.dr_diag_chunk_fwd_variant.restype = ctypes.c_int
         L.dr_diag_decode_step_variant.argtypes = [ctypes.c_int, P] + [vp] * 9 + [vp]
         L.dr_diag_decode_step_variant.restype = ctypes.c_int
+        L.dr_diag_backward_workspace.argtypes = [ctypes.c_int, P]
+        L.dr_diag_backward_workspace.restype = sz
+        L.dr_diag_backward_variant.argtypes = [ctypes.c_int, P] + [vp] * 18 + [vp, sz, vp]
+        L.dr_diag_backward_variant.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -390,6 +396,17 @@ def dr_backward(q, k, v, beta_k, dout, alpha=None, beta_v=None, s=None, S0=None,
 
     Returns a dict with keys q, k, v, beta_k, alpha, beta_v, s, S0 (None where absent / not wanted).
     """
+    return _backward(None, q, k, v, beta_k, dout, alpha, beta_v, s, S0, dS_T, want_dS0, workspace, stream)
+
+
+def dr_diag_backward_variant(variant, q, k, v, beta_k, dout, alpha=None, beta_v=None, s=None, S0=None, dS_T=None,
+                             want_dS0=True, workspace=None, stream=None):
+    """dr_backward through a named kernel (``BACKWARD_VARIANTS``) instead of the library's choice."""
+    return _backward(BACKWARD_VARIANTS[variant], q, k, v, beta_k, dout, alpha, beta_v, s, S0, dS_T, want_dS0,
+                     workspace, stream)
+
+
+def _backward(variant, q, k, v, beta_k, dout, alpha, beta_v, s, S0, dS_T, want_dS0, workspace, stream):
     _check_shapes(q, v, [("k", k), ("v", v), ("dout", dout), ("alpha", alpha), ("beta_k", beta_k),
                          ("beta_v", beta_v), ("s", s), ("S0", S0), ("dS_T", dS_T)])
     p = make_problem(q, v, alpha, beta_k, beta_v, 64)
@@ -401,15 +418,24 @@ def dr_backward(q, k, v, beta_k, dout, alpha=None, beta_v=None, s=None, S0=None,
                              ("beta_v", beta_v), ("s", s), ("S0", S0), ("S_T", dS_T)])
     if s is not None and tuple(s.shape) != tuple(q.shape):
         raise ValueError("s must have the shape of q / k")
-    need = int(lib().dr_backward_workspace(ctypes.byref(p)))
+    if variant is None:
+        need = int(lib().dr_backward_workspace(ctypes.byref(p)))
+    else:
+        need = int(lib().dr_diag_backward_workspace(int(variant), ctypes.byref(p)))
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    rc = _call("dr_backward", dev, ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
-               _ptr(beta_v), _ptr(s), _ptr(S0), _ptr(dout), _ptr(dS_T), _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]),
-               _ptr(g["alpha"]), _ptr(g["beta_k"]), _ptr(g["beta_v"]), _ptr(g["s"]), _ptr(g["S0"]),
-               _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream, dev))
+    args = [ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k), _ptr(beta_v), _ptr(s), _ptr(S0),
+            _ptr(dout), _ptr(dS_T), _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]), _ptr(g["alpha"]), _ptr(g["beta_k"]),
+            _ptr(g["beta_v"]), _ptr(g["s"]), _ptr(g["S0"]), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+            _stream(stream, dev)]
+    if variant is None:
+        rc = _call("dr_backward", dev, *args)
+        name = "dr_backward"
+    else:
+        rc = _call("dr_diag_backward_variant", dev, int(variant), *args)
+        name = "dr_diag_backward_variant"
     if rc != DR_OK:
-        raise DeltaRuleError(rc, "dr_backward")
+        raise DeltaRuleError(rc, name)
     return g
 
 

@@ -1,0 +1,910 @@
+// backward_chunk.cuh -- the backward pass in the chunkwise (WY/UT) form on the tensor cores
+// (tcgen05.mma, fp16 operands in 128-byte-swizzled shared memory, fp32 accumulators in TMEM), for
+// bf16 I/O, dk = dv = 128 and chunks of 64 tokens.
+//
+// Algebra (DeltaNet page, step 7; FG2-GDN page, section 2), per chunk with initial state S (stored
+// by the forward ring kernel) and dS = the gradient of the chunk's final state, rows r of the chunk,
+// gamma_r = prod_{j<=r} alpha_j per key channel, b = sqrt(beta_k) (.) k, a = s (.) b (or b), w the
+// write vector:
+//   Qh = gamma q, Bh = gamma b, Ac = a / gamma, A = strictly-lower(Bh Ac^T), P = lower(Qh Ac^T),
+//   T = (I + A)^-1, Y = W - Bh S, U = T Y, M = S + Ac^T U, dM = Diag(gamma_C) dS
+//   dU = P^T dO + Ac dM,  dV = T^T dU,  dS_prev = Qh^T dO + dM - Bh^T dV   (the chain between chunks)
+//   dP = lower(dO U^T), dA = strictly-lower(-dV U^T)
+//   dQh^T = S dO^T + Ac^T dP^T,  dBh^T = -S dV^T + Ac^T dA^T,  dAc^T = Bh^T dA + Qh^T dP + dM U^T
+//   dgamma_r = q (.) dQh + b (.) dBh - Ac (.) dAc / gamma  (+ rowsum(dS (.) M) on the last row)
+//   dalpha_j = sum_{r>=j} dgamma_r gamma_r / alpha_j,  dq = gamma dQh,  db = gamma dBh,  da = dAc / gamma
+// then the chain rule through b, a and w.  The products that carry the gradients per key channel
+// (dQh, dBh, dAc) are formed transposed -- TMEM lane = key channel -- so that the per-channel
+// gate arithmetic (the running product gamma, the reverse cumulative sum of dalpha) is local to a
+// thread.
+//
+// One CTA of 256 threads per (b, h) walks its chunks from the last to the first; the fp32 gradient
+// of the state is carried in registers (thread: key row i, 64 value columns).  Every product uses
+// M = 128; where only 64 rows are meaningful, the other 64 rows read neighbouring tiles and are
+// ignored in TMEM.
+#pragma once
+#include "chunk_tc.cuh"
+
+namespace dr {
+namespace bwc {
+
+using tc::C;
+using tc::DK;
+using tc::kF16Max;
+using tc::kMinChunkDecayF16;
+constexpr int DV = 128;
+constexpr int NT = 256;
+
+// shared memory (bytes from a 1024-aligned base); 64-column blocks of R rows x 128 bytes
+constexpr uint32_t SX = 0;                        // [Bh; Qh]   128 x 128 (raw k, q land here)
+constexpr uint32_t SX_CB = 128 * 128;
+constexpr uint32_t SAC = 2 * SX_CB;               // Ac         64 x 128
+constexpr uint32_t SAC_CB = 64 * 128;
+constexpr uint32_t STP = SAC + 2 * SAC_CB;        // [A -> T; T^T scratch -> P]  128 x 64
+constexpr uint32_t SSS = STP + 128 * 128;         // S (fp16)   128 (dk) x 128 (dv)
+constexpr uint32_t SWY = SSS + 2 * 128 * 128;     // raw v -> W -> Y -> dU   64 x 128
+constexpr uint32_t SWY_CB = 64 * 128;
+constexpr uint32_t SUU = SWY + 2 * SWY_CB;        // U          64 x 128
+constexpr uint32_t SDM = SUU + 2 * SWY_CB;        // dM         128 x 128 (K1's gate products before)
+constexpr uint32_t SDO = SDM + 2 * 128 * 128;     // [dO; -dV]  128 x 128
+constexpr uint32_t SDPA = SDO + 2 * 128 * 128;    // [dP; dA]   128 x 64
+constexpr uint32_t SGC = SDPA + 128 * 128;        // gamma_C, 128 fp32
+constexpr uint32_t SROW = SGC + 512;              // scalar gates: gamma_r, 1/gamma_r, sqrt(beta_r), 64 each
+constexpr uint32_t SRT = SROW + 1024;             // last-row term partials, [2][128] fp32
+constexpr uint32_t SXC = SRT + 1024;              // per-channel exchange between the row halves, [2][128]
+constexpr uint32_t SRED = SXC + 1024;             // per-row sums over channels: [64 rows][4 warps][2] fp32
+constexpr uint32_t SRV = SRED + 64 * 4 * 2 * 4;   // per-row sums over value columns: [64 rows][2] fp32
+constexpr uint32_t SEND = SRV + 64 * 2 * 4;
+constexpr size_t SMEM_BYTES = SEND + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// TMEM columns
+constexpr uint32_t COL_D1 = 0;     // [A | P] raw (64); later [dP | dA] raw
+constexpr uint32_t COL_BS = 64;    // [Bh S | .] (128); later dU, then [dQh^T | dBh^T]
+constexpr uint32_t COL_U = 192;    // [U | .] (128); later dV, then dAc^T (64)
+constexpr uint32_t COL_AU = 320;   // Ac^T U (128); later the state gradient's step
+constexpr uint32_t TMEM_COLS = 512;
+
+struct BwdChunkParams {
+  int T, H, nchunks;
+  const float *alpha;
+  int alpha_mode;
+  const float *beta_k;
+  int beta_k_mode;
+  const float *beta_v;
+  int beta_v_mode;
+  const float *s;            // write-side key scale or nullptr
+  const __nv_bfloat16 *q, *k, *v;
+  const float *states;       // [B, H, nchunks, dk, dv]: the state at the start of every chunk
+  const float *dS_T;         // [B, H, dk, dv] or nullptr
+  float *dq, *dk, *dv, *dalpha, *dbeta_k, *dbeta_v, *ds, *dS0;
+  uint32_t *status;
+};
+
+template <bool kChanGates, bool kScaled>
+__global__ void __launch_bounds__(NT, 1)
+chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                 const BwdChunkParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_ld, bar_mma;
+  __shared__ uint32_t tmem_base_sh;
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quarter = warp & 3, half = warp >> 2;
+  const int h = blockIdx.x, b = blockIdx.y, H = p.H, T = p.T, NC = p.nchunks;
+  const size_t head = static_cast<size_t>(b) * H + h;
+  const bool sym_write = p.beta_v_mode == MODE_ABSENT;  // w = sqrt(beta_k) (.) v
+
+  uint8_t *X = sm + SX, *tAC = sm + SAC, *tTP = sm + STP, *tSS = sm + SSS, *tWY = sm + SWY, *tUU = sm + SUU;
+  uint8_t *tDM = sm + SDM, *tDO = sm + SDO, *tDPA = sm + SDPA;
+  float *sGC = reinterpret_cast<float *>(sm + SGC);
+  float *sRow = reinterpret_cast<float *>(sm + SROW);
+  float *sRT = reinterpret_cast<float *>(sm + SRT);
+  float *sXC = reinterpret_cast<float *>(sm + SXC);
+  float *sRed = reinterpret_cast<float *>(sm + SRED);
+  float *sRV = reinterpret_cast<float *>(sm + SRV);
+
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar_ld, 1);
+    mbar_init(&bar_mma, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  uint32_t ph_ld = 0, ph_mma = 0;
+  bool ok = true;
+
+  // bounded waits; a failure in any thread stops every thread at the same point
+  auto wait_mma = [&]() -> bool {
+    bool w = true;
+    if (tid == 0) w = mbar_wait(&bar_mma, ph_mma & 1u, kWaitLimitNs);
+    ph_mma++;
+    const bool fail = bar_or(1, NT, !w);
+    tc_fence_after();
+    if (fail && tid == 0) raise_status(p.status, STATUS_TIMEOUT);
+    return !fail;
+  };
+  // single-thread MMA issue: nk K-steps of 16 into column `col`; desc(kk) give the operands
+  auto issue = [&](uint32_t col, int nk, uint32_t idesc, bool acc, auto adesc, auto bdesc) {
+    for (int kk = 0; kk < nk; ++kk) umma_f16(tmem + col, adesc(kk), bdesc(kk), idesc, (acc || kk > 0) ? 1u : 0u);
+  };
+  auto kmaj = [](uint32_t saddr, int R) {  // K-major tile of R rows: descriptor of K-step kk
+    return [saddr, R](int kk) {
+      return sdesc_sw128(saddr + static_cast<uint32_t>((kk >> 2) * R * 128 + (kk & 3) * 32), 16, 1024);
+    };
+  };
+  auto mnmaj = [](uint32_t saddr, int R) {  // MN-major tile (rows = K) whose column blocks are R rows apart
+    return [saddr, R](int kk) {
+      return sdesc_sw128(saddr + static_cast<uint32_t>(kk) * 2048u, static_cast<uint32_t>(R) * 128u, 1024);
+    };
+  };
+
+  // the gradient of the state: row i = 32 quarter + lane, value columns 64 half .. 64 half + 63
+  const int srow = quarter * 32 + lane;
+  float dS[64];
+  {
+    const float *src = p.dS_T ? p.dS_T + head * DK * DV + static_cast<size_t>(srow) * DV + half * 64 : nullptr;
+#pragma unroll
+    for (int j = 0; j < 64; j += 4) {
+      const float4 x = src ? __ldg(reinterpret_cast<const float4 *>(src + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      dS[j] = x.x;
+      dS[j + 1] = x.y;
+      dS[j + 2] = x.z;
+      dS[j + 3] = x.w;
+    }
+  }
+
+  // element helpers for a thread's row of a 128-row, 128-column tile (two 64-column blocks)
+  auto st_row64 = [](uint8_t *tile, int R, int row, int col0, const float *v) {  // 64 values from col0
+#pragma unroll
+    for (int j = 0; j < 64; j += 16) tc::st_h16x16(tile, row, col0 + j, R, v + j);
+  };
+
+#pragma unroll 1
+  for (int c = NC - 1; c >= 0 && ok; --c) {
+    const int t0 = c * C, L = min(C, T - t0);
+    const size_t tok0 = static_cast<size_t>(b) * T + t0;  // first token of the chunk (dense batch)
+
+    // ------------------------------------------------------------------ loads: q, k, v, dO (TMA), S (global)
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&bar_ld, 8 * 64 * 128);
+      tma_load_4d(X + 64 * 128, &tm_q, &bar_ld, 0, h, t0, b);
+      tma_load_4d(X + SX_CB + 64 * 128, &tm_q, &bar_ld, 64, h, t0, b);
+      tma_load_4d(X, &tm_k, &bar_ld, 0, h, t0, b);
+      tma_load_4d(X + SX_CB, &tm_k, &bar_ld, 64, h, t0, b);
+      tma_load_4d(tWY, &tm_v, &bar_ld, 0, h, t0, b);
+      tma_load_4d(tWY + SWY_CB, &tm_v, &bar_ld, 64, h, t0, b);
+      tma_load_4d(tDO, &tm_do, &bar_ld, 0, h, t0, b);
+      tma_load_4d(tDO + 128 * 128, &tm_do, &bar_ld, 64, h, t0, b);
+      if (c > 0) {
+        for (int x = 0; x < 128; x += 64) {
+          tma_prefetch_l2_4d(&tm_q, x, h, t0 - C, b);
+          tma_prefetch_l2_4d(&tm_k, x, h, t0 - C, b);
+          tma_prefetch_l2_4d(&tm_v, x, h, t0 - C, b);
+          tma_prefetch_l2_4d(&tm_do, x, h, t0 - C, b);
+        }
+      }
+    }
+    // S of this chunk: fp16 operand tile, and the state part of the last-row term sum_v dS S
+    float rt = 0.f;
+    {
+      const float *src = p.states + (head * NC + c) * DK * DV + static_cast<size_t>(srow) * DV + half * 64;
+      if (c > 0) {  // the previous chunk's state into L2 (two 128-byte lines of my row half... all four)
+        const float *nx = p.states + (head * NC + c - 1) * DK * DV + static_cast<size_t>(srow) * DV + half * 64;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(nx));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(nx + 32));
+      }
+#pragma unroll
+      for (int j = 0; j < 64; j += 16) {
+        float x[16];
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const float4 y = __ldg(reinterpret_cast<const float4 *>(src + j + e));
+          x[e] = y.x;
+          x[e + 1] = y.y;
+          x[e + 2] = y.z;
+          x[e + 3] = y.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) rt += dS[j + e] * x[e];
+        tc::st_h16x16(tSS, srow, half * 64 + j, 128, x);
+      }
+    }
+    // gates
+    float pal[4 * 8], pbe[4 * 8];  // channel gates: rows 8 rg .. 8 rg + 7, channels c0 .. c0 + 3
+    const int rg = tid >> 5, c0 = 4 * (tid & 31);
+    if constexpr (kChanGates) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const size_t th = (tok0 + min(rg * 8 + j, L - 1)) * H + h;
+        if (p.alpha_mode == MODE_CHANNEL) {
+          const float4 a = __ldg(reinterpret_cast<const float4 *>(p.alpha + th * DK + c0));
+          pal[4 * j] = a.x; pal[4 * j + 1] = a.y; pal[4 * j + 2] = a.z; pal[4 * j + 3] = a.w;
+        } else {
+          const float a = p.alpha_mode == MODE_SCALAR ? __ldg(p.alpha + th) : 1.f;
+          pal[4 * j] = pal[4 * j + 1] = pal[4 * j + 2] = pal[4 * j + 3] = a;
+        }
+        if (p.beta_k_mode == MODE_CHANNEL) {
+          const float4 x = __ldg(reinterpret_cast<const float4 *>(p.beta_k + th * DK + c0));
+          pbe[4 * j] = x.x; pbe[4 * j + 1] = x.y; pbe[4 * j + 2] = x.z; pbe[4 * j + 3] = x.w;
+        } else {
+          const float x = __ldg(p.beta_k + th);
+          pbe[4 * j] = pbe[4 * j + 1] = pbe[4 * j + 2] = pbe[4 * j + 3] = x;
+        }
+        if (rg * 8 + j >= L) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            pal[4 * j + e] = 1.f;
+            pbe[4 * j + e] = 0.f;
+          }
+        }
+      }
+    } else if (warp == 0) {  // scalar gates: warp 0 scans the row gates (lane: rows 2 lane, 2 lane + 1)
+      float al[2], be[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int r = 2 * lane + e;
+        const size_t th = (tok0 + min(r, L - 1)) * H + h;
+        al[e] = (p.alpha_mode == MODE_SCALAR && r < L) ? __ldg(p.alpha + th) : 1.f;
+        be[e] = r < L ? __ldg(p.beta_k + th) : 0.f;
+      }
+      float incl = al[0] * al[1];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl *= y;
+      }
+      const float up = __shfl_up_sync(0xffffffffu, incl, 1);
+      const float g0 = (lane == 0 ? 1.f : up) * al[0], g1 = g0 * al[1];
+      sRow[2 * lane] = g0;
+      sRow[2 * lane + 1] = g1;
+      sRow[64 + 2 * lane] = __fdividef(1.f, g0);
+      sRow[64 + 2 * lane + 1] = __fdividef(1.f, g1);
+      sRow[128 + 2 * lane] = tc::sqrt_fast(be[0]);
+      sRow[128 + 2 * lane + 1] = tc::sqrt_fast(be[1]);
+      const float gC = __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sGC[4 * lane + e] = gC;
+      if (lane == 0 && !(gC >= kMinChunkDecayF16)) raise_status(p.status, STATUS_RANGE);
+    }
+    // wait for the tiles
+    {
+      const bool w = mbar_wait(&bar_ld, ph_ld & 1u, kWaitLimitNs);
+      ph_ld++;
+      if (bar_or(1, NT, !w)) {
+        if (tid == 0) raise_status(p.status, STATUS_TIMEOUT);
+        ok = false;
+        break;
+      }
+    }
+
+    // ------------------------------------------------------------------ K1: Qh, Bh, Ac; write vectors; dO -> fp16
+    float amax = 0.f;
+    if constexpr (kChanGates) {
+      float *sPX = reinterpret_cast<float *>(tDM);  // row-group gate products, 8 x 128 fp32
+      float pg[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pg[e] *= pal[4 * j + e];
+      *reinterpret_cast<float4 *>(sPX + rg * 128 + c0) = make_float4(pg[0], pg[1], pg[2], pg[3]);
+      __syncthreads();
+      float gr[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        if (g < rg) {
+          const float4 x = *reinterpret_cast<const float4 *>(sPX + g * 128 + c0);
+          gr[0] *= x.x; gr[1] *= x.y; gr[2] *= x.z; gr[3] *= x.w;
+        }
+      }
+      if (rg == 7) {
+        const float4 gC = make_float4(gr[0] * pg[0], gr[1] * pg[1], gr[2] * pg[2], gr[3] * pg[3]);
+        *reinterpret_cast<float4 *>(sGC + c0) = gC;
+        if (!(fminf(fminf(gC.x, gC.y), fminf(gC.z, gC.w)) >= kMinChunkDecayF16)) raise_status(p.status, STATUS_RANGE);
+      }
+      const uint32_t blk = static_cast<uint32_t>(c0 >> 6), grp = static_cast<uint32_t>((c0 & 63) >> 3);
+      const uint32_t inb = static_cast<uint32_t>((c0 & 7) * 2);
+      uint8_t *pQ = X + blk * SX_CB + (64 + rg * 8) * 128 + inb;
+      uint8_t *pB = X + blk * SX_CB + (rg * 8) * 128 + inb;
+      uint8_t *pA = tAC + blk * SAC_CB + (rg * 8) * 128 + inb;
+#pragma unroll 2
+      for (int jj = 0; jj < 8; ++jj) {
+        const uint32_t sw = ((grp ^ static_cast<uint32_t>(jj)) << 4) + jj * 128;
+        const uint2 kraw = *reinterpret_cast<const uint2 *>(pB + sw), qraw = *reinterpret_cast<const uint2 *>(pQ + sw);
+        const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kraw);
+        const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qraw);
+        const float2 k01 = __bfloat1622float2(k2[0]), k23 = __bfloat1622float2(k2[1]);
+        const float2 q01 = __bfloat1622float2(q2[0]), q23 = __bfloat1622float2(q2[1]);
+        const float kf[4] = {k01.x, k01.y, k23.x, k23.y}, qf[4] = {q01.x, q01.y, q23.x, q23.y};
+        float sc[4] = {1.f, 1.f, 1.f, 1.f};
+        if constexpr (kScaled) {
+          const size_t th = (tok0 + min(rg * 8 + jj, L - 1)) * H + h;
+          const float4 x = __ldg(reinterpret_cast<const float4 *>(p.s + th * DK + c0));
+          sc[0] = x.x; sc[1] = x.y; sc[2] = x.z; sc[3] = x.w;
+        }
+        float oq[4], ob[4], oa[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          gr[e] *= pal[4 * jj + e];
+          const float bv = tc::sqrt_fast(pbe[4 * jj + e]) * kf[e];
+          float av = bv * __fdividef(1.f, gr[e]);
+          if constexpr (kScaled) av *= sc[e];
+          amax = fmaxf(amax, fabsf(av));
+          oq[e] = gr[e] * qf[e];
+          ob[e] = gr[e] * bv;
+          oa[e] = av;
+        }
+        *reinterpret_cast<uint2 *>(pQ + sw) = make_uint2(pack_f16x2(oq[0], oq[1]), pack_f16x2(oq[2], oq[3]));
+        *reinterpret_cast<uint2 *>(pB + sw) = make_uint2(pack_f16x2(ob[0], ob[1]), pack_f16x2(ob[2], ob[3]));
+        *reinterpret_cast<uint2 *>(pA + sw) = make_uint2(pack_f16x2(oa[0], oa[1]), pack_f16x2(oa[2], oa[3]));
+      }
+    } else {
+      __syncthreads();  // the row gates of warp 0
+      const int j8 = tid & 15;
+#pragma unroll 1
+      for (int i = 0; i < 4; ++i) {
+        const int r = (tid >> 4) + 16 * i;
+        const float g = sRow[r], gi = sRow[64 + r], sbt = sRow[128 + r];
+        float ssc[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+        if constexpr (kScaled) {
+          const float4 *src = reinterpret_cast<const float4 *>(p.s + ((tok0 + min(r, L - 1)) * H + h) * DK + j8 * 8);
+          const float4 lo = __ldg(src), hi = __ldg(src + 1);
+          ssc[0] = lo.x; ssc[1] = lo.y; ssc[2] = lo.z; ssc[3] = lo.w;
+          ssc[4] = hi.x; ssc[5] = hi.y; ssc[6] = hi.z; ssc[7] = hi.w;
+        }
+        uint4 *pq = reinterpret_cast<uint4 *>(X + sw128_off16(64 + r, j8, 128));
+        uint4 *pk = reinterpret_cast<uint4 *>(X + sw128_off16(r, j8, 128));
+        const uint4 qraw = *pq, kraw = *pk;
+        const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qraw);
+        const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kraw);
+        uint32_t oq[4], ob[4], oa[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 qf = __bfloat1622float2(q2[e]), kf = __bfloat1622float2(k2[e]);
+          const float b0 = sbt * kf.x, b1 = sbt * kf.y;
+          float x0 = b0 * gi, x1 = b1 * gi;
+          if constexpr (kScaled) {
+            x0 *= ssc[2 * e];
+            x1 *= ssc[2 * e + 1];
+          }
+          amax = fmaxf(amax, fmaxf(fabsf(x0), fabsf(x1)));
+          oq[e] = pack_f16x2(g * qf.x, g * qf.y);
+          ob[e] = pack_f16x2(g * b0, g * b1);
+          oa[e] = pack_f16x2(x0, x1);
+        }
+        *pq = make_uint4(oq[0], oq[1], oq[2], oq[3]);
+        *pk = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+        *reinterpret_cast<uint4 *>(tAC + sw128_off16(r, j8, 64)) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+      }
+    }
+    if (!(amax < kF16Max)) raise_status(p.status, STATUS_RANGE);
+    // write vectors W = wsc (.) v in place of raw v, and dO as fp16 in place: thread row tid >> 2,
+    // 8-column groups 4 (tid & 3) .. 4 (tid & 3) + 3 of 16
+    {
+      const int r = tid >> 2;
+      const size_t th = (tok0 + min(r, L - 1)) * H + h;
+#pragma unroll 1
+      for (int g = 0; g < 4; ++g) {
+        const int c8 = 4 * (tid & 3) + g;  // 8-column group (0..15)
+        float wsc[8];
+        if (p.beta_v_mode == MODE_CHANNEL) {
+          const float4 *src = reinterpret_cast<const float4 *>(p.beta_v + th * DV + c8 * 8);
+          const float4 lo = __ldg(src), hi = __ldg(src + 1);
+          wsc[0] = lo.x; wsc[1] = lo.y; wsc[2] = lo.z; wsc[3] = lo.w;
+          wsc[4] = hi.x; wsc[5] = hi.y; wsc[6] = hi.z; wsc[7] = hi.w;
+        } else if (p.beta_v_mode == MODE_SCALAR) {
+          const float x = __ldg(p.beta_v + th);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) wsc[e] = x;
+        } else if (p.beta_k_mode == MODE_CHANNEL) {
+          const float4 *src = reinterpret_cast<const float4 *>(p.beta_k + th * DK + c8 * 8);
+          const float4 lo = __ldg(src), hi = __ldg(src + 1);
+          wsc[0] = tc::sqrt_fast(lo.x); wsc[1] = tc::sqrt_fast(lo.y); wsc[2] = tc::sqrt_fast(lo.z);
+          wsc[3] = tc::sqrt_fast(lo.w); wsc[4] = tc::sqrt_fast(hi.x); wsc[5] = tc::sqrt_fast(hi.y);
+          wsc[6] = tc::sqrt_fast(hi.z); wsc[7] = tc::sqrt_fast(hi.w);
+        } else {
+          const float x = tc::sqrt_fast(__ldg(p.beta_k + th));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) wsc[e] = x;
+        }
+        uint4 *pv = reinterpret_cast<uint4 *>(tWY + sw128_off16(r, c8, 64));
+        uint4 *pd = reinterpret_cast<uint4 *>(tDO + sw128_off16(r, c8, 128));
+        const uint4 vraw = *pv, draw = *pd;
+        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vraw);
+        const __nv_bfloat162 *d2 = reinterpret_cast<const __nv_bfloat162 *>(&draw);
+        uint32_t ow[4], od[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 vf = __bfloat1622float2(v2[e]), df = __bfloat1622float2(d2[e]);
+          const bool valid = r < L;
+          ow[e] = pack_f16x2(valid ? wsc[2 * e] * vf.x : 0.f, valid ? wsc[2 * e + 1] * vf.y : 0.f);
+          od[e] = pack_f16x2(valid ? df.x : 0.f, valid ? df.y : 0.f);
+        }
+        *pv = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        *pd = make_uint4(od[0], od[1], od[2], od[3]);
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ------------------------------------------------------------------ m1: [A | P] = [Bh; Qh] Ac^T;  Bh S
+    if (warp == 0) {
+      if (elect_one()) {
+        tc_fence_after();
+        issue(COL_D1, DK / 16, idesc_f16_f32(128, 64, false, false), false, kmaj(sb + SX, 128), kmaj(sb + SAC, 64));
+        issue(COL_BS, DK / 16, idesc_f16_f32(128, 128, false, true), false, kmaj(sb + SX, 128),
+              mnmaj(sb + SSS, 128));
+        umma_commit(&bar_mma);
+      }
+      __syncwarp();
+    }
+    if (!wait_mma()) { ok = false; break; }
+    // E1a: A (strictly lower) -> TP rows 0..63
+    if (quarter < 2) {
+      float x[32];
+      tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D1 + half * 32), *reinterpret_cast<float(*)[16]>(x));
+      tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D1 + half * 32 + 16), *reinterpret_cast<float(*)[16]>(x + 16));
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) x[i] = (half * 32 + i < srow) ? x[i] : 0.f;
+      tc::st_h16x16(tTP, srow, half * 32, 128, x);
+      tc::st_h16x16(tTP, srow, half * 32 + 16, 128, x + 16);
+    }
+    tc_fence_before();
+    __syncthreads();
+    // T = (I + A)^-1 (warps 0..3)
+    if (warp < 4) {
+      tri::Frag Trow[4];
+      tri::inverse64_rows<tri::Sw128Layout>(tTP, tTP + 64 * 128, warp, lane, Trow, [] { bar_sync(2, 128); });
+      const int rr = lane >> 2, qq = lane & 3;
+#pragma unroll
+      for (int d = 0; d < 4; ++d) {
+        if (d <= warp) {
+          const tri::Frag &F = Trow[d];
+          const int row = 16 * warp + rr, col = 16 * (warp - d) + 2 * qq;
+          *reinterpret_cast<uint32_t *>(tTP + sw128_off(row, col, 128)) = pack_f16x2(F.v[0], F.v[1]);
+          *reinterpret_cast<uint32_t *>(tTP + sw128_off(row + 8, col, 128)) = pack_f16x2(F.v[2], F.v[3]);
+          *reinterpret_cast<uint32_t *>(tTP + sw128_off(row, col + 8, 128)) = pack_f16x2(F.v[4], F.v[5]);
+          *reinterpret_cast<uint32_t *>(tTP + sw128_off(row + 8, col + 8, 128)) = pack_f16x2(F.v[6], F.v[7]);
+        }
+      }
+    }
+    __syncthreads();
+    // E1b: P (lower with diagonal) -> TP rows 64..127 (after the inverse's scratch use);  Y = W - Bh S
+    if (quarter >= 2) {
+      const int r = srow - 64;
+      float x[32];
+      tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D1 + half * 32), *reinterpret_cast<float(*)[16]>(x));
+      tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D1 + half * 32 + 16), *reinterpret_cast<float(*)[16]>(x + 16));
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) x[i] = (half * 32 + i <= r) ? x[i] : 0.f;
+      tc::st_h16x16(tTP, srow, half * 32, 128, x);
+      tc::st_h16x16(tTP, srow, half * 32 + 16, 128, x + 16);
+    } else {
+      // rows 0..63 of Bh S: Y = W - Bh S into the write-vector tile, in place
+#pragma unroll 1
+      for (int j = 0; j < 64; j += 16) {
+        float x[16];
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_BS + half * 64 + j), x);
+        tmem_ld_wait();
+        float y[16];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const int c8 = (half * 64 + j) / 8 + g;
+          const uint4 wraw = *reinterpret_cast<const uint4 *>(tWY + sw128_off16(srow, c8, 64));
+          const __half2 *w2 = reinterpret_cast<const __half2 *>(&wraw);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 wf = __half22float2(w2[e]);
+            y[8 * g + 2 * e] = wf.x - x[8 * g + 2 * e];
+            y[8 * g + 2 * e + 1] = wf.y - x[8 * g + 2 * e + 1];
+          }
+        }
+        float mx = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(y[e]));
+        if (!(mx < kF16Max)) raise_status(p.status, STATUS_RANGE);
+        tc::st_h16x16(tWY, srow, half * 64 + j, 64, y);
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ------------------------------------------------------------------ U = [T; P] Y
+    if (warp == 0) {
+      if (elect_one()) {
+        tc_fence_after();
+        issue(COL_U, C / 16, idesc_f16_f32(128, 128, false, true), false, kmaj(sb + STP, 128), mnmaj(sb + SWY, 64));
+        umma_commit(&bar_mma);
+      }
+      __syncwarp();
+    }
+    if (!wait_mma()) { ok = false; break; }
+    if (quarter < 2) {
+#pragma unroll 1
+      for (int j = 0; j < 64; j += 16) {
+        float x[16];
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_U + half * 64 + j), x);
+        tmem_ld_wait();
+        float mx = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(x[e]));
+        if (!(mx < kF16Max)) raise_status(p.status, STATUS_RANGE);
+        tc::st_h16x16(tUU, srow, half * 64 + j, 64, x);
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ------------------------------------------------------------------ Ac^T U;  dM = Diag(gamma_C) dS
+    if (warp == 0) {
+      if (elect_one()) {
+        tc_fence_after();
+        issue(COL_AU, C / 16, idesc_f16_f32(128, 128, true, true), false, mnmaj(sb + SAC, 64), mnmaj(sb + SUU, 64));
+        umma_commit(&bar_mma);
+      }
+      __syncwarp();
+    }
+    const float gci = sGC[srow];
+    {
+      float dm[64];
+#pragma unroll
+      for (int e = 0; e < 64; ++e) dm[e] = gci * dS[e];
+      st_row64(tDM, 128, srow, half * 64, dm);
+    }
+    if (!wait_mma()) { ok = false; break; }
+    // last-row term: sum_v dS (S + Ac^T U), per key row; the two value halves meet in shared memory
+#pragma unroll 1
+    for (int j = 0; j < 64; j += 16) {
+      float x[16];
+      tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), x);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) rt += dS[j + e] * x[e];
+    }
+    sRT[half * 128 + srow] = rt;
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ------------------------------------------------------------------ dU = P^T dO + Ac dM
+    if (warp == 0) {
+      if (elect_one()) {
+        tc_fence_after();
+        issue(COL_BS, C / 16, idesc_f16_f32(128, 128, true, true), false, mnmaj(sb + STP + 64 * 128, 128),
+              mnmaj(sb + SDO, 128));
+        issue(COL_BS, DK / 16, idesc_f16_f32(128, 128, false, true), true, kmaj(sb + SAC, 64), mnmaj(sb + SDM, 128));
+        umma_commit(&bar_mma);
+      }
+      __syncwarp();
+    }
+    if (!wait_mma()) { ok = false; break; }
+    if (quarter < 2) {  // dU -> the write-vector tile (Y is no longer read)
+#pragma unroll 1
+      for (int j = 0; j < 64; j += 16) {
+        float x[16];
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_BS + half * 64 + j), x);
+        tmem_ld_wait();
+        float mx = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(x[e]));
+        if (!(mx < kF16Max)) raise_status(p.status, STATUS_RANGE);
+        tc::st_h16x16(tWY, srow, half * 64 + j, 64, x);
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ------------------------------------------------------------------ dV = T^T dU -> -dV, dv, write strengths
+    if (warp == 0) {
+      if (elect_one()) {
+        tc_fence_after();
+        issue(COL_U, C / 16, idesc_f16_f32(128, 128, true, true), false, mnmaj(sb + STP, 128), mnmaj(sb + SWY, 64));
+        umma_commit(&bar_mma);
+      }
+      __syncwarp();
+    }
+    if (!wait_mma()) { ok = false; break; }
+    if (quarter < 2) {
+      const int r = srow;
+      const size_t th = (tok0 + min(r, L - 1)) * H + h;
+      float rsum = 0.f;  // sum over my value columns of v dV (scalar write strength)
+#pragma unroll 1
+      for (int j = 0; j < 64; j += 16) {
+        float x[16];
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_U + half * 64 + j), x);
+        tmem_ld_wait();
+        const int v0 = half * 64 + j;
+        float nd[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) nd[e] = -x[e];
+        tc::st_h16x16(tDO, 64 + r, v0, 128, nd);
+        if (r < L) {
+          // raw v and the write scale of these 16 columns
+          float vf[16], wsc[16];
+          const uint4 *vsrc = reinterpret_cast<const uint4 *>(p.v + th * DV + v0);
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            const uint4 raw = __ldg(vsrc + g);
+            const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(v2[e]);
+              vf[8 * g + 2 * e] = f.x;
+              vf[8 * g + 2 * e + 1] = f.y;
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 16; e += 4) {
+            float4 wq;
+            if (p.beta_v_mode == MODE_CHANNEL) {
+              wq = __ldg(reinterpret_cast<const float4 *>(p.beta_v + th * DV + v0 + e));
+            } else if (p.beta_v_mode == MODE_SCALAR) {
+              const float y = __ldg(p.beta_v + th);
+              wq = make_float4(y, y, y, y);
+            } else if (p.beta_k_mode == MODE_CHANNEL) {
+              const float4 y = __ldg(reinterpret_cast<const float4 *>(p.beta_k + th * DK + v0 + e));
+              wq = make_float4(tc::sqrt_fast(y.x), tc::sqrt_fast(y.y), tc::sqrt_fast(y.z), tc::sqrt_fast(y.w));
+            } else {
+              const float y = tc::sqrt_fast(__ldg(p.beta_k + th));
+              wq = make_float4(y, y, y, y);
+            }
+            wsc[e] = wq.x; wsc[e + 1] = wq.y; wsc[e + 2] = wq.z; wsc[e + 3] = wq.w;
+          }
+          float *dvo = p.dv + th * DV + v0;
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<float4 *>(dvo + e) =
+                make_float4(wsc[e] * x[e], wsc[e + 1] * x[e + 1], wsc[e + 2] * x[e + 2], wsc[e + 3] * x[e + 3]);
+          // gradient of the write scale: v (.) dV per column
+          if (p.beta_v_mode == MODE_CHANNEL) {
+            float *o = p.dbeta_v + th * DV + v0;
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+              *reinterpret_cast<float4 *>(o + e) =
+                  make_float4(vf[e] * x[e], vf[e + 1] * x[e + 1], vf[e + 2] * x[e + 2], vf[e + 3] * x[e + 3]);
+          } else if (p.beta_v_mode == MODE_SCALAR) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) rsum += vf[e] * x[e];
+          } else if (p.beta_k_mode == MODE_CHANNEL) {
+            // symmetric channel write: d beta_k += 0.5 v dV / sqrt(beta_k), stored now, added to below
+            float *o = p.dbeta_k + th * DK + v0;
+#pragma unroll
+            for (int e = 0; e < 16; e += 4) {
+              float4 y;
+              y.x = wsc[e] > 0.f ? 0.5f * vf[e] * x[e] / wsc[e] : 0.f;
+              y.y = wsc[e + 1] > 0.f ? 0.5f * vf[e + 1] * x[e + 1] / wsc[e + 1] : 0.f;
+              y.z = wsc[e + 2] > 0.f ? 0.5f * vf[e + 2] * x[e + 2] / wsc[e + 2] : 0.f;
+              y.w = wsc[e + 3] > 0.f ? 0.5f * vf[e + 3] * x[e + 3] / wsc[e + 3] : 0.f;
+              *reinterpret_cast<float4 *>(o + e) = y;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) rsum += vf[e] * x[e];
+          }
+        }
+      }
+      sRV[r * 2 + half] = rsum;
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid < 64 && tid < L) {  // scalar write strength: one value per row
+      const int r = tid;
+      const size_t th = (tok0 + r) * H + h;
+      const float rs = sRV[2 * r] + sRV[2 * r + 1];
+      if (p.beta_v_mode == MODE_SCALAR) p.dbeta_v[th] = rs;
+      else if (p.beta_k_mode == MODE_SCALAR) sRV[2 * r] = rs;  // symmetric scalar write: folded in below
+    }
+
+    // ------------------------------------------------------------------ dS_prev = Qh^T dO - Bh^T dV + dM;  [dP | dA]
+    if (warp == 0) {
+      if (elect_one()) {
+        tc_fence_after();
+        const uint32_t id = idesc_f16_f32(128, 128, true, true);
+        issue(COL_AU, C / 16, id, false, mnmaj(sb + SX + 64 * 128, 128), mnmaj(sb + SDO, 128));
+        issue(COL_AU, C / 16, id, true, mnmaj(sb + SX, 128), mnmaj(sb + SDO + 64 * 128, 128));
+        issue(COL_D1, DV / 16, idesc_f16_f32(128, 64, false, false), false, kmaj(sb + SDO, 128), kmaj(sb + SUU, 64));
+        umma_commit(&bar_mma);
+      }
+      __syncwarp();
+    }
+    if (!wait_mma()) { ok = false; break; }
+    {
+      float mx = 0.f;
+#pragma unroll 1
+      for (int j = 0; j < 64; j += 16) {
+        float x[16];
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), x);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          dS[j + e] = gci * dS[j + e] + x[e];
+          mx = fmaxf(mx, fabsf(dS[j + e]));
+        }
+      }
+      if (!(mx < kF16Max)) raise_status(p.status, STATUS_RANGE);
+    }
+    {  // dP (lower with diagonal, lanes 0..63) and dA (strictly lower, lanes 64..127)
+      const int r = srow & 63;
+      float x[32];
+      tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D1 + half * 32), *reinterpret_cast<float(*)[16]>(x));
+      tmem_ld16(tmem_addr(tmem, quarter * 32, COL_D1 + half * 32 + 16), *reinterpret_cast<float(*)[16]>(x + 16));
+      tmem_ld_wait();
+      const bool strict = quarter >= 2;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int col = half * 32 + i;
+        x[i] = (strict ? col < r : col <= r) ? x[i] : 0.f;
+      }
+      tc::st_h16x16(tDPA, srow, half * 32, 128, x);
+      tc::st_h16x16(tDPA, srow, half * 32 + 16, 128, x + 16);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ------------------------------------------------------------------ [dQh^T | dBh^T] and dAc^T, lanes = key channels
+    if (warp == 0) {
+      if (elect_one()) {
+        tc_fence_after();
+        issue(COL_BS, DV / 16, idesc_f16_f32(128, 128, false, false), false, kmaj(sb + SSS, 128), kmaj(sb + SDO, 128));
+        issue(COL_BS, C / 16, idesc_f16_f32(128, 128, true, false), true, mnmaj(sb + SAC, 64), kmaj(sb + SDPA, 128));
+        const uint32_t id = idesc_f16_f32(128, 64, true, true);
+        issue(COL_U, C / 16, id, false, mnmaj(sb + SX, 128), mnmaj(sb + SDPA + 64 * 128, 128));
+        issue(COL_U, C / 16, id, true, mnmaj(sb + SX + 64 * 128, 128), mnmaj(sb + SDPA, 128));
+        issue(COL_U, DV / 16, idesc_f16_f32(128, 64, false, false), true, kmaj(sb + SDM, 128), kmaj(sb + SUU, 64));
+        umma_commit(&bar_mma);
+      }
+      __syncwarp();
+    }
+    if (!wait_mma()) { ok = false; break; }
+
+    // ------------------------------------------------------------------ per key channel: gate gradients and outputs
+    // thread: channel i = srow, rows 32 half .. 32 half + 31 of the chunk
+    {
+      const int i = srow, r0 = 32 * half;
+      const float rowterm = sRT[i] + sRT[128 + i];
+      // gamma of my rows: forward products (the lower half passes its product to the upper half)
+      float al[32], gam[32];
+      float prod = 1.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int r = r0 + j;
+        const size_t th = (tok0 + min(r, L - 1)) * H + h;
+        float a = 1.f;
+        if (r < L) {
+          if (p.alpha_mode == MODE_CHANNEL) a = __ldg(p.alpha + th * DK + i);
+          else if (p.alpha_mode == MODE_SCALAR) a = __ldg(p.alpha + th);
+        }
+        al[j] = a;
+        prod *= a;
+      }
+      if (half == 0) sXC[i] = prod;
+      __syncthreads();
+      float g = half == 0 ? 1.f : sXC[i];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        g *= al[j];
+        gam[j] = g;
+      }
+      // reverse over my rows: dgamma, the local suffix sums of dgamma gamma, and the outputs
+      float suf[32];
+      float acc = 0.f;
+#pragma unroll
+      for (int jb = 16; jb >= 0; jb -= 16) {
+        float dq[16], db[16], da[16];
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_BS + r0 + jb), dq);
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_BS + 64 + r0 + jb), db);
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_U + r0 + jb), da);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 15; e >= 0; --e) {
+          const int j = jb + e, r = r0 + j;
+          const size_t th = (tok0 + min(r, L - 1)) * H + h;
+          const float gm = gam[j];
+          const float qv = __bfloat162float(p.q[th * DK + i]);
+          const float kv = __bfloat162float(p.k[th * DK + i]);
+          float bet = 0.f;
+          if (r < L) bet = p.beta_k_mode == MODE_CHANNEL ? __ldg(p.beta_k + th * DK + i) : __ldg(p.beta_k + th);
+          const float sbt = tc::sqrt_fast(bet);
+          const float scv = kScaled ? (r < L ? __ldg(p.s + th * DK + i) : 0.f) : 1.f;
+          const float bv = sbt * kv, av = scv * bv;
+          const float ginv = __fdividef(1.f, gm);
+          float dg = qv * dq[e] + bv * db[e] - av * ginv * da[e] * ginv;
+          if (r == C - 1) dg += rowterm;
+          acc += dg * gm;
+          suf[j] = acc;
+          if (r < L) {
+            const float dqv = gm * dq[e];
+            const float dbv = gm * db[e], dav = da[e] * ginv;
+            const float dbt = dbv + scv * dav;  // through b = sqrt(beta) k and a = s b
+            p.dq[th * DK + i] = dqv;
+            p.dk[th * DK + i] = sbt * dbt;
+            if constexpr (kScaled) p.ds[th * DK + i] = bv * dav;
+            const float dsb = kv * dbt;  // d / d sqrt(beta_k)
+            const float dbk = sbt > 0.f ? 0.5f * dsb / sbt : 0.f;
+            if (p.beta_k_mode == MODE_CHANNEL) {
+              const float prev = (sym_write) ? p.dbeta_k[th * DK + i] : 0.f;
+              p.dbeta_k[th * DK + i] = prev + dbk;
+            } else {
+              // scalar: summed over channels below
+              float v = dbk;
+#pragma unroll
+              for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+              if (lane == 0) sRed[(r * 4 + quarter) * 2 + 0] = v;
+            }
+          }
+        }
+      }
+      // the upper half's total flows into the lower half's suffix sums
+      if (half == 1) sXC[128 + i] = acc;
+      __syncthreads();
+      const float off = half == 0 ? sXC[128 + i] : 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int r = r0 + j;
+        if (r < L) {
+          const size_t th = (tok0 + r) * H + h;
+          const float da_ = (suf[j] + off) / al[j];
+          if (p.alpha_mode == MODE_CHANNEL) {
+            p.dalpha[th * DK + i] = da_;
+          } else if (p.alpha_mode == MODE_SCALAR) {
+            float v = da_;
+#pragma unroll
+            for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
+            if (lane == 0) sRed[(r * 4 + quarter) * 2 + 1] = v;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (tid < 64 && tid < L) {  // scalar gates: sums over the four channel quarters
+      const int r = tid;
+      const size_t th = (tok0 + r) * H + h;
+      if (p.alpha_mode == MODE_SCALAR)
+        p.dalpha[th] = sRed[(r * 4) * 2 + 1] + sRed[(r * 4 + 1) * 2 + 1] + sRed[(r * 4 + 2) * 2 + 1] +
+                       sRed[(r * 4 + 3) * 2 + 1];
+      if (p.beta_k_mode == MODE_SCALAR) {
+        float v = sRed[(r * 4) * 2] + sRed[(r * 4 + 1) * 2] + sRed[(r * 4 + 2) * 2] + sRed[(r * 4 + 3) * 2];
+        if (sym_write) {  // w = sqrt(beta_k) v as well: 0.5 / sqrt(beta_k) sum_v v dV
+          const float sbt = tc::sqrt_fast(__ldg(p.beta_k + th));
+          v += sbt > 0.f ? 0.5f * sRV[2 * r] / sbt : 0.f;
+        }
+        p.dbeta_k[th] = v;
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+
+  if (ok && p.dS0) {
+    float *dst = p.dS0 + head * DK * DV + static_cast<size_t>(srow) * DV + half * 64;
+#pragma unroll
+    for (int j = 0; j < 64; j += 4) *reinterpret_cast<float4 *>(dst + j) = make_float4(dS[j], dS[j + 1], dS[j + 2], dS[j + 3]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace bwc
+}  // namespace dr

@@ -92,6 +92,9 @@ struct Params {
   uint32_t *status;
   const float *s = nullptr;  // write-side key scale [B,T,H,dk] (a = s (.) b); only the ring kernel reads it
   const int *cu_seqlens = nullptr;  // packed batch: sequence b is tokens cu[b] .. cu[b+1]-1 (ring kernel only)
+  // ring kernel, dense batch only: the state at the start of every chunk, [B, H, ceil(T/64), dk, dv] fp32
+  // (for the chunkwise backward pass); NULL: not stored
+  float *states = nullptr;
 };
 
 __device__ __forceinline__ void st_h16x8(uint8_t *tile, int row, int col0, int R, const float *v) {

@@ -723,7 +723,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           float x[16];
           tmem_ld16(tmem_addr(tmem, quarter * 32, col_d3(c) + half * 32 + j), x);
           tmem_ld_wait();
-          if (r < L) {
+          if (r < L && p.o) {
             const size_t th = (tok0 + t0 + r) * H + h;
             IO *dst = static_cast<IO *>(p.o) + th * DV + v0 + half * 32 + j;
             uint4 lo, hi;
@@ -831,6 +831,13 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       }
       if (c > 0) store_o(c - 1);  // overlaps the MMAs above
       if (!run) break;
+      if (p.states) {  // this chunk's initial state, for the backward pass (dense batches only)
+        float *dst = p.states + ((sbase / (static_cast<size_t>(DK) * DV)) * nchunks + c) * DK * DV +
+                     static_cast<size_t>(trow) * DV + v0 + half * 32;
+#pragma unroll
+        for (int jj = 0; jj < 32; jj += 4)
+          *reinterpret_cast<float4 *>(dst + jj) = make_float4(Sreg[jj], Sreg[jj + 1], Sreg[jj + 2], Sreg[jj + 3]);
+      }
       // MMA group 1 done; U goes into X rows 0..63 of this slot, which in the producing CTA must
       // wait until the copies out of it have landed in the other CTA
       {

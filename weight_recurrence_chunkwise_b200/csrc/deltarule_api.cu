@@ -19,6 +19,7 @@
 #include "decode_stream.cuh"
 #include "state_map.cuh"
 #include "backward.cuh"
+#include "backward_chunk.cuh"
 #include "umma_selftest.cuh"
 #include "wait_selftest.cuh"
 
@@ -172,9 +173,12 @@ dr_status tc_launch(const dr_problem *p, const void *q, const void *k, const voi
   return launch_status();
 }
 
+// states: NULL, or [B, H, ceil(T/64), dk, dv] fp32 receiving the state at the start of every chunk
+// (dense batch only; the chunkwise backward's first pass, which passes o = NULL).
 dr_status tc_ring_launch(const dr_problem *p, const int *cu, const void *q, const void *k, const void *v,
                          const float *alpha, const float *beta_k, const float *beta_v, const float *s_scale,
-                         const float *S0, void *o, float *S_T, uint32_t *status, cudaStream_t st) {
+                         const float *S0, void *o, float *S_T, uint32_t *status, cudaStream_t st,
+                         float *states = nullptr) {
   using IO = __nv_bfloat16;
   namespace tc = dr::tc;
   namespace tc3 = dr::tc3;
@@ -187,7 +191,7 @@ dr_status tc_ring_launch(const dr_problem *p, const int *cu, const void *q, cons
       !make_map(&mv, bf, 2, v, mB, p->T, p->H, p->dv, tc::VS, tc::C, sw))
     return DR_ERR_CUDA;
   tc::Params prm{p->T, p->H, p->dv, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v, p->beta_v_mode,
-                 S0, o, S_T, status, s_scale, cu};
+                 S0, o, S_T, status, s_scale, cu, states};
   const bool chan_gates = p->alpha_mode == DR_CHANNEL || p->beta_k_mode != DR_SCALAR;
   auto kern = s_scale ? (chan_gates ? tc3::chunk_fwd_ring_kernel<IO, true, true>
                                     : tc3::chunk_fwd_ring_kernel<IO, false, true>)
@@ -357,21 +361,81 @@ dr_status bwd_dispatch(const dr_problem *p, const dr::BwdParams &bp, cudaStream_
   return bwd_launch<IO, 64, 64>(bp, heads, st);
 }
 
+// ----------------------------------------------------------------- backward, chunkwise on the tensor cores
+// bf16 I/O, dk = dv = 128: a forward pass of the ring prefill keeps the state at the start of every
+// chunk, then one CTA per (b, h) walks the chunks from the last (backward_chunk.cuh).
+enum BackwardVariant { kBwdDefault = 0, kBwdSequential = 1, kBwdChunk = 2 };
+
+bool bwd_chunk_shape(const dr_problem *p) { return p->io_dtype == DR_BF16 && p->dk == 128 && p->dv == 128; }
+
+size_t bwd_chunk_workspace_bytes(const dr_problem *p) {
+  const size_t nc = (static_cast<size_t>(p->T) + dr::tc::C - 1) / dr::tc::C;
+  return kWorkspaceBytes + sizeof(float) * static_cast<size_t>(p->B) * p->H * nc * p->dk * p->dv;
+}
+
+int resolve_bwd_variant(const dr_problem *p, int variant) {
+  if (variant == kBwdDefault) return bwd_chunk_shape(p) ? kBwdChunk : kBwdSequential;
+  return variant;
+}
+
+size_t bwd_variant_workspace_bytes(const dr_problem *p, int variant) {
+  return resolve_bwd_variant(p, variant) == kBwdChunk ? bwd_chunk_workspace_bytes(p) : bwd_workspace_bytes(p);
+}
+
+dr_status bwd_chunk_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                           const float *beta_k, const float *beta_v, const float *s, const float *S0,
+                           const void *dout, const float *dS_T, float *dq, float *dk, float *dv, float *dalpha,
+                           float *dbeta_k, float *dbeta_v, float *ds, float *dS0, void *workspace, cudaStream_t st) {
+  namespace bwc = dr::bwc;
+  uint32_t *status = static_cast<uint32_t *>(workspace);
+  float *states = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kWorkspaceBytes);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DR_ERR_CUDA;
+  dr_problem pf = *p;
+  pf.chunk = dr::tc::C;
+  dr_status r = tc_ring_launch(&pf, nullptr, q, k, v, alpha, beta_k, beta_v, s, S0, nullptr, nullptr, status, st,
+                               states);
+  if (r != DR_OK) return r;
+  alignas(64) CUtensorMap mq, mk, mv, mdo;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_map(&mq, bf, 2, q, p->B, p->T, p->H, p->dk, 64, dr::tc::C, sw) ||
+      !make_map(&mk, bf, 2, k, p->B, p->T, p->H, p->dk, 64, dr::tc::C, sw) ||
+      !make_map(&mv, bf, 2, v, p->B, p->T, p->H, p->dv, 64, dr::tc::C, sw) ||
+      !make_map(&mdo, bf, 2, dout, p->B, p->T, p->H, p->dv, 64, dr::tc::C, sw))
+    return DR_ERR_CUDA;
+  const int nc = (p->T + dr::tc::C - 1) / dr::tc::C;
+  bwc::BwdChunkParams bp{p->T, p->H, nc, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v, p->beta_v_mode, s,
+                         static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                         static_cast<const __nv_bfloat16 *>(v), states, dS_T, dq, dk, dv, dalpha, dbeta_k, dbeta_v,
+                         ds, dS0, status};
+  const bool chan = p->alpha_mode == DR_CHANNEL || p->beta_k_mode != DR_SCALAR;
+  auto kern = s ? (chan ? bwc::chunk_bwd_kernel<true, true> : bwc::chunk_bwd_kernel<false, true>)
+                : (chan ? bwc::chunk_bwd_kernel<true, false> : bwc::chunk_bwd_kernel<false, false>);
+  constexpr size_t smem = bwc::SMEM_BYTES;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return DR_ERR_CUDA;
+  kern<<<dim3(p->H, p->B), bwc::NT, smem, st>>>(mq, mk, mv, mdo, bp);
+  return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
 
 size_t dr_backward_workspace(const dr_problem *p) {
-  return check_common(p, false) == DR_OK ? bwd_workspace_bytes(p) : 0;
+  return check_common(p, false) == DR_OK ? bwd_variant_workspace_bytes(p, kBwdDefault) : 0;
 }
 
-dr_status dr_backward(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
-                      const float *beta_k, const float *beta_v, const float *s, const float *S0, const void *dout,
-                      const float *dS_T, float *dq, float *dk, float *dv, float *dalpha, float *dbeta_k,
-                      float *dbeta_v, float *ds, float *dS0, void *workspace, size_t workspace_bytes,
-                      void *stream) {
+static dr_status backward_impl(int variant, const dr_problem *p, const void *q, const void *k, const void *v,
+                               const float *alpha, const float *beta_k, const float *beta_v, const float *s,
+                               const float *S0, const void *dout, const float *dS_T, float *dq, float *dk,
+                               float *dv, float *dalpha, float *dbeta_k, float *dbeta_v, float *ds, float *dS0,
+                               void *workspace, size_t workspace_bytes, void *stream) {
   dr_status st = check_common(p, false);
   if (st != DR_OK) return st;
+  if (variant < kBwdDefault || variant > kBwdChunk) return DR_ERR_UNSUPPORTED;
+  if (variant == kBwdChunk && !bwd_chunk_shape(p)) return DR_ERR_UNSUPPORTED;
   st = check_pointers(p, q, k, v, alpha, beta_k, beta_v, dout);
   if (st != DR_OK) return st;
   const bool need = p->T > 0;
@@ -391,7 +455,10 @@ dr_status dr_backward(const dr_problem *p, const void *q, const void *k, const v
                                : cudaMemsetAsync(dS0, 0, state_bytes, cs);
     return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
   }
-  if (!workspace || workspace_bytes < bwd_workspace_bytes(p)) return DR_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < bwd_variant_workspace_bytes(p, variant)) return DR_ERR_WORKSPACE;
+  if (resolve_bwd_variant(p, variant) == kBwdChunk)
+    return bwd_chunk_launch(p, q, k, v, alpha, beta_k, beta_v, s, S0, dout, dS_T, dq, dk, dv, dalpha, dbeta_k,
+                            dbeta_v, ds, dS0, workspace, cs);
   float *ws = static_cast<float *>(workspace);
   {  // the per-key-channel gradients are sums over value-column slices, accumulated in place
     const size_t tok = static_cast<size_t>(p->B) * p->T * p->H;
@@ -409,6 +476,15 @@ dr_status dr_backward(const dr_problem *p, const void *q, const void *k, const v
                    ws + static_cast<size_t>(p->B) * p->H * nck * p->dk * p->dv};
   if (p->io_dtype == DR_F32) return bwd_dispatch<float>(p, bp, cs);
   return bwd_dispatch<__nv_bfloat16>(p, bp, cs);
+}
+
+dr_status dr_backward(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
+                      const float *beta_k, const float *beta_v, const float *s, const float *S0, const void *dout,
+                      const float *dS_T, float *dq, float *dk, float *dv, float *dalpha, float *dbeta_k,
+                      float *dbeta_v, float *ds, float *dS0, void *workspace, size_t workspace_bytes,
+                      void *stream) {
+  return backward_impl(kBwdDefault, p, q, k, v, alpha, beta_k, beta_v, s, S0, dout, dS_T, dq, dk, dv, dalpha,
+                       dbeta_k, dbeta_v, ds, dS0, workspace, workspace_bytes, stream);
 }
 
 int dr_version(void) { return 100; }
@@ -563,6 +639,21 @@ int dr_diag_decode_step_variant(int variant, const dr_problem *p, const void *q,
                                 const float *alpha, const float *beta_k, const float *beta_v, const float *s,
                                 float *S, void *o, void *stream) {
   return decode_step_impl(p, q, k, v, alpha, beta_k, beta_v, s, S, o, stream, variant);
+}
+
+size_t dr_diag_backward_workspace(int variant, const dr_problem *p) {
+  if (check_common(p, false) != DR_OK || variant < kBwdDefault || variant > kBwdChunk) return 0;
+  if (variant == kBwdChunk && !bwd_chunk_shape(p)) return 0;
+  return bwd_variant_workspace_bytes(p, variant);
+}
+
+int dr_diag_backward_variant(int variant, const dr_problem *p, const void *q, const void *k, const void *v,
+                             const float *alpha, const float *beta_k, const float *beta_v, const float *s,
+                             const float *S0, const void *dout, const float *dS_T, float *dq, float *dk, float *dv,
+                             float *dalpha, float *dbeta_k, float *dbeta_v, float *ds, float *dS0, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+  return backward_impl(variant, p, q, k, v, alpha, beta_k, beta_v, s, S0, dout, dS_T, dq, dk, dv, dalpha, dbeta_k,
+                       dbeta_v, ds, dS0, workspace, workspace_bytes, stream);
 }
 
 int dr_diag_umma_selftest(int N, int K, int a_mn, int b_mn, int bf16, const void *A, const void *B, float *D,
