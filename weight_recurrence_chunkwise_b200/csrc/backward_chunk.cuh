@@ -40,16 +40,16 @@ constexpr uint32_t SX = 0;                        // [Bh; Qh]   128 x 128 (raw k
 constexpr uint32_t SX_CB = 128 * 128;
 constexpr uint32_t SAC = 2 * SX_CB;               // Ac         64 x 128
 constexpr uint32_t SAC_CB = 64 * 128;
-constexpr uint32_t STP = SAC + 2 * SAC_CB;        // [A -> T; T^T scratch -> P]  128 x 64
+constexpr uint32_t STP = SAC + 2 * SAC_CB;        // [A -> T; T^T scratch -> P]  128 x 64; raw q at the end
 constexpr uint32_t SSS = STP + 128 * 128;         // S (fp16)   128 (dk) x 128 (dv)
-constexpr uint32_t SWY = SSS + 2 * 128 * 128;     // raw v -> W -> Y -> dU   64 x 128
+constexpr uint32_t SWY = SSS + 2 * 128 * 128;     // W -> Y -> dU   64 x 128; raw k at the end
 constexpr uint32_t SWY_CB = 64 * 128;
 constexpr uint32_t SUU = SWY + 2 * SWY_CB;        // U          64 x 128
 constexpr uint32_t SDM = SUU + 2 * SWY_CB;        // dM         128 x 128 (K1's gate products before)
 constexpr uint32_t SDO = SDM + 2 * 128 * 128;     // [dO; -dV]  128 x 128
-constexpr uint32_t SDPA = SDO + 2 * 128 * 128;    // [dP; dA]   128 x 64
+constexpr uint32_t SDPA = SDO + 2 * 128 * 128;    // raw v (64 x 128), then [dP; dA]   128 x 64
 constexpr uint32_t SGC = SDPA + 128 * 128;        // gamma_C, 128 fp32
-constexpr uint32_t SROW = SGC + 512;              // scalar gates: gamma_r, 1/gamma_r, sqrt(beta_r), 64 each
+constexpr uint32_t SROW = SGC + 512;              // scalar gates: gamma_r, 1/gamma_r, sqrt(beta_r), alpha_r
 constexpr uint32_t SRT = SROW + 1024;             // last-row term partials, [2][128] fp32
 constexpr uint32_t SXC = SRT + 1024;              // per-channel exchange between the row halves, [2][128]
 constexpr uint32_t SRED = SXC + 1024;             // per-row sums over channels: [64 rows][4 warps][2] fp32
@@ -64,6 +64,29 @@ constexpr uint32_t COL_BS = 64;    // [Bh S | .] (128); later dU, then [dQh^T | 
 constexpr uint32_t COL_U = 192;    // [U | .] (128); later dV, then dAc^T (64)
 constexpr uint32_t COL_AU = 320;   // Ac^T U (128); later the state gradient's step
 constexpr uint32_t TMEM_COLS = 512;
+
+// Sums of v[k] over the 32 lanes of a warp for k = 0 .. N-1 (N = 8 or 32); lane l returns the sum of entry
+// l % N.  Butterfly steps over the lane bits above log2 N add whole arrays; each later step on lane bit b
+// keeps the half of the entries whose index bit b equals the lane's bit and adds the partner's copy of
+// it, so 31 shuffles serve 32 entries.
+template <int N>
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[N], int lane) {
+#pragma unroll
+  for (int off = 16; off >= N; off >>= 1)
+#pragma unroll
+    for (int k = 0; k < N; ++k) v[k] += __shfl_xor_sync(0xffffffffu, v[k], off);
+#pragma unroll
+  for (int off = N / 2; off >= 1; off >>= 1) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int k = 0; k < off; ++k) {
+      const float send = up ? v[k] : v[k + off];
+      const float keep = up ? v[k + off] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
+}
 
 struct BwdChunkParams {
   int T, H, nchunks;
@@ -96,6 +119,19 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int h = blockIdx.x, b = blockIdx.y, H = p.H, T = p.T, NC = p.nchunks;
   const size_t head = static_cast<size_t>(b) * H + h;
   const bool sym_write = p.beta_v_mode == MODE_ABSENT;  // w = sqrt(beta_k) (.) v
+  // the kernel's global inputs and outputs never overlap
+  const float *__restrict__ g_alpha = p.alpha;
+  const float *__restrict__ g_beta_k = p.beta_k;
+  const float *__restrict__ g_beta_v = p.beta_v;
+  const float *__restrict__ g_s = p.s;
+  const float *__restrict__ g_states = p.states;
+  float *__restrict__ g_dq = p.dq;
+  float *__restrict__ g_dk = p.dk;
+  float *__restrict__ g_dv = p.dv;
+  float *__restrict__ g_dalpha = p.dalpha;
+  float *__restrict__ g_dbeta_k = p.dbeta_k;
+  float *__restrict__ g_dbeta_v = p.dbeta_v;
+  float *__restrict__ g_ds = p.ds;
 
   uint8_t *X = sm + SX, *tAC = sm + SAC, *tTP = sm + STP, *tSS = sm + SSS, *tWY = sm + SWY, *tUU = sm + SUU;
   uint8_t *tDM = sm + SDM, *tDO = sm + SDO, *tDPA = sm + SDPA;
@@ -136,6 +172,13 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (fail && tid == 0) raise_status(p.status, STATUS_TIMEOUT);
     return !fail;
   };
+  auto wait_ld = [&]() -> bool {
+    const bool w = mbar_wait(&bar_ld, ph_ld & 1u, kWaitLimitNs);
+    ph_ld++;
+    const bool fail = bar_or(1, NT, !w);
+    if (fail && tid == 0) raise_status(p.status, STATUS_TIMEOUT);
+    return !fail;
+  };
   // single-thread MMA issue: nk K-steps of 16 into column `col`; desc(kk) give the operands
   auto issue = [&](uint32_t col, int nk, uint32_t idesc, bool acc, auto adesc, auto bdesc) {
     for (int kk = 0; kk < nk; ++kk) umma_f16(tmem + col, adesc(kk), bdesc(kk), idesc, (acc || kk > 0) ? 1u : 0u);
@@ -172,6 +215,24 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int j = 0; j < 64; j += 16) tc::st_h16x16(tile, row, col0 + j, R, v + j);
   };
 
+  // write scale of value columns col .. col + 3 of chunk row r (token index th): beta_v, or sqrt(beta_k)
+  // when the write is symmetric (dk = dv)
+  auto wscale4 = [&](int r, size_t th, int col) -> float4 {
+    if (p.beta_v_mode == MODE_CHANNEL) return __ldg(reinterpret_cast<const float4 *>(g_beta_v + th * DV + col));
+    if (p.beta_v_mode == MODE_SCALAR) {
+      const float y = __ldg(g_beta_v + th);
+      return make_float4(y, y, y, y);
+    }
+    if (p.beta_k_mode == MODE_CHANNEL) {
+      const float4 y = __ldg(reinterpret_cast<const float4 *>(g_beta_k + th * DK + col));
+      return make_float4(tc::sqrt_fast(y.x), tc::sqrt_fast(y.y), tc::sqrt_fast(y.z), tc::sqrt_fast(y.w));
+    }
+    float y;
+    if constexpr (kChanGates) y = tc::sqrt_fast(__ldg(g_beta_k + th));
+    else y = sRow[128 + r];  // the scan's sqrt(beta_k) of the row (0 past the end of the sequence)
+    return make_float4(y, y, y, y);
+  };
+
 #pragma unroll 1
   for (int c = NC - 1; c >= 0 && ok; --c) {
     const int t0 = c * C, L = min(C, T - t0);
@@ -184,8 +245,8 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tma_load_4d(X + SX_CB + 64 * 128, &tm_q, &bar_ld, 64, h, t0, b);
       tma_load_4d(X, &tm_k, &bar_ld, 0, h, t0, b);
       tma_load_4d(X + SX_CB, &tm_k, &bar_ld, 64, h, t0, b);
-      tma_load_4d(tWY, &tm_v, &bar_ld, 0, h, t0, b);
-      tma_load_4d(tWY + SWY_CB, &tm_v, &bar_ld, 64, h, t0, b);
+      tma_load_4d(tDPA, &tm_v, &bar_ld, 0, h, t0, b);
+      tma_load_4d(tDPA + 64 * 128, &tm_v, &bar_ld, 64, h, t0, b);
       tma_load_4d(tDO, &tm_do, &bar_ld, 0, h, t0, b);
       tma_load_4d(tDO + 128 * 128, &tm_do, &bar_ld, 64, h, t0, b);
       if (c > 0) {
@@ -200,9 +261,13 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // S of this chunk: fp16 operand tile, and the state part of the last-row term sum_v dS S
     float rt = 0.f;
     {
-      const float *src = p.states + (head * NC + c) * DK * DV + static_cast<size_t>(srow) * DV + half * 64;
-      if (c > 0) {  // the previous chunk's state into L2 (two 128-byte lines of my row half... all four)
-        const float *nx = p.states + (head * NC + c - 1) * DK * DV + static_cast<size_t>(srow) * DV + half * 64;
+      const float4 *src =
+          reinterpret_cast<const float4 *>(g_states + (head * NC + c) * DK * DV + static_cast<size_t>(srow) * DV + half * 64);
+      float4 sv[16];  // all of my 64 values in flight at once
+#pragma unroll
+      for (int e = 0; e < 16; ++e) sv[e] = __ldg(src + e);
+      if (c > 0) {  // the previous chunk's state into L2: my row half is two 128-byte lines
+        const float *nx = g_states + (head * NC + c - 1) * DK * DV + static_cast<size_t>(srow) * DV + half * 64;
         asm volatile("prefetch.global.L2 [%0];" ::"l"(nx));
         asm volatile("prefetch.global.L2 [%0];" ::"l"(nx + 32));
       }
@@ -210,12 +275,11 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int j = 0; j < 64; j += 16) {
         float x[16];
 #pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          const float4 y = __ldg(reinterpret_cast<const float4 *>(src + j + e));
-          x[e] = y.x;
-          x[e + 1] = y.y;
-          x[e + 2] = y.z;
-          x[e + 3] = y.w;
+        for (int e = 0; e < 4; ++e) {
+          x[4 * e] = sv[j / 4 + e].x;
+          x[4 * e + 1] = sv[j / 4 + e].y;
+          x[4 * e + 2] = sv[j / 4 + e].z;
+          x[4 * e + 3] = sv[j / 4 + e].w;
         }
 #pragma unroll
         for (int e = 0; e < 16; ++e) rt += dS[j + e] * x[e];
@@ -274,21 +338,15 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       sRow[64 + 2 * lane + 1] = __fdividef(1.f, g1);
       sRow[128 + 2 * lane] = tc::sqrt_fast(be[0]);
       sRow[128 + 2 * lane + 1] = tc::sqrt_fast(be[1]);
+      sRow[192 + 2 * lane] = al[0];
+      sRow[192 + 2 * lane + 1] = al[1];
       const float gC = __shfl_sync(0xffffffffu, incl, 31);
 #pragma unroll
       for (int e = 0; e < 4; ++e) sGC[4 * lane + e] = gC;
       if (lane == 0 && !(gC >= kMinChunkDecayF16)) raise_status(p.status, STATUS_RANGE);
     }
     // wait for the tiles
-    {
-      const bool w = mbar_wait(&bar_ld, ph_ld & 1u, kWaitLimitNs);
-      ph_ld++;
-      if (bar_or(1, NT, !w)) {
-        if (tid == 0) raise_status(p.status, STATUS_TIMEOUT);
-        ok = false;
-        break;
-      }
-    }
+    if (!wait_ld()) { ok = false; break; }
 
     // ------------------------------------------------------------------ K1: Qh, Bh, Ac; write vectors; dO -> fp16
     float amax = 0.f;
@@ -319,7 +377,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       uint8_t *pQ = X + blk * SX_CB + (64 + rg * 8) * 128 + inb;
       uint8_t *pB = X + blk * SX_CB + (rg * 8) * 128 + inb;
       uint8_t *pA = tAC + blk * SAC_CB + (rg * 8) * 128 + inb;
-#pragma unroll 2
+#pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
         const uint32_t sw = ((grp ^ static_cast<uint32_t>(jj)) << 4) + jj * 128;
         const uint2 kraw = *reinterpret_cast<const uint2 *>(pB + sw), qraw = *reinterpret_cast<const uint2 *>(pQ + sw);
@@ -390,49 +448,36 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
     }
     if (!(amax < kF16Max)) raise_status(p.status, STATUS_RANGE);
-    // write vectors W = wsc (.) v in place of raw v, and dO as fp16 in place: thread row tid >> 2,
-    // 8-column groups 4 (tid & 3) .. 4 (tid & 3) + 3 of 16
+    // write vectors W = wsc (.) v (raw v waits in the dP/dA tile), and dO as fp16 in place: thread row
+    // tid >> 2, 8-column groups 4 (tid & 3) .. 4 (tid & 3) + 3 of 16
     {
       const int r = tid >> 2;
+      const bool valid = r < L;
       const size_t th = (tok0 + min(r, L - 1)) * H + h;
-#pragma unroll 1
+      float4 wq[8];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int col = 8 * (4 * (tid & 3) + g);
+        wq[2 * g] = wscale4(r, th, col);
+        wq[2 * g + 1] = wscale4(r, th, col + 4);
+      }
+#pragma unroll
       for (int g = 0; g < 4; ++g) {
         const int c8 = 4 * (tid & 3) + g;  // 8-column group (0..15)
-        float wsc[8];
-        if (p.beta_v_mode == MODE_CHANNEL) {
-          const float4 *src = reinterpret_cast<const float4 *>(p.beta_v + th * DV + c8 * 8);
-          const float4 lo = __ldg(src), hi = __ldg(src + 1);
-          wsc[0] = lo.x; wsc[1] = lo.y; wsc[2] = lo.z; wsc[3] = lo.w;
-          wsc[4] = hi.x; wsc[5] = hi.y; wsc[6] = hi.z; wsc[7] = hi.w;
-        } else if (p.beta_v_mode == MODE_SCALAR) {
-          const float x = __ldg(p.beta_v + th);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) wsc[e] = x;
-        } else if (p.beta_k_mode == MODE_CHANNEL) {
-          const float4 *src = reinterpret_cast<const float4 *>(p.beta_k + th * DK + c8 * 8);
-          const float4 lo = __ldg(src), hi = __ldg(src + 1);
-          wsc[0] = tc::sqrt_fast(lo.x); wsc[1] = tc::sqrt_fast(lo.y); wsc[2] = tc::sqrt_fast(lo.z);
-          wsc[3] = tc::sqrt_fast(lo.w); wsc[4] = tc::sqrt_fast(hi.x); wsc[5] = tc::sqrt_fast(hi.y);
-          wsc[6] = tc::sqrt_fast(hi.z); wsc[7] = tc::sqrt_fast(hi.w);
-        } else {
-          const float x = tc::sqrt_fast(__ldg(p.beta_k + th));
-#pragma unroll
-          for (int e = 0; e < 8; ++e) wsc[e] = x;
-        }
-        uint4 *pv = reinterpret_cast<uint4 *>(tWY + sw128_off16(r, c8, 64));
+        const float wsc[8] = {wq[2 * g].x,     wq[2 * g].y,     wq[2 * g].z,     wq[2 * g].w,
+                              wq[2 * g + 1].x, wq[2 * g + 1].y, wq[2 * g + 1].z, wq[2 * g + 1].w};
         uint4 *pd = reinterpret_cast<uint4 *>(tDO + sw128_off16(r, c8, 128));
-        const uint4 vraw = *pv, draw = *pd;
+        const uint4 vraw = *reinterpret_cast<const uint4 *>(tDPA + sw128_off16(r, c8, 64)), draw = *pd;
         const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vraw);
         const __nv_bfloat162 *d2 = reinterpret_cast<const __nv_bfloat162 *>(&draw);
         uint32_t ow[4], od[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 vf = __bfloat1622float2(v2[e]), df = __bfloat1622float2(d2[e]);
-          const bool valid = r < L;
           ow[e] = pack_f16x2(valid ? wsc[2 * e] * vf.x : 0.f, valid ? wsc[2 * e + 1] * vf.y : 0.f);
           od[e] = pack_f16x2(valid ? df.x : 0.f, valid ? df.y : 0.f);
         }
-        *pv = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        *reinterpret_cast<uint4 *>(tWY + sw128_off16(r, c8, 64)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
         *pd = make_uint4(od[0], od[1], od[2], od[3]);
       }
     }
@@ -570,13 +615,14 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     if (!wait_mma()) { ok = false; break; }
     // last-row term: sum_v dS (S + Ac^T U), per key row; the two value halves meet in shared memory
-#pragma unroll 1
-    for (int j = 0; j < 64; j += 16) {
-      float x[16];
-      tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), x);
+    {
+      float x[64];
+#pragma unroll
+      for (int j = 0; j < 64; j += 16)
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), *reinterpret_cast<float(*)[16]>(x + j));
       tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) rt += dS[j + e] * x[e];
+      for (int e = 0; e < 64; ++e) rt += dS[e] * x[e];
     }
     sRT[half * 128 + srow] = rt;
     fence_async_smem();
@@ -624,9 +670,13 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (!wait_mma()) { ok = false; break; }
     if (quarter < 2) {
       const int r = srow;
+      const bool valid = r < L;
       const size_t th = (tok0 + min(r, L - 1)) * H + h;
+      float4 wq[16];  // the write scales of my 64 value columns, in flight before the TMEM reads
+#pragma unroll
+      for (int e = 0; e < 16; ++e) wq[e] = wscale4(r, th, half * 64 + 4 * e);
       float rsum = 0.f;  // sum over my value columns of v dV (scalar write strength)
-#pragma unroll 1
+#pragma unroll
       for (int j = 0; j < 64; j += 16) {
         float x[16];
         tmem_ld16(tmem_addr(tmem, quarter * 32, COL_U + half * 64 + j), x);
@@ -636,13 +686,12 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
         for (int e = 0; e < 16; ++e) nd[e] = -x[e];
         tc::st_h16x16(tDO, 64 + r, v0, 128, nd);
-        if (r < L) {
-          // raw v and the write scale of these 16 columns
+        if (valid) {
+          // raw v of these 16 columns (from the dP/dA tile) and their write scales
           float vf[16], wsc[16];
-          const uint4 *vsrc = reinterpret_cast<const uint4 *>(p.v + th * DV + v0);
 #pragma unroll
           for (int g = 0; g < 2; ++g) {
-            const uint4 raw = __ldg(vsrc + g);
+            const uint4 raw = *reinterpret_cast<const uint4 *>(tDPA + sw128_off16(r, v0 / 8 + g, 64));
             const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -652,40 +701,28 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
           }
 #pragma unroll
-          for (int e = 0; e < 16; e += 4) {
-            float4 wq;
-            if (p.beta_v_mode == MODE_CHANNEL) {
-              wq = __ldg(reinterpret_cast<const float4 *>(p.beta_v + th * DV + v0 + e));
-            } else if (p.beta_v_mode == MODE_SCALAR) {
-              const float y = __ldg(p.beta_v + th);
-              wq = make_float4(y, y, y, y);
-            } else if (p.beta_k_mode == MODE_CHANNEL) {
-              const float4 y = __ldg(reinterpret_cast<const float4 *>(p.beta_k + th * DK + v0 + e));
-              wq = make_float4(tc::sqrt_fast(y.x), tc::sqrt_fast(y.y), tc::sqrt_fast(y.z), tc::sqrt_fast(y.w));
-            } else {
-              const float y = tc::sqrt_fast(__ldg(p.beta_k + th));
-              wq = make_float4(y, y, y, y);
-            }
-            wsc[e] = wq.x; wsc[e + 1] = wq.y; wsc[e + 2] = wq.z; wsc[e + 3] = wq.w;
+          for (int e = 0; e < 4; ++e) {
+            const float4 w = wq[j / 4 + e];
+            wsc[4 * e] = w.x; wsc[4 * e + 1] = w.y; wsc[4 * e + 2] = w.z; wsc[4 * e + 3] = w.w;
           }
-          float *dvo = p.dv + th * DV + v0;
+          float *dvo = g_dv + th * DV + v0;
 #pragma unroll
           for (int e = 0; e < 16; e += 4)
             *reinterpret_cast<float4 *>(dvo + e) =
                 make_float4(wsc[e] * x[e], wsc[e + 1] * x[e + 1], wsc[e + 2] * x[e + 2], wsc[e + 3] * x[e + 3]);
           // gradient of the write scale: v (.) dV per column
           if (p.beta_v_mode == MODE_CHANNEL) {
-            float *o = p.dbeta_v + th * DV + v0;
+            float *o = g_dbeta_v + th * DV + v0;
 #pragma unroll
             for (int e = 0; e < 16; e += 4)
               *reinterpret_cast<float4 *>(o + e) =
                   make_float4(vf[e] * x[e], vf[e + 1] * x[e + 1], vf[e + 2] * x[e + 2], vf[e + 3] * x[e + 3]);
-          } else if (p.beta_v_mode == MODE_SCALAR) {
+          } else if (p.beta_v_mode == MODE_SCALAR || p.beta_k_mode != MODE_CHANNEL) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) rsum += vf[e] * x[e];
-          } else if (p.beta_k_mode == MODE_CHANNEL) {
+          } else {
             // symmetric channel write: d beta_k += 0.5 v dV / sqrt(beta_k), stored now, added to below
-            float *o = p.dbeta_k + th * DK + v0;
+            float *o = g_dbeta_k + th * DK + v0;
 #pragma unroll
             for (int e = 0; e < 16; e += 4) {
               float4 y;
@@ -695,9 +732,6 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               y.w = wsc[e + 3] > 0.f ? 0.5f * vf[e + 3] * x[e + 3] / wsc[e + 3] : 0.f;
               *reinterpret_cast<float4 *>(o + e) = y;
             }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) rsum += vf[e] * x[e];
           }
         }
       }
@@ -710,7 +744,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const int r = tid;
       const size_t th = (tok0 + r) * H + h;
       const float rs = sRV[2 * r] + sRV[2 * r + 1];
-      if (p.beta_v_mode == MODE_SCALAR) p.dbeta_v[th] = rs;
+      if (p.beta_v_mode == MODE_SCALAR) g_dbeta_v[th] = rs;
       else if (p.beta_k_mode == MODE_SCALAR) sRV[2 * r] = rs;  // symmetric scalar write: folded in below
     }
 
@@ -729,16 +763,15 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (!wait_mma()) { ok = false; break; }
     {
       float mx = 0.f;
-#pragma unroll 1
-      for (int j = 0; j < 64; j += 16) {
-        float x[16];
-        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), x);
-        tmem_ld_wait();
+      float x[64];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          dS[j + e] = gci * dS[j + e] + x[e];
-          mx = fmaxf(mx, fabsf(dS[j + e]));
-        }
+      for (int j = 0; j < 64; j += 16)
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), *reinterpret_cast<float(*)[16]>(x + j));
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        dS[e] = gci * dS[e] + x[e];
+        mx = fmaxf(mx, fabsf(dS[e]));
       }
       if (!(mx < kF16Max)) raise_status(p.status, STATUS_RANGE);
     }
@@ -772,124 +805,241 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         issue(COL_U, C / 16, id, true, mnmaj(sb + SX + 64 * 128, 128), mnmaj(sb + SDPA, 128));
         issue(COL_U, DV / 16, idesc_f16_f32(128, 64, false, false), true, kmaj(sb + SDM, 128), kmaj(sb + SUU, 64));
         umma_commit(&bar_mma);
+        // the chunk's raw q and k for the per-channel stage, into the tiles T and dU have left
+        mbar_arrive_expect_tx(&bar_ld, 4 * 64 * 128);
+        tma_load_4d(tTP, &tm_q, &bar_ld, 0, h, t0, b);
+        tma_load_4d(tTP + 64 * 128, &tm_q, &bar_ld, 64, h, t0, b);
+        tma_load_4d(tWY, &tm_k, &bar_ld, 0, h, t0, b);
+        tma_load_4d(tWY + SWY_CB, &tm_k, &bar_ld, 64, h, t0, b);
       }
       __syncwarp();
     }
     if (!wait_mma()) { ok = false; break; }
 
     // ------------------------------------------------------------------ per key channel: gate gradients and outputs
-    // thread: channel i = srow, rows 32 half .. 32 half + 31 of the chunk
+    // thread: key channel i = srow, rows 32 half .. 32 half + 31 of the chunk.  The state gradient waits in
+    // TMEM meanwhile (the state step's columns are free); q and k are read raw from the tiles just loaded.
     {
       const int i = srow, r0 = 32 * half;
+#pragma unroll
+      for (int j = 0; j < 64; j += 16)
+        tmem_st16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), *reinterpret_cast<const float(*)[16]>(dS + j));
       const float rowterm = sRT[i] + sRT[128 + i];
-      // gamma of my rows: forward products (the lower half passes its product to the upper half)
-      float al[32], gam[32];
-      float prod = 1.f;
+      auto raw_at = [&](const uint8_t *tile, int r) {  // bf16 (r, channel i) of a 64-row swizzled tile
+        return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + sw128_off(r, i, 64)));
+      };
+      if (!wait_ld()) { ok = false; break; }
+      if constexpr (kChanGates) {
+        // gamma of my rows: forward products (the lower half passes its product to the upper half)
+        float al[32], gam[32];
+        float prod = 1.f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int r = r0 + j;
-        const size_t th = (tok0 + min(r, L - 1)) * H + h;
-        float a = 1.f;
-        if (r < L) {
-          if (p.alpha_mode == MODE_CHANNEL) a = __ldg(p.alpha + th * DK + i);
-          else if (p.alpha_mode == MODE_SCALAR) a = __ldg(p.alpha + th);
-        }
-        al[j] = a;
-        prod *= a;
-      }
-      if (half == 0) sXC[i] = prod;
-      __syncthreads();
-      float g = half == 0 ? 1.f : sXC[i];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        g *= al[j];
-        gam[j] = g;
-      }
-      // reverse over my rows: dgamma, the local suffix sums of dgamma gamma, and the outputs
-      float suf[32];
-      float acc = 0.f;
-#pragma unroll
-      for (int jb = 16; jb >= 0; jb -= 16) {
-        float dq[16], db[16], da[16];
-        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_BS + r0 + jb), dq);
-        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_BS + 64 + r0 + jb), db);
-        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_U + r0 + jb), da);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 15; e >= 0; --e) {
-          const int j = jb + e, r = r0 + j;
+        for (int j = 0; j < 32; ++j) {
+          const int r = r0 + j;
           const size_t th = (tok0 + min(r, L - 1)) * H + h;
-          const float gm = gam[j];
-          const float qv = __bfloat162float(p.q[th * DK + i]);
-          const float kv = __bfloat162float(p.k[th * DK + i]);
-          float bet = 0.f;
-          if (r < L) bet = p.beta_k_mode == MODE_CHANNEL ? __ldg(p.beta_k + th * DK + i) : __ldg(p.beta_k + th);
-          const float sbt = tc::sqrt_fast(bet);
-          const float scv = kScaled ? (r < L ? __ldg(p.s + th * DK + i) : 0.f) : 1.f;
-          const float bv = sbt * kv, av = scv * bv;
-          const float ginv = __fdividef(1.f, gm);
-          float dg = qv * dq[e] + bv * db[e] - av * ginv * da[e] * ginv;
-          if (r == C - 1) dg += rowterm;
-          acc += dg * gm;
-          suf[j] = acc;
+          float a = 1.f;
           if (r < L) {
-            const float dqv = gm * dq[e];
-            const float dbv = gm * db[e], dav = da[e] * ginv;
-            const float dbt = dbv + scv * dav;  // through b = sqrt(beta) k and a = s b
-            p.dq[th * DK + i] = dqv;
-            p.dk[th * DK + i] = sbt * dbt;
-            if constexpr (kScaled) p.ds[th * DK + i] = bv * dav;
-            const float dsb = kv * dbt;  // d / d sqrt(beta_k)
-            const float dbk = sbt > 0.f ? 0.5f * dsb / sbt : 0.f;
-            if (p.beta_k_mode == MODE_CHANNEL) {
-              const float prev = (sym_write) ? p.dbeta_k[th * DK + i] : 0.f;
-              p.dbeta_k[th * DK + i] = prev + dbk;
-            } else {
-              // scalar: summed over channels below
-              float v = dbk;
+            if (p.alpha_mode == MODE_CHANNEL) a = __ldg(g_alpha + th * DK + i);
+            else if (p.alpha_mode == MODE_SCALAR) a = __ldg(g_alpha + th);
+          }
+          al[j] = a;
+          prod *= a;
+        }
+        if (half == 0) sXC[i] = prod;
+        __syncthreads();
+        {
+          float g = half == 0 ? 1.f : sXC[i];
 #pragma unroll
-              for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-              if (lane == 0) sRed[(r * 4 + quarter) * 2 + 0] = v;
+          for (int j = 0; j < 32; ++j) {
+            g *= al[j];
+            gam[j] = g;
+          }
+        }
+        // reverse over my rows, in blocks of 8 whose gate loads run one block ahead: dgamma, the local
+        // suffix sums of dgamma gamma, and the outputs
+        float *sSuf = reinterpret_cast<float *>(tSS);  // the lower half's suffix sums, [32][256] (S is spent)
+        float acc = 0.f;
+        float cb[8], cs[8], cp[8];  // beta_k, s and the stored write-side d beta_k of the block's rows
+        auto load_blk = [&](int jb, float (&bk)[8], float (&sc)[8], float (&pv)[8]) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int r = r0 + jb + e;
+            const size_t th = (tok0 + min(r, L - 1)) * H + h;
+            bk[e] = p.beta_k_mode == MODE_CHANNEL ? __ldg(g_beta_k + th * DK + i) : __ldg(g_beta_k + th);
+            sc[e] = kScaled ? __ldg(g_s + th * DK + i) : 1.f;
+            pv[e] = (sym_write && p.beta_k_mode == MODE_CHANNEL) ? g_dbeta_k[th * DK + i] : 0.f;
+          }
+        };
+        load_blk(24, cb, cs, cp);
+#pragma unroll
+        for (int blk = 3; blk >= 0; --blk) {
+          const int jb = 8 * blk;
+          float nb[8], ns[8], np[8];
+          if (blk > 0) load_blk(jb - 8, nb, ns, np);
+          float dq[8], db[8], da[8];
+          tmem_ld8(tmem_addr(tmem, quarter * 32, COL_BS + r0 + jb), dq);
+          tmem_ld8(tmem_addr(tmem, quarter * 32, COL_BS + 64 + r0 + jb), db);
+          tmem_ld8(tmem_addr(tmem, quarter * 32, COL_U + r0 + jb), da);
+          tmem_ld_wait();
+          float xg[8], xb[8];  // dgamma gamma and d beta_k per row, for gates that are scalar per row
+#pragma unroll
+          for (int e = 7; e >= 0; --e) {
+            const int j = jb + e, r = r0 + j;
+            const bool valid = r < L;
+            const float gm = gam[j], ginv = __fdividef(1.f, gm);
+            const float qv = raw_at(tTP, r), kv = raw_at(tWY, r);
+            const float sbt = valid ? tc::sqrt_fast(cb[e]) : 0.f;
+            const float scv = kScaled ? (valid ? cs[e] : 0.f) : 1.f;
+            const float bv = sbt * kv, av = scv * bv, dav = da[e] * ginv;
+            float dg = qv * dq[e] + bv * db[e] - av * dav * ginv;
+            if (r == C - 1) dg += rowterm;
+            acc += dg * gm;
+            if (half == 0) sSuf[j * NT + tid] = acc;
+            xg[e] = dg * gm;
+            const float dbt = gm * db[e] + scv * dav;  // through b = sqrt(beta) k and a = s b
+            const float dbk = sbt > 0.f ? 0.5f * kv * dbt / sbt : 0.f;
+            xb[e] = dbk;
+            if (valid) {
+              const size_t o = ((tok0 + r) * H + h) * DK + i;
+              g_dq[o] = gm * dq[e];
+              g_dk[o] = sbt * dbt;
+              if constexpr (kScaled) g_ds[o] = bv * dav;
+              if (p.beta_k_mode == MODE_CHANNEL) g_dbeta_k[o] = cp[e] + dbk;
+              if (p.alpha_mode == MODE_CHANNEL && half == 1) g_dalpha[o] = acc / al[j];
+            }
+          }
+          if (p.beta_k_mode != MODE_CHANNEL) {  // summed over channels: rows r0 + jb + (lane & 7)
+            const float v = warp_transpose_sum<8>(xb, lane);
+            if (lane < 8) sRed[((r0 + jb + lane) * 4 + quarter) * 2] = v;
+          }
+          if (p.alpha_mode == MODE_SCALAR) {
+            const float v = warp_transpose_sum<8>(xg, lane);
+            if (lane < 8) sRed[((r0 + jb + lane) * 4 + quarter) * 2 + 1] = v;
+          }
+          if (blk > 0) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              cb[e] = nb[e];
+              cs[e] = ns[e];
+              cp[e] = np[e];
+            }
+          }
+        }
+        // the upper half's total flows into the lower half's suffix sums
+        if (half == 1) sXC[128 + i] = acc;
+        __syncthreads();
+        if (half == 0 && p.alpha_mode == MODE_CHANNEL) {
+          const float off = sXC[128 + i];
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < L) g_dalpha[((tok0 + j) * H + h) * DK + i] = (sSuf[j * NT + tid] + off) / al[j];
+        }
+      } else {
+        // gates scalar per row (the scan's gamma, 1/gamma, sqrt(beta_k) in shared memory); the per-row
+        // terms are summed over channels after the loop
+        float xg[32], xb[32];
+        float cs[8];
+        auto load_s = [&](int jb, float (&sc)[8]) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            sc[e] = kScaled ? __ldg(g_s + ((tok0 + min(r0 + jb + e, L - 1)) * H + h) * DK + i) : 1.f;
+        };
+        load_s(24, cs);
+#pragma unroll
+        for (int blk = 3; blk >= 0; --blk) {
+          const int jb = 8 * blk;
+          float ns[8];
+          if (blk > 0) load_s(jb - 8, ns);
+          float dq[8], db[8], da[8];
+          tmem_ld8(tmem_addr(tmem, quarter * 32, COL_BS + r0 + jb), dq);
+          tmem_ld8(tmem_addr(tmem, quarter * 32, COL_BS + 64 + r0 + jb), db);
+          tmem_ld8(tmem_addr(tmem, quarter * 32, COL_U + r0 + jb), da);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int j = jb + e, r = r0 + j;
+            const bool valid = r < L;
+            const float gm = sRow[r], ginv = sRow[64 + r], sbt = sRow[128 + r];
+            const float qv = raw_at(tTP, r), kv = raw_at(tWY, r);
+            const float scv = kScaled ? (valid ? cs[e] : 0.f) : 1.f;
+            const float bv = sbt * kv, av = scv * bv, dav = da[e] * ginv;
+            float dg = qv * dq[e] + bv * db[e] - av * dav * ginv;
+            if (r == C - 1) dg += rowterm;
+            xg[j] = dg * gm;
+            const float dbt = gm * db[e] + scv * dav;
+            xb[j] = sbt > 0.f ? 0.5f * kv * __fdividef(dbt, sbt) : 0.f;
+            if (valid) {
+              const size_t o = ((tok0 + r) * H + h) * DK + i;
+              g_dq[o] = gm * dq[e];
+              g_dk[o] = sbt * dbt;
+              if constexpr (kScaled) g_ds[o] = bv * dav;
+            }
+          }
+          if (blk > 0) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) cs[e] = ns[e];
+          }
+        }
+        // sums over my warp's 32 channels: lane l holds row r0 + l
+        const float sb = warp_transpose_sum<32>(xb, lane);
+        sRed[((r0 + lane) * 4 + quarter) * 2] = sb;
+        if (p.alpha_mode == MODE_SCALAR) {
+          const float sg = warp_transpose_sum<32>(xg, lane);
+          sRed[((r0 + lane) * 4 + quarter) * 2 + 1] = sg;
+        }
+      }
+      __syncthreads();
+      // scalar gates: per-row sums over the four channel quarters; the decay's gradient is then a suffix
+      // sum over the rows, divided by the row's alpha (warp 0: rows 2 lane, 2 lane + 1)
+      if (warp == 0 && (p.alpha_mode == MODE_SCALAR || p.beta_k_mode == MODE_SCALAR)) {
+        float gs[2], bs[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int r = 2 * lane + e;
+          gs[e] = sRed[(r * 4) * 2 + 1] + sRed[(r * 4 + 1) * 2 + 1] + sRed[(r * 4 + 2) * 2 + 1] + sRed[(r * 4 + 3) * 2 + 1];
+          bs[e] = sRed[(r * 4) * 2] + sRed[(r * 4 + 1) * 2] + sRed[(r * 4 + 2) * 2] + sRed[(r * 4 + 3) * 2];
+        }
+        if (p.alpha_mode == MODE_SCALAR) {
+          float sfx = gs[0] + gs[1];  // becomes the sum over rows >= 2 lane
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_down_sync(0xffffffffu, sfx, off);
+            if (lane + off < 32) sfx += y;
+          }
+          const float after = __shfl_down_sync(0xffffffffu, sfx, 1);
+          const float s1 = gs[1] + (lane < 31 ? after : 0.f), s0 = gs[0] + s1;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int r = 2 * lane + e;
+            if (r < L) {
+              const size_t th = (tok0 + r) * H + h;
+              const float a = kChanGates ? __ldg(g_alpha + th) : sRow[192 + r];
+              g_dalpha[th] = (e ? s1 : s0) / a;
+            }
+          }
+        }
+        if (p.beta_k_mode == MODE_SCALAR) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int r = 2 * lane + e;
+            if (r < L) {
+              const size_t th = (tok0 + r) * H + h;
+              float v = bs[e];
+              if (sym_write) {  // w = sqrt(beta_k) v as well: 0.5 / sqrt(beta_k) sum_v v dV
+                const float sbt = kChanGates ? tc::sqrt_fast(__ldg(g_beta_k + th)) : sRow[128 + r];
+                v += sbt > 0.f ? 0.5f * sRV[2 * r] / sbt : 0.f;
+              }
+              g_dbeta_k[th] = v;
             }
           }
         }
       }
-      // the upper half's total flows into the lower half's suffix sums
-      if (half == 1) sXC[128 + i] = acc;
-      __syncthreads();
-      const float off = half == 0 ? sXC[128 + i] : 0.f;
+      // the state gradient back into registers
+      tmem_st_wait();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int r = r0 + j;
-        if (r < L) {
-          const size_t th = (tok0 + r) * H + h;
-          const float da_ = (suf[j] + off) / al[j];
-          if (p.alpha_mode == MODE_CHANNEL) {
-            p.dalpha[th * DK + i] = da_;
-          } else if (p.alpha_mode == MODE_SCALAR) {
-            float v = da_;
-#pragma unroll
-            for (int o2 = 16; o2 > 0; o2 >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o2);
-            if (lane == 0) sRed[(r * 4 + quarter) * 2 + 1] = v;
-          }
-        }
-      }
-    }
-    __syncthreads();
-    if (tid < 64 && tid < L) {  // scalar gates: sums over the four channel quarters
-      const int r = tid;
-      const size_t th = (tok0 + r) * H + h;
-      if (p.alpha_mode == MODE_SCALAR)
-        p.dalpha[th] = sRed[(r * 4) * 2 + 1] + sRed[(r * 4 + 1) * 2 + 1] + sRed[(r * 4 + 2) * 2 + 1] +
-                       sRed[(r * 4 + 3) * 2 + 1];
-      if (p.beta_k_mode == MODE_SCALAR) {
-        float v = sRed[(r * 4) * 2] + sRed[(r * 4 + 1) * 2] + sRed[(r * 4 + 2) * 2] + sRed[(r * 4 + 3) * 2];
-        if (sym_write) {  // w = sqrt(beta_k) v as well: 0.5 / sqrt(beta_k) sum_v v dV
-          const float sbt = tc::sqrt_fast(__ldg(p.beta_k + th));
-          v += sbt > 0.f ? 0.5f * sRV[2 * r] / sbt : 0.f;
-        }
-        p.dbeta_k[th] = v;
-      }
+      for (int j = 0; j < 64; j += 16)
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), *reinterpret_cast<float(*)[16]>(dS + j));
+      tmem_ld_wait();
     }
     tc_fence_before();
     __syncthreads();
