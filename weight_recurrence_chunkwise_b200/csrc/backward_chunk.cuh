@@ -19,7 +19,7 @@
 // thread.
 //
 // One CTA of 256 threads per (b, h) walks its chunks from the last to the first; the fp32 gradient
-// of the state is carried in registers (thread: key row i, 64 value columns).  Every product uses
+// of the state is carried in TMEM (lane = key row i), where the step of every chunk accumulates onto it.  Every product uses
 // M = 128; where only 64 rows are meaningful, the other 64 rows read neighbouring tiles and are
 // ignored in TMEM.
 #pragma once
@@ -40,29 +40,33 @@ constexpr uint32_t SX = 0;                        // [Bh; Qh]   128 x 128 (raw k
 constexpr uint32_t SX_CB = 128 * 128;
 constexpr uint32_t SAC = 2 * SX_CB;               // Ac         64 x 128
 constexpr uint32_t SAC_CB = 64 * 128;
-constexpr uint32_t STP = SAC + 2 * SAC_CB;        // [A -> T; T^T scratch -> P]  128 x 64; raw q at the end
+constexpr uint32_t STP = SAC + 2 * SAC_CB;        // K1's gate products; [A -> T; T^T scratch -> P]  128 x 64; raw q
 constexpr uint32_t SSS = STP + 128 * 128;         // S (fp16)   128 (dk) x 128 (dv)
 constexpr uint32_t SWY = SSS + 2 * 128 * 128;     // W -> Y -> dU   64 x 128; raw k at the end
 constexpr uint32_t SWY_CB = 64 * 128;
 constexpr uint32_t SUU = SWY + 2 * SWY_CB;        // U          64 x 128
-constexpr uint32_t SDM = SUU + 2 * SWY_CB;        // dM         128 x 128 (K1's gate products before)
+constexpr uint32_t SDM = SUU + 2 * SWY_CB;        // dM         128 x 128
 constexpr uint32_t SDO = SDM + 2 * 128 * 128;     // [dO; -dV]  128 x 128
+// the chunk's fp32 state lands in [SWY, SDO) (free at the chunk's start): four 128-row boxes of 32 columns
+constexpr uint32_t SST = SWY;
+constexpr uint32_t SST_B = 128 * 128;
+static_assert(SST + 4 * SST_B == SDO, "state staging spans the write-vector, U and dM tiles");
 constexpr uint32_t SDPA = SDO + 2 * 128 * 128;    // raw v (64 x 128), then [dP; dA]   128 x 64
 constexpr uint32_t SGC = SDPA + 128 * 128;        // gamma_C, 128 fp32
 constexpr uint32_t SROW = SGC + 512;              // scalar gates: gamma_r, 1/gamma_r, sqrt(beta_r), alpha_r
 constexpr uint32_t SRT = SROW + 1024;             // last-row term partials, [2][128] fp32
 constexpr uint32_t SXC = SRT + 1024;              // per-channel exchange between the row halves, [2][128]
 constexpr uint32_t SRED = SXC + 1024;             // per-row sums over channels: [64 rows][4 warps][2] fp32
-constexpr uint32_t SRV = SRED + 64 * 4 * 2 * 4;   // per-row sums over value columns: [64 rows][2] fp32
-constexpr uint32_t SEND = SRV + 64 * 2 * 4;
+constexpr uint32_t SRV = SRED + 64 * 4 * 2 * 4;   // per-row sums over value columns: [64 rows][4 warps] fp32
+constexpr uint32_t SEND = SRV + 64 * 4 * 4;
 constexpr size_t SMEM_BYTES = SEND + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // TMEM columns
 constexpr uint32_t COL_D1 = 0;     // [A | P] raw (64); later [dP | dA] raw
-constexpr uint32_t COL_BS = 64;    // [Bh S | .] (128); later dU, then [dQh^T | dBh^T]
+constexpr uint32_t COL_BS = 64;    // [Bh S | .] (128); later Ac^T U, dU, then [dQh^T | dBh^T]
 constexpr uint32_t COL_U = 192;    // [U | .] (128); later dV, then dAc^T (64)
-constexpr uint32_t COL_AU = 320;   // Ac^T U (128); later the state gradient's step
+constexpr uint32_t COL_AU = 320;   // the state gradient (128), across chunks
 constexpr uint32_t TMEM_COLS = 512;
 
 // Sums of v[k] over the 32 lanes of a warp for k = 0 .. N-1 (N = 8 or 32); lane l returns the sum of entry
@@ -108,7 +112,7 @@ template <bool kChanGates, bool kScaled>
 __global__ void __launch_bounds__(NT, 1)
 chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                 const BwdChunkParams p) {
+                 const __grid_constant__ CUtensorMap tm_st, const BwdChunkParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_ld, bar_mma;
   __shared__ uint32_t tmem_base_sh;
@@ -124,7 +128,6 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const float *__restrict__ g_beta_k = p.beta_k;
   const float *__restrict__ g_beta_v = p.beta_v;
   const float *__restrict__ g_s = p.s;
-  const float *__restrict__ g_states = p.states;
   float *__restrict__ g_dq = p.dq;
   float *__restrict__ g_dk = p.dk;
   float *__restrict__ g_dv = p.dv;
@@ -154,6 +157,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_st);
   }
   tc_fence_before();
   __syncthreads();
@@ -196,17 +200,29 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   // the gradient of the state: row i = 32 quarter + lane, value columns 64 half .. 64 half + 63
   const int srow = quarter * 32 + lane;
-  float dS[64];
+  // Between chunks it lives in TMEM columns COL_AU .. COL_AU + 127 (lane = key row): the state step's
+  // product accumulates onto it there, and registers hold it only where a stage reads it.
+  auto ld_au = [&](float (&x)[64]) {  // my row half of the 128 columns at COL_AU
+#pragma unroll
+    for (int j = 0; j < 64; j += 16)
+      tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), *reinterpret_cast<float(*)[16]>(x + j));
+    tmem_ld_wait();
+  };
   {
+    float x[64];
     const float *src = p.dS_T ? p.dS_T + head * DK * DV + static_cast<size_t>(srow) * DV + half * 64 : nullptr;
 #pragma unroll
     for (int j = 0; j < 64; j += 4) {
-      const float4 x = src ? __ldg(reinterpret_cast<const float4 *>(src + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      dS[j] = x.x;
-      dS[j + 1] = x.y;
-      dS[j + 2] = x.z;
-      dS[j + 3] = x.w;
+      const float4 y = src ? __ldg(reinterpret_cast<const float4 *>(src + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      x[j] = y.x;
+      x[j + 1] = y.y;
+      x[j + 2] = y.z;
+      x[j + 3] = y.w;
     }
+#pragma unroll
+    for (int j = 0; j < 64; j += 16)
+      tmem_st16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), *reinterpret_cast<const float(*)[16]>(x + j));
+    tmem_st_wait();
   }
 
   // element helpers for a thread's row of a 128-row, 128-column tile (two 64-column blocks)
@@ -217,6 +233,13 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   // write scale of value columns col .. col + 3 of chunk row r (token index th): beta_v, or sqrt(beta_k)
   // when the write is symmetric (dk = dv)
+  auto wscale1 = [&](int r, size_t th, int col) -> float {
+    if (p.beta_v_mode == MODE_CHANNEL) return __ldg(g_beta_v + th * DV + col);
+    if (p.beta_v_mode == MODE_SCALAR) return __ldg(g_beta_v + th);
+    if (p.beta_k_mode == MODE_CHANNEL) return tc::sqrt_fast(__ldg(g_beta_k + th * DK + col));
+    if constexpr (kChanGates) return tc::sqrt_fast(__ldg(g_beta_k + th));
+    else return sRow[128 + r];
+  };
   auto wscale4 = [&](int r, size_t th, int col) -> float4 {
     if (p.beta_v_mode == MODE_CHANNEL) return __ldg(reinterpret_cast<const float4 *>(g_beta_v + th * DV + col));
     if (p.beta_v_mode == MODE_SCALAR) {
@@ -238,9 +261,10 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int t0 = c * C, L = min(C, T - t0);
     const size_t tok0 = static_cast<size_t>(b) * T + t0;  // first token of the chunk (dense batch)
 
-    // ------------------------------------------------------------------ loads: q, k, v, dO (TMA), S (global)
+    // ------------------------------------------------------------------ loads: q, k, v, dO and the fp32 state (TMA)
     if (tid == 0) {
-      mbar_arrive_expect_tx(&bar_ld, 8 * 64 * 128);
+      const int srow0 = (static_cast<int>(head) * NC + c) * DK;  // the state's first row in the states map
+      mbar_arrive_expect_tx(&bar_ld, 8 * 64 * 128 + 4 * 128 * 128);
       tma_load_4d(X + 64 * 128, &tm_q, &bar_ld, 0, h, t0, b);
       tma_load_4d(X + SX_CB + 64 * 128, &tm_q, &bar_ld, 64, h, t0, b);
       tma_load_4d(X, &tm_k, &bar_ld, 0, h, t0, b);
@@ -249,6 +273,8 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tma_load_4d(tDPA + 64 * 128, &tm_v, &bar_ld, 64, h, t0, b);
       tma_load_4d(tDO, &tm_do, &bar_ld, 0, h, t0, b);
       tma_load_4d(tDO + 128 * 128, &tm_do, &bar_ld, 64, h, t0, b);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tma_load_2d(sm + SST + j * SST_B, &tm_st, &bar_ld, 32 * j, srow0);
       if (c > 0) {
         for (int x = 0; x < 128; x += 64) {
           tma_prefetch_l2_4d(&tm_q, x, h, t0 - C, b);
@@ -256,35 +282,18 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tma_prefetch_l2_4d(&tm_v, x, h, t0 - C, b);
           tma_prefetch_l2_4d(&tm_do, x, h, t0 - C, b);
         }
+        for (int j = 0; j < 4; ++j) tma_prefetch_l2_2d(&tm_st, 32 * j, srow0 - DK);
       }
     }
-    // S of this chunk: fp16 operand tile, and the state part of the last-row term sum_v dS S
-    float rt = 0.f;
-    {
-      const float4 *src =
-          reinterpret_cast<const float4 *>(g_states + (head * NC + c) * DK * DV + static_cast<size_t>(srow) * DV + half * 64);
-      float4 sv[16];  // all of my 64 values in flight at once
-#pragma unroll
-      for (int e = 0; e < 16; ++e) sv[e] = __ldg(src + e);
-      if (c > 0) {  // the previous chunk's state into L2: my row half is two 128-byte lines
-        const float *nx = g_states + (head * NC + c - 1) * DK * DV + static_cast<size_t>(srow) * DV + half * 64;
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(nx));
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(nx + 32));
-      }
-#pragma unroll
-      for (int j = 0; j < 64; j += 16) {
-        float x[16];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          x[4 * e] = sv[j / 4 + e].x;
-          x[4 * e + 1] = sv[j / 4 + e].y;
-          x[4 * e + 2] = sv[j / 4 + e].z;
-          x[4 * e + 3] = sv[j / 4 + e].w;
-        }
-#pragma unroll
-        for (int e = 0; e < 16; ++e) rt += dS[j + e] * x[e];
-        tc::st_h16x16(tSS, srow, half * 64 + j, 128, x);
-      }
+    if (c > 0) {  // the previous chunk's gates into L2: thread = (row tid / 4, 128-byte line tid % 4)
+      const int pr = tid >> 2, pl = tid & 3;
+      const size_t tp = (tok0 - C + pr) * H + h;
+      if (p.alpha_mode == MODE_CHANNEL) asm volatile("prefetch.global.L2 [%0];" ::"l"(g_alpha + tp * DK + 32 * pl));
+      else if (p.alpha_mode == MODE_SCALAR && pl == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(g_alpha + tp));
+      if (p.beta_k_mode == MODE_CHANNEL) asm volatile("prefetch.global.L2 [%0];" ::"l"(g_beta_k + tp * DK + 32 * pl));
+      else if (pl == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(g_beta_k + tp));
+      if (p.beta_v_mode == MODE_CHANNEL) asm volatile("prefetch.global.L2 [%0];" ::"l"(g_beta_v + tp * DV + 32 * pl));
+      if (kScaled) asm volatile("prefetch.global.L2 [%0];" ::"l"(g_s + tp * DK + 32 * pl));
     }
     // gates
     float pal[4 * 8], pbe[4 * 8];  // channel gates: rows 8 rg .. 8 rg + 7, channels c0 .. c0 + 3
@@ -347,11 +356,33 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     // wait for the tiles
     if (!wait_ld()) { ok = false; break; }
+    // S of this chunk: the fp16 operand tile, and the state part of the last-row term sum_v dS S.  The
+    // staged fp32 rows are 128-byte-swizzled boxes of 32 columns.
+    float rt = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < 64; j += 16) {
+      float x[16], d[16];
+      tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), d);
+      const uint8_t *box = sm + SST + ((half * 64 + j) >> 5) * SST_B + srow * 128;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int ch = (((half * 64 + j) & 31) >> 2) + e;  // 16-byte chunk of the row within the box
+        const float4 y = *reinterpret_cast<const float4 *>(box + ((ch ^ (srow & 7)) << 4));
+        x[4 * e] = y.x;
+        x[4 * e + 1] = y.y;
+        x[4 * e + 2] = y.z;
+        x[4 * e + 3] = y.w;
+      }
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) rt += d[e] * x[e];
+      tc::st_h16x16(tSS, srow, half * 64 + j, 128, x);
+    }
 
     // ------------------------------------------------------------------ K1: Qh, Bh, Ac; write vectors; dO -> fp16
     float amax = 0.f;
     if constexpr (kChanGates) {
-      float *sPX = reinterpret_cast<float *>(tDM);  // row-group gate products, 8 x 128 fp32
+      float *sPX = reinterpret_cast<float *>(tTP);  // row-group gate products, 8 x 128 fp32 (T comes later)
       float pg[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
       for (int j = 0; j < 8; ++j)
@@ -449,7 +480,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     if (!(amax < kF16Max)) raise_status(p.status, STATUS_RANGE);
     // write vectors W = wsc (.) v (raw v waits in the dP/dA tile), and dO as fp16 in place: thread row
-    // tid >> 2, 8-column groups 4 (tid & 3) .. 4 (tid & 3) + 3 of 16
+    // tid >> 2, 8-column groups (tid & 3) + 4 g of 16 (four lanes cover 32 adjacent columns)
     {
       const int r = tid >> 2;
       const bool valid = r < L;
@@ -457,13 +488,13 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       float4 wq[8];
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
-        const int col = 8 * (4 * (tid & 3) + g);
+        const int col = 8 * ((tid & 3) + 4 * g);
         wq[2 * g] = wscale4(r, th, col);
         wq[2 * g + 1] = wscale4(r, th, col + 4);
       }
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
-        const int c8 = 4 * (tid & 3) + g;  // 8-column group (0..15)
+        const int c8 = (tid & 3) + 4 * g;  // 8-column group (0..15)
         const float wsc[8] = {wq[2 * g].x,     wq[2 * g].y,     wq[2 * g].z,     wq[2 * g].w,
                               wq[2 * g + 1].x, wq[2 * g + 1].y, wq[2 * g + 1].z, wq[2 * g + 1].w};
         uint4 *pd = reinterpret_cast<uint4 *>(tDO + sw128_off16(r, c8, 128));
@@ -597,33 +628,49 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tc_fence_before();
     __syncthreads();
 
-    // ------------------------------------------------------------------ Ac^T U;  dM = Diag(gamma_C) dS
+    // ------------------------------------------------------------------ Ac^T U (into the spent Bh S columns);  dM = Diag(gamma_C) dS
     if (warp == 0) {
       if (elect_one()) {
         tc_fence_after();
-        issue(COL_AU, C / 16, idesc_f16_f32(128, 128, true, true), false, mnmaj(sb + SAC, 64), mnmaj(sb + SUU, 64));
+        issue(COL_BS, C / 16, idesc_f16_f32(128, 128, true, true), false, mnmaj(sb + SAC, 64), mnmaj(sb + SUU, 64));
         umma_commit(&bar_mma);
       }
       __syncwarp();
     }
     const float gci = sGC[srow];
-    {
-      float dm[64];
+    {  // dM as the fp16 operand while the product runs
+      float mx = 0.f;
+#pragma unroll 1
+      for (int j = 0; j < 64; j += 16) {
+        float d[16];
+        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), d);
+        tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 64; ++e) dm[e] = gci * dS[e];
-      st_row64(tDM, 128, srow, half * 64, dm);
+        for (int e = 0; e < 16; ++e) {
+          d[e] *= gci;
+          mx = fmaxf(mx, fabsf(d[e]));
+        }
+        tc::st_h16x16(tDM, srow, half * 64 + j, 128, d);
+      }
+      if (!(mx < kF16Max)) raise_status(p.status, STATUS_RANGE);
     }
     if (!wait_mma()) { ok = false; break; }
-    // last-row term: sum_v dS (S + Ac^T U), per key row; the two value halves meet in shared memory
-    {
-      float x[64];
-#pragma unroll
-      for (int j = 0; j < 64; j += 16)
-        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), *reinterpret_cast<float(*)[16]>(x + j));
+    // last-row term: sum_v dS (S + Ac^T U), per key row; the two value halves meet in shared memory.  Then
+    // dM in fp32 replaces dS in TMEM: the state step accumulates onto it.
+#pragma unroll 1
+    for (int j = 0; j < 64; j += 16) {
+      float d[16], a[16];
+      tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), d);
+      tmem_ld16(tmem_addr(tmem, quarter * 32, COL_BS + half * 64 + j), a);
       tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 64; ++e) rt += dS[e] * x[e];
+      for (int e = 0; e < 16; ++e) {
+        rt += d[e] * a[e];
+        d[e] *= gci;
+      }
+      tmem_st16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), d);
     }
+    tmem_st_wait();
     sRT[half * 128 + srow] = rt;
     fence_async_smem();
     tc_fence_before();
@@ -658,84 +705,65 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tc_fence_before();
     __syncthreads();
 
-    // ------------------------------------------------------------------ dV = T^T dU -> -dV, dv, write strengths
+    // ------------------------------------------------------------------ dV^T = dU^T T -> -dV, dv, write strengths
+    // formed transposed (TMEM lane = value column) so that every global access below is a whole 128-byte
+    // line per warp and all eight warps share the epilogue
     if (warp == 0) {
       if (elect_one()) {
         tc_fence_after();
-        issue(COL_U, C / 16, idesc_f16_f32(128, 128, true, true), false, mnmaj(sb + STP, 128), mnmaj(sb + SWY, 64));
+        issue(COL_U, C / 16, idesc_f16_f32(128, 64, true, true), false, mnmaj(sb + SWY, 64), mnmaj(sb + STP, 128));
         umma_commit(&bar_mma);
       }
       __syncwarp();
     }
-    if (!wait_mma()) { ok = false; break; }
-    if (quarter < 2) {
-      const int r = srow;
-      const bool valid = r < L;
-      const size_t th = (tok0 + min(r, L - 1)) * H + h;
-      float4 wq[16];  // the write scales of my 64 value columns, in flight before the TMEM reads
+    {
+      // thread: value column vc = srow, rows 32 half .. 32 half + 31 in blocks of 8 whose write scales load
+      // one block ahead
+      const int vc = srow, r0 = 32 * half;
+      const bool row_sums = p.beta_v_mode == MODE_SCALAR || (p.beta_v_mode == MODE_ABSENT && p.beta_k_mode != MODE_CHANNEL);
+      auto ld_w = [&](int jb, float (&w)[8]) {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) wq[e] = wscale4(r, th, half * 64 + 4 * e);
-      float rsum = 0.f;  // sum over my value columns of v dV (scalar write strength)
-#pragma unroll
-      for (int j = 0; j < 64; j += 16) {
-        float x[16];
-        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_U + half * 64 + j), x);
+        for (int e = 0; e < 8; ++e) {
+          const int r = r0 + jb + e;
+          w[e] = wscale1(r, (tok0 + min(r, L - 1)) * H + h, vc);
+        }
+      };
+      float cw[8];
+      ld_w(0, cw);
+      if (!wait_mma()) { ok = false; break; }
+#pragma unroll 1
+      for (int jb = 0; jb < 32; jb += 8) {
+        float nw[8];
+        if (jb < 24) ld_w(jb + 8, nw);
+        float x[8], xr[8];  // dV of the block's rows; v dV for a write strength that is scalar per row
+        tmem_ld8(tmem_addr(tmem, quarter * 32, COL_U + r0 + jb), x);
         tmem_ld_wait();
-        const int v0 = half * 64 + j;
-        float nd[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) nd[e] = -x[e];
-        tc::st_h16x16(tDO, 64 + r, v0, 128, nd);
-        if (valid) {
-          // raw v of these 16 columns (from the dP/dA tile) and their write scales
-          float vf[16], wsc[16];
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            const uint4 raw = *reinterpret_cast<const uint4 *>(tDPA + sw128_off16(r, v0 / 8 + g, 64));
-            const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(v2[e]);
-              vf[8 * g + 2 * e] = f.x;
-              vf[8 * g + 2 * e + 1] = f.y;
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float4 w = wq[j / 4 + e];
-            wsc[4 * e] = w.x; wsc[4 * e + 1] = w.y; wsc[4 * e + 2] = w.z; wsc[4 * e + 3] = w.w;
-          }
-          float *dvo = g_dv + th * DV + v0;
-#pragma unroll
-          for (int e = 0; e < 16; e += 4)
-            *reinterpret_cast<float4 *>(dvo + e) =
-                make_float4(wsc[e] * x[e], wsc[e + 1] * x[e + 1], wsc[e + 2] * x[e + 2], wsc[e + 3] * x[e + 3]);
-          // gradient of the write scale: v (.) dV per column
-          if (p.beta_v_mode == MODE_CHANNEL) {
-            float *o = g_dbeta_v + th * DV + v0;
-#pragma unroll
-            for (int e = 0; e < 16; e += 4)
-              *reinterpret_cast<float4 *>(o + e) =
-                  make_float4(vf[e] * x[e], vf[e + 1] * x[e + 1], vf[e + 2] * x[e + 2], vf[e + 3] * x[e + 3]);
-          } else if (p.beta_v_mode == MODE_SCALAR || p.beta_k_mode != MODE_CHANNEL) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) rsum += vf[e] * x[e];
-          } else {
-            // symmetric channel write: d beta_k += 0.5 v dV / sqrt(beta_k), stored now, added to below
-            float *o = g_dbeta_k + th * DK + v0;
-#pragma unroll
-            for (int e = 0; e < 16; e += 4) {
-              float4 y;
-              y.x = wsc[e] > 0.f ? 0.5f * vf[e] * x[e] / wsc[e] : 0.f;
-              y.y = wsc[e + 1] > 0.f ? 0.5f * vf[e + 1] * x[e + 1] / wsc[e + 1] : 0.f;
-              y.z = wsc[e + 2] > 0.f ? 0.5f * vf[e + 2] * x[e + 2] / wsc[e + 2] : 0.f;
-              y.w = wsc[e + 3] > 0.f ? 0.5f * vf[e + 3] * x[e + 3] / wsc[e + 3] : 0.f;
-              *reinterpret_cast<float4 *>(o + e) = y;
+        for (int e = 0; e < 8; ++e) {
+          const int r = r0 + jb + e;
+          *reinterpret_cast<__half *>(tDO + sw128_off(64 + r, vc, 128)) = __float2half_rn(-x[e]);
+          const float vf = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tDPA + sw128_off(r, vc, 64)));
+          xr[e] = vf * x[e];
+          if (r < L) {
+            const size_t th = (tok0 + r) * H + h;
+            g_dv[th * DV + vc] = cw[e] * x[e];
+            if (p.beta_v_mode == MODE_CHANNEL) {
+              g_dbeta_v[th * DV + vc] = xr[e];
+            } else if (p.beta_v_mode == MODE_ABSENT && p.beta_k_mode == MODE_CHANNEL) {
+              // symmetric channel write: d beta_k += 0.5 v dV / sqrt(beta_k), stored now, added to below
+              g_dbeta_k[th * DK + vc] = cw[e] > 0.f ? 0.5f * __fdividef(xr[e], cw[e]) : 0.f;
             }
           }
         }
+        if (row_sums) {  // rows r0 + jb + (lane & 7), summed over my warp's 32 value columns
+          const float v = warp_transpose_sum<8>(xr, lane);
+          if (lane < 8) sRV[(r0 + jb + lane) * 4 + quarter] = v;
+        }
+        if (jb < 24) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) cw[e] = nw[e];
+        }
       }
-      sRV[r * 2 + half] = rsum;
     }
     fence_async_smem();
     tc_fence_before();
@@ -743,9 +771,9 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (tid < 64 && tid < L) {  // scalar write strength: one value per row
       const int r = tid;
       const size_t th = (tok0 + r) * H + h;
-      const float rs = sRV[2 * r] + sRV[2 * r + 1];
+      const float rs = sRV[4 * r] + sRV[4 * r + 1] + sRV[4 * r + 2] + sRV[4 * r + 3];
       if (p.beta_v_mode == MODE_SCALAR) g_dbeta_v[th] = rs;
-      else if (p.beta_k_mode == MODE_SCALAR) sRV[2 * r] = rs;  // symmetric scalar write: folded in below
+      else if (p.beta_k_mode == MODE_SCALAR) sRV[4 * r] = rs;  // symmetric scalar write: folded in below
     }
 
     // ------------------------------------------------------------------ dS_prev = Qh^T dO - Bh^T dV + dM;  [dP | dA]
@@ -753,7 +781,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (elect_one()) {
         tc_fence_after();
         const uint32_t id = idesc_f16_f32(128, 128, true, true);
-        issue(COL_AU, C / 16, id, false, mnmaj(sb + SX + 64 * 128, 128), mnmaj(sb + SDO, 128));
+        issue(COL_AU, C / 16, id, true, mnmaj(sb + SX + 64 * 128, 128), mnmaj(sb + SDO, 128));
         issue(COL_AU, C / 16, id, true, mnmaj(sb + SX, 128), mnmaj(sb + SDO + 64 * 128, 128));
         issue(COL_D1, DV / 16, idesc_f16_f32(128, 64, false, false), false, kmaj(sb + SDO, 128), kmaj(sb + SUU, 64));
         umma_commit(&bar_mma);
@@ -761,20 +789,6 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       __syncwarp();
     }
     if (!wait_mma()) { ok = false; break; }
-    {
-      float mx = 0.f;
-      float x[64];
-#pragma unroll
-      for (int j = 0; j < 64; j += 16)
-        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), *reinterpret_cast<float(*)[16]>(x + j));
-      tmem_ld_wait();
-#pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        dS[e] = gci * dS[e] + x[e];
-        mx = fmaxf(mx, fabsf(dS[e]));
-      }
-      if (!(mx < kF16Max)) raise_status(p.status, STATUS_RANGE);
-    }
     {  // dP (lower with diagonal, lanes 0..63) and dA (strictly lower, lanes 64..127)
       const int r = srow & 63;
       float x[32];
@@ -817,47 +831,52 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (!wait_mma()) { ok = false; break; }
 
     // ------------------------------------------------------------------ per key channel: gate gradients and outputs
-    // thread: key channel i = srow, rows 32 half .. 32 half + 31 of the chunk.  The state gradient waits in
-    // TMEM meanwhile (the state step's columns are free); q and k are read raw from the tiles just loaded.
+    // thread: key channel i = srow, rows 32 half .. 32 half + 31 of the chunk; q and k are read raw from the
+    // tiles just loaded
     {
       const int i = srow, r0 = 32 * half;
-#pragma unroll
-      for (int j = 0; j < 64; j += 16)
-        tmem_st16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), *reinterpret_cast<const float(*)[16]>(dS + j));
       const float rowterm = sRT[i] + sRT[128 + i];
       auto raw_at = [&](const uint8_t *tile, int r) {  // bf16 (r, channel i) of a 64-row swizzled tile
         return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + sw128_off(r, i, 64)));
       };
       if (!wait_ld()) { ok = false; break; }
       if constexpr (kChanGates) {
+        // shared scratch [32 rows][256 threads] in tiles the products above have released
+        float *sAl = reinterpret_cast<float *>(X);     // alpha of my rows
+        float *sGam = reinterpret_cast<float *>(tDM);  // gamma of my rows
+        float *sSuf = reinterpret_cast<float *>(tSS);  // the lower half's suffix sums
         // gamma of my rows: forward products (the lower half passes its product to the upper half)
-        float al[32], gam[32];
         float prod = 1.f;
+        {
+          float a[32];  // all loads in flight together
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int r = r0 + j;
-          const size_t th = (tok0 + min(r, L - 1)) * H + h;
-          float a = 1.f;
-          if (r < L) {
-            if (p.alpha_mode == MODE_CHANNEL) a = __ldg(g_alpha + th * DK + i);
-            else if (p.alpha_mode == MODE_SCALAR) a = __ldg(g_alpha + th);
+          for (int j = 0; j < 32; ++j) {
+            const int r = r0 + j;
+            const size_t th = (tok0 + min(r, L - 1)) * H + h;
+            a[j] = 1.f;
+            if (r < L) {
+              if (p.alpha_mode == MODE_CHANNEL) a[j] = __ldg(g_alpha + th * DK + i);
+              else if (p.alpha_mode == MODE_SCALAR) a[j] = __ldg(g_alpha + th);
+            }
           }
-          al[j] = a;
-          prod *= a;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            sAl[j * NT + tid] = a[j];
+            prod *= a[j];
+          }
         }
         if (half == 0) sXC[i] = prod;
         __syncthreads();
         {
           float g = half == 0 ? 1.f : sXC[i];
-#pragma unroll
+#pragma unroll 4
           for (int j = 0; j < 32; ++j) {
-            g *= al[j];
-            gam[j] = g;
+            g *= sAl[j * NT + tid];
+            sGam[j * NT + tid] = g;
           }
         }
-        // reverse over my rows, in blocks of 8 whose gate loads run one block ahead: dgamma, the local
+        // reverse over my rows in blocks of 8 whose gate loads run one block ahead: dgamma, the local
         // suffix sums of dgamma gamma, and the outputs
-        float *sSuf = reinterpret_cast<float *>(tSS);  // the lower half's suffix sums, [32][256] (S is spent)
         float acc = 0.f;
         float cb[8], cs[8], cp[8];  // beta_k, s and the stored write-side d beta_k of the block's rows
         auto load_blk = [&](int jb, float (&bk)[8], float (&sc)[8], float (&pv)[8]) {
@@ -871,11 +890,10 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           }
         };
         load_blk(24, cb, cs, cp);
-#pragma unroll
-        for (int blk = 3; blk >= 0; --blk) {
-          const int jb = 8 * blk;
+#pragma unroll 1
+        for (int jb = 24; jb >= 0; jb -= 8) {
           float nb[8], ns[8], np[8];
-          if (blk > 0) load_blk(jb - 8, nb, ns, np);
+          if (jb > 0) load_blk(jb - 8, nb, ns, np);
           float dq[8], db[8], da[8];
           tmem_ld8(tmem_addr(tmem, quarter * 32, COL_BS + r0 + jb), dq);
           tmem_ld8(tmem_addr(tmem, quarter * 32, COL_BS + 64 + r0 + jb), db);
@@ -886,7 +904,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int e = 7; e >= 0; --e) {
             const int j = jb + e, r = r0 + j;
             const bool valid = r < L;
-            const float gm = gam[j], ginv = __fdividef(1.f, gm);
+            const float gm = sGam[j * NT + tid], ginv = __fdividef(1.f, gm);
             const float qv = raw_at(tTP, r), kv = raw_at(tWY, r);
             const float sbt = valid ? tc::sqrt_fast(cb[e]) : 0.f;
             const float scv = kScaled ? (valid ? cs[e] : 0.f) : 1.f;
@@ -897,7 +915,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (half == 0) sSuf[j * NT + tid] = acc;
             xg[e] = dg * gm;
             const float dbt = gm * db[e] + scv * dav;  // through b = sqrt(beta) k and a = s b
-            const float dbk = sbt > 0.f ? 0.5f * kv * dbt / sbt : 0.f;
+            const float dbk = sbt > 0.f ? 0.5f * kv * __fdividef(dbt, sbt) : 0.f;
             xb[e] = dbk;
             if (valid) {
               const size_t o = ((tok0 + r) * H + h) * DK + i;
@@ -905,7 +923,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               g_dk[o] = sbt * dbt;
               if constexpr (kScaled) g_ds[o] = bv * dav;
               if (p.beta_k_mode == MODE_CHANNEL) g_dbeta_k[o] = cp[e] + dbk;
-              if (p.alpha_mode == MODE_CHANNEL && half == 1) g_dalpha[o] = acc / al[j];
+              if (p.alpha_mode == MODE_CHANNEL && half == 1) g_dalpha[o] = acc / sAl[j * NT + tid];
             }
           }
           if (p.beta_k_mode != MODE_CHANNEL) {  // summed over channels: rows r0 + jb + (lane & 7)
@@ -916,7 +934,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const float v = warp_transpose_sum<8>(xg, lane);
             if (lane < 8) sRed[((r0 + jb + lane) * 4 + quarter) * 2 + 1] = v;
           }
-          if (blk > 0) {
+          if (jb > 0) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               cb[e] = nb[e];
@@ -930,34 +948,33 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         __syncthreads();
         if (half == 0 && p.alpha_mode == MODE_CHANNEL) {
           const float off = sXC[128 + i];
-#pragma unroll
+#pragma unroll 4
           for (int j = 0; j < 32; ++j)
-            if (j < L) g_dalpha[((tok0 + j) * H + h) * DK + i] = (sSuf[j * NT + tid] + off) / al[j];
+            if (j < L) g_dalpha[((tok0 + j) * H + h) * DK + i] = (sSuf[j * NT + tid] + off) / sAl[j * NT + tid];
         }
       } else {
         // gates scalar per row (the scan's gamma, 1/gamma, sqrt(beta_k) in shared memory); the per-row
-        // terms are summed over channels after the loop
-        float xg[32], xb[32];
+        // terms are summed over channels block by block
         float cs[8];
         auto load_s = [&](int jb, float (&sc)[8]) {
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             sc[e] = kScaled ? __ldg(g_s + ((tok0 + min(r0 + jb + e, L - 1)) * H + h) * DK + i) : 1.f;
         };
-        load_s(24, cs);
-#pragma unroll
-        for (int blk = 3; blk >= 0; --blk) {
-          const int jb = 8 * blk;
+        load_s(0, cs);
+#pragma unroll 1
+        for (int jb = 0; jb < 32; jb += 8) {
           float ns[8];
-          if (blk > 0) load_s(jb - 8, ns);
+          if (jb < 24) load_s(jb + 8, ns);
           float dq[8], db[8], da[8];
           tmem_ld8(tmem_addr(tmem, quarter * 32, COL_BS + r0 + jb), dq);
           tmem_ld8(tmem_addr(tmem, quarter * 32, COL_BS + 64 + r0 + jb), db);
           tmem_ld8(tmem_addr(tmem, quarter * 32, COL_U + r0 + jb), da);
           tmem_ld_wait();
+          float xg[8], xb[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int j = jb + e, r = r0 + j;
+            const int r = r0 + jb + e;
             const bool valid = r < L;
             const float gm = sRow[r], ginv = sRow[64 + r], sbt = sRow[128 + r];
             const float qv = raw_at(tTP, r), kv = raw_at(tWY, r);
@@ -965,9 +982,9 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const float bv = sbt * kv, av = scv * bv, dav = da[e] * ginv;
             float dg = qv * dq[e] + bv * db[e] - av * dav * ginv;
             if (r == C - 1) dg += rowterm;
-            xg[j] = dg * gm;
+            xg[e] = dg * gm;
             const float dbt = gm * db[e] + scv * dav;
-            xb[j] = sbt > 0.f ? 0.5f * kv * __fdividef(dbt, sbt) : 0.f;
+            xb[e] = sbt > 0.f ? 0.5f * kv * __fdividef(dbt, sbt) : 0.f;
             if (valid) {
               const size_t o = ((tok0 + r) * H + h) * DK + i;
               g_dq[o] = gm * dq[e];
@@ -975,17 +992,17 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               if constexpr (kScaled) g_ds[o] = bv * dav;
             }
           }
-          if (blk > 0) {
+          // sums over my warp's 32 channels: rows r0 + jb + (lane & 7)
+          const float sbk = warp_transpose_sum<8>(xb, lane);
+          if (lane < 8) sRed[((r0 + jb + lane) * 4 + quarter) * 2] = sbk;
+          if (p.alpha_mode == MODE_SCALAR) {
+            const float sg = warp_transpose_sum<8>(xg, lane);
+            if (lane < 8) sRed[((r0 + jb + lane) * 4 + quarter) * 2 + 1] = sg;
+          }
+          if (jb < 24) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) cs[e] = ns[e];
           }
-        }
-        // sums over my warp's 32 channels: lane l holds row r0 + l
-        const float sb = warp_transpose_sum<32>(xb, lane);
-        sRed[((r0 + lane) * 4 + quarter) * 2] = sb;
-        if (p.alpha_mode == MODE_SCALAR) {
-          const float sg = warp_transpose_sum<32>(xg, lane);
-          sRed[((r0 + lane) * 4 + quarter) * 2 + 1] = sg;
         }
       }
       __syncthreads();
@@ -1027,19 +1044,13 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               float v = bs[e];
               if (sym_write) {  // w = sqrt(beta_k) v as well: 0.5 / sqrt(beta_k) sum_v v dV
                 const float sbt = kChanGates ? tc::sqrt_fast(__ldg(g_beta_k + th)) : sRow[128 + r];
-                v += sbt > 0.f ? 0.5f * sRV[2 * r] / sbt : 0.f;
+                v += sbt > 0.f ? 0.5f * sRV[4 * r] / sbt : 0.f;
               }
               g_dbeta_k[th] = v;
             }
           }
         }
       }
-      // the state gradient back into registers
-      tmem_st_wait();
-#pragma unroll
-      for (int j = 0; j < 64; j += 16)
-        tmem_ld16(tmem_addr(tmem, quarter * 32, COL_AU + half * 64 + j), *reinterpret_cast<float(*)[16]>(dS + j));
-      tmem_ld_wait();
     }
     tc_fence_before();
     __syncthreads();
@@ -1047,6 +1058,8 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   }
 
   if (ok && p.dS0) {
+    float dS[64];
+    ld_au(dS);
     float *dst = p.dS0 + head * DK * DV + static_cast<size_t>(srow) * DV + half * 64;
 #pragma unroll
     for (int j = 0; j < 64; j += 4) *reinterpret_cast<float4 *>(dst + j) = make_float4(dS[j], dS[j + 1], dS[j + 2], dS[j + 3]);

@@ -404,6 +404,17 @@ dr_status bwd_chunk_launch(const dr_problem *p, const void *q, const void *k, co
       !make_map(&mdo, bf, 2, dout, p->B, p->T, p->H, p->dv, 64, dr::tc::C, sw))
     return DR_ERR_CUDA;
   const int nc = (p->T + dr::tc::C - 1) / dr::tc::C;
+  alignas(64) CUtensorMap mst;  // the chunk-start states as rows of dv fp32: 32-column x 128-row boxes
+  {
+    auto enc = tensor_map_encoder();
+    const cuuint64_t dims[2] = {cuuint64_t(p->dv), cuuint64_t(p->B) * p->H * nc * p->dk};
+    const cuuint64_t strides[1] = {cuuint64_t(p->dv) * sizeof(float)};
+    const cuuint32_t box[2] = {32u, 128u}, estr[2] = {1u, 1u};
+    if (!enc || enc(&mst, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, states, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return DR_ERR_CUDA;
+  }
   bwc::BwdChunkParams bp{p->T, p->H, nc, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v, p->beta_v_mode, s,
                          static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
                          static_cast<const __nv_bfloat16 *>(v), states, dS_T, dq, dk, dv, dalpha, dbeta_k, dbeta_v,
@@ -415,7 +426,7 @@ dr_status bwd_chunk_launch(const dr_problem *p, const void *q, const void *k, co
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
     return DR_ERR_CUDA;
-  kern<<<dim3(p->H, p->B), bwc::NT, smem, st>>>(mq, mk, mv, mdo, bp);
+  kern<<<dim3(p->H, p->B), bwc::NT, smem, st>>>(mq, mk, mv, mdo, mst, bp);
   return launch_status();
 }
 
