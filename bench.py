@@ -35,6 +35,7 @@ import torch
 from synth import CONFIGS, DECODE, decode_inputs, make_inputs, problem
 
 METRIC = "delta-rule fwd Mtokens·heads/s (prefill) & decode GB/s; % of roofline"
+HOST_COVER_CYCLES = 400_000  # about 0.2 ms of GPU sleep ahead of a timed launch that follows an L2 flush
 WORKLOAD = "fg2plus_bf16"  # the headline step's workload: the largest single-GPU configuration
 PREFILL_WORKLOADS = ("fg2plus_bf16", "kda_bf16", "gdn_bf16", "deltanet_f32")
 L2_BYTES = 126 * 2 ** 20
@@ -382,7 +383,11 @@ def time_prefill_workload(dr, p, dev, st, steps, warmup, ws, peaks, peaks_src):
     torch.cuda.synchronize()
     for e0, e1 in ev:
         if flush is not None:
-            flush.fill_(1)
+            with torch.cuda.stream(st):
+                flush.fill_(1)
+                # keep the stream busy while the host enqueues the launch, so that the events time the
+                # kernel and not the host's launch latency
+                torch.cuda._sleep(HOST_COVER_CYCLES)
         e0.record(st)
         run()
         e1.record(st)

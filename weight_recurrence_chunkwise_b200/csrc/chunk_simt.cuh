@@ -9,12 +9,13 @@
 //   gamma_r = prod_{j<=r} alpha_j             cumulative gate (K1)
 //   Bh_r = gamma_r b_r,  Ac_r = a_r / gamma_r,  Qh_r = gamma_r q_r
 //   (write key a = b, or a = s (.) b under OSDN's write-side key scaling)
-//   A = strictly-lower(Bh Ac^T),  T = (I + A)^-1,  P = lower(Qh Ac^T)   (K2)
-//   U = T (Wr - Bh S)                         (K2 + K3: rows u_r of the chunk)
+//   A = strictly-lower(Bh Ac^T),  P = lower(Qh Ac^T)                     (K2)
+//   U = (I + A)^-1 (Wr - Bh S)                (K2 + K3: forward substitution, rows u_r of the chunk)
 //   O = Qh S + P U                            (K4)
 //   S <- Diag(gamma_L) (S + Ac^T U)           (K3; Ac_r gamma_L = decayed key)
 //
-// Grid: (dv / VS, H, B); one CTA walks all chunks of one (b, h, value slice).
+// Grid: (dv / VS, H, B); one CTA walks all chunks of one (b, h, value slice).  Every product is a
+// register-tiled loop over shared-memory operands, so its loads overlap its FFMA chains.
 #pragma once
 #include "common.cuh"
 
@@ -24,21 +25,42 @@ template <int DK, int VS, int C>
 struct SimtSmem {
   static constexpr int LDK = DK + 1, LC = C + 1, LV = VS + 1;
   static constexpr size_t floats = 3 * C * LDK     // Bh, Ac, Qh
-                                   + 3 * C * LC    // A, T, P
-                                   + 2 * C * LV    // Wr/U, X
+                                   + 2 * C * LC    // A, P
+                                   + 3 * C * LV    // write vectors, X -> U, the output's Qh S part
                                    + DK * LV       // S slice
-                                   + DK;           // gamma at chunk end
+                                   + DK            // gamma at chunk end
+                                   + C * LDK       // staged channel decays of the chunk
+                                   + 2 * C;        // staged per-row decays and strengths
   static constexpr size_t bytes = floats * sizeof(float);
 };
 
+// acc[TR][TN] += sum_k a(r0 + i, k) b(k, c0 + j): a thread's register tile of a product of two
+// shared-memory operands (the k loop's loads are independent of the accumulation chains)
+template <int TR, int TN, typename FA, typename FB>
+__device__ __forceinline__ void simt_tile_mm(float (&acc)[TR][TN], int r0, int c0, int K, FA a, FB b) {
+#pragma unroll 4
+  for (int k = 0; k < K; ++k) {
+    float av[TR], bv[TN];
+#pragma unroll
+    for (int i = 0; i < TR; ++i) av[i] = a(r0 + i, k);
+#pragma unroll
+    for (int j = 0; j < TN; ++j) bv[j] = b(k, c0 + j);
+#pragma unroll
+    for (int i = 0; i < TR; ++i)
+#pragma unroll
+      for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+  }
+}
+
 template <typename IO, int DK, int DV, int VS, int C>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restrict__ k,
                       const IO *__restrict__ v, const float *__restrict__ alpha, int alpha_mode,
                       const float *__restrict__ beta_k, int beta_k_mode, const float *__restrict__ beta_v,
                       int beta_v_mode, const float *__restrict__ s_scale, const int *__restrict__ cu_seqlens,
                       const float *__restrict__ S0, IO *__restrict__ o, float *__restrict__ S_T,
                       uint32_t *__restrict__ status) {
+  static_assert(VS == 32 && (C == 16 || C == 32 || C == 64) && (DK == 64 || DK == 128), "tile shapes");
   using L_ = SimtSmem<DK, VS, C>;
   constexpr int LDK = L_::LDK, LC = L_::LC, LV = L_::LV;
   extern __shared__ float sm[];
@@ -46,12 +68,14 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
   float *Ac = Bh + C * LDK;
   float *Qh = Ac + C * LDK;
   float *Am = Qh + C * LDK;
-  float *Tm = Am + C * LC;
-  float *Pm = Tm + C * LC;
-  float *Wr = Pm + C * LC;   // write vectors, then U
-  float *Xm = Wr + C * LV;
-  float *Ss = Xm + C * LV;
+  float *Pm = Am + C * LC;
+  float *Wr = Pm + C * LC;   // write vectors
+  float *Xm = Wr + C * LV;   // X = Wr - Bh S, then U in place
+  float *Om = Xm + C * LV;   // Qh S
+  float *Ss = Om + C * LV;
   float *gL = Ss + DK * LV;
+  float *sAl = gL + DK;         // [C][LDK] channel decays of the chunk
+  float *sRow = sAl + C * LDK;  // [2][C] per-row decay and erase strength
 
   const int tid = threadIdx.x;
   const int v0 = blockIdx.x * VS, h = blockIdx.y, b = blockIdx.z;
@@ -70,126 +94,160 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
     Ss[i * LV + j] = S0 ? S0[sbase + static_cast<size_t>(i) * DV + v0 + j] : 0.f;
   }
 
+  // thread tiles: [Bh; Qh] x (Ac^T | S) over 2C rows; the output over C rows; the state over DK rows
+  constexpr int TR2 = C / 16, TNA = C / 8, TNV = 4;      // 32 row blocks x 8 column blocks
+  constexpr int TRO = C == 16 ? 1 : C / 32, TNO = C == 16 ? 2 : 4, NCO = VS / TNO;  // output tile
+  constexpr int TRS = DK / 32;                            // state tile: 32 row blocks x 8 column blocks
   for (int t0 = 0; t0 < T; t0 += C) {
     const int L = min(C, T - t0);
     __syncthreads();
-    // ---- K1 + input scaling: one thread per key channel walks the chunk
+    // ---- stage the chunk: q, k, the gates (coalesced, all threads) and the write vectors; rows past
+    // the chunk's end read as identity transitions (alpha 1, beta 0, zero vectors)
+    for (int e = tid; e < C * DK; e += blockDim.x) {
+      const int r = e / DK, c = e % DK;
+      const bool valid = r < L;
+      const size_t th = (tok0 + t0 + min(r, L - 1)) * H + h;
+      Qh[r * LDK + c] = valid ? to_f32(q[th * DK + c]) : 0.f;
+      Bh[r * LDK + c] = valid ? to_f32(k[th * DK + c]) : 0.f;
+      if (alpha_mode == MODE_CHANNEL) sAl[r * LDK + c] = valid ? __ldg(alpha + th * DK + c) : 1.f;
+      if (beta_k_mode == MODE_CHANNEL) Ac[r * LDK + c] = valid ? __ldg(beta_k + th * DK + c) : 0.f;
+    }
+    for (int r = tid; r < C; r += blockDim.x) {
+      const bool valid = r < L;
+      const size_t th = (tok0 + t0 + min(r, L - 1)) * H + h;
+      sRow[r] = (valid && alpha_mode == MODE_SCALAR) ? __ldg(alpha + th) : 1.f;
+      sRow[C + r] = (valid && beta_k_mode == MODE_SCALAR) ? __ldg(beta_k + th) : 0.f;
+    }
+    for (int e = tid; e < C * VS; e += blockDim.x) {
+      const int r = e / VS, j = e % VS;
+      float w = 0.f;
+      if (r < L) {
+        const size_t th = (tok0 + t0 + r) * H + h;
+        const float vj = to_f32(v[th * DV + v0 + j]);
+        const float ws = (beta_v_mode != MODE_ABSENT) ? gate_at(beta_v, beta_v_mode, th, DV, v0 + j)
+                                                      : sqrtf(gate_at(beta_k, beta_k_mode, th, DK, v0 + j));
+        w = ws * vj;
+      }
+      Wr[r * LV + j] = w;
+    }
+    __syncthreads();
+    // ---- K1 + input scaling: one thread per key channel walks the staged chunk
     if (tid < DK) {
       float g = 1.f;
+#pragma unroll 8
       for (int r = 0; r < C; ++r) {
-        if (r < L) {
-          const size_t th = (tok0 + t0 + r) * H + h;
-          g *= gate_at(alpha, alpha_mode, th, DK, tid);
-          const float bk = sqrtf(gate_at(beta_k, beta_k_mode, th, DK, tid)) * to_f32(k[th * DK + tid]);
-          Bh[r * LDK + tid] = g * bk;
-          const float ak = s_scale ? s_scale[th * DK + tid] * bk : bk;  // write key a
-          Ac[r * LDK + tid] = ak / g;
-          Qh[r * LDK + tid] = g * to_f32(q[th * DK + tid]);
-        } else {
-          Bh[r * LDK + tid] = 0.f;
-          Ac[r * LDK + tid] = 0.f;
-          Qh[r * LDK + tid] = 0.f;
-        }
+        const float a = alpha_mode == MODE_CHANNEL ? sAl[r * LDK + tid] : sRow[r];
+        const float bt = beta_k_mode == MODE_CHANNEL ? Ac[r * LDK + tid] : sRow[C + r];
+        g *= a;
+        const float bk = sqrtf(bt) * Bh[r * LDK + tid];
+        float ak = bk;  // write key a
+        if (s_scale && r < L) ak *= s_scale[((tok0 + t0 + r) * H + h) * DK + tid];
+        Bh[r * LDK + tid] = g * bk;
+        Ac[r * LDK + tid] = ak / g;
+        Qh[r * LDK + tid] *= g;
       }
       gL[tid] = g;
       if (!(g >= kMinChunkDecay)) raise_status(status, STATUS_RANGE);
-    } else {
-      for (int e = tid - DK; e < C * VS; e += blockDim.x - DK) {
-        const int r = e / VS, j = e % VS;
-        float w = 0.f;
+    }
+    __syncthreads();
+    // ---- K2: [A; P] = [Bh; Qh] Ac^T (A strictly lower, P lower), and [X; Qh S] = [Wr; 0] - [Bh; -Qh] S
+    {
+      const int rb = tid >> 3, cb = tid & 7;
+      auto xq = [&](int r, int c) { return r < C ? Bh[r * LDK + c] : Qh[(r - C) * LDK + c]; };
+      {
+        float acc[TR2][TNA] = {};
+        simt_tile_mm(acc, rb * TR2, cb * TNA, DK, xq, [&](int c, int n) { return Ac[n * LDK + c]; });
+#pragma unroll
+        for (int i = 0; i < TR2; ++i) {
+          const int r = rb * TR2 + i;
+#pragma unroll
+          for (int jn = 0; jn < TNA; ++jn) {
+            const int n = cb * TNA + jn;
+            if (r < C) Am[r * LC + n] = n < r ? acc[i][jn] : 0.f;
+            else Pm[(r - C) * LC + n] = n <= r - C ? acc[i][jn] : 0.f;
+          }
+        }
+      }
+      {
+        float acc[TR2][TNV] = {};
+        simt_tile_mm(acc, rb * TR2, cb * TNV, DK, xq, [&](int c, int j) { return Ss[c * LV + j]; });
+#pragma unroll
+        for (int i = 0; i < TR2; ++i) {
+          const int r = rb * TR2 + i;
+#pragma unroll
+          for (int jv = 0; jv < TNV; ++jv) {
+            const int j = cb * TNV + jv;
+            if (r < C) Xm[r * LV + j] = Wr[r * LV + j] - acc[i][jv];
+            else Om[(r - C) * LV + j] = acc[i][jv];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // ---- K2 + K3: U = (I + A)^-1 X by forward substitution, in place over X.  Eight threads per value
+    // column; thread qd keeps rows qd, qd + 8, ... of its column in registers and adds its share of
+    // each row's sum, which a three-step butterfly completes.  Rows past the chunk's end have x = 0
+    // and a zero row of A, so their u is 0.
+    {
+      const int j = tid >> 3, qd = tid & 7;
+      float u[C / 8];
+#pragma unroll
+      for (int r = 0; r < C; ++r) {
+        float acc0 = 0.f, acc1 = 0.f;  // two chains
+#pragma unroll
+        for (int i = 0; i < C / 8; ++i) {
+          const int m = 8 * i + qd;
+          if (8 * i < r && m < r) {
+            if (i & 1) acc1 = fmaf(Am[r * LC + m], u[i], acc1);
+            else acc0 = fmaf(Am[r * LC + m], u[i], acc0);
+          }
+        }
+        float acc = acc0 + acc1;
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        if ((r & 7) == qd) u[r >> 3] = Xm[r * LV + j] - acc;
+      }
+#pragma unroll
+      for (int i = 0; i < C / 8; ++i) Xm[(8 * i + qd) * LV + j] = u[i];
+    }
+    __syncthreads();
+    // ---- K4: O = Qh S + P U;  K3: S <- Diag(gamma_L) (S + Ac^T U)  (disjoint outputs, no barrier)
+    {
+      const int rb = tid / NCO, cb = tid % NCO;
+      float acc[TRO][TNO];
+#pragma unroll
+      for (int i = 0; i < TRO; ++i)
+#pragma unroll
+        for (int jo = 0; jo < TNO; ++jo) acc[i][jo] = Om[(rb * TRO + i) * LV + cb * TNO + jo];
+      simt_tile_mm(acc, rb * TRO, cb * TNO, C, [&](int r, int m) { return Pm[r * LC + m]; },
+                   [&](int m, int j) { return Xm[m * LV + j]; });
+#pragma unroll
+      for (int i = 0; i < TRO; ++i) {
+        const int r = rb * TRO + i;
         if (r < L) {
           const size_t th = (tok0 + t0 + r) * H + h;
-          const float vj = to_f32(v[th * DV + v0 + j]);
-          const float ws = (beta_v_mode != MODE_ABSENT) ? gate_at(beta_v, beta_v_mode, th, DV, v0 + j)
-                                                        : sqrtf(gate_at(beta_k, beta_k_mode, th, DK, v0 + j));
-          w = ws * vj;
-        }
-        Wr[r * LV + j] = w;
-      }
-    }
-    __syncthreads();
-    // ---- K2: A = strictly-lower(Bh Ac^T), P = lower(Qh Ac^T)
-    for (int e = tid; e < C * C; e += blockDim.x) {
-      const int r = e / C, i = e % C;
-      float sa = 0.f, sp = 0.f;
-      if (i <= r) {
-        for (int c = 0; c < DK; ++c) {
-          const float ac = Ac[i * LDK + c];
-          sa = fmaf(Bh[r * LDK + c], ac, sa);
-          sp = fmaf(Qh[r * LDK + c], ac, sp);
+#pragma unroll
+          for (int jo = 0; jo < TNO; ++jo) o[th * DV + v0 + cb * TNO + jo] = from_f32<IO>(acc[i][jo]);
         }
       }
-      Am[r * LC + i] = (i < r) ? sa : 0.f;
-      Pm[r * LC + i] = sp;
     }
-    __syncthreads();
-    // ---- K2: T = (I + A)^-1, forward substitution, one column per thread
-    if (tid < C) {
-      const int j = tid;
-      for (int r = 0; r < C; ++r) Tm[r * LC + j] = (r == j) ? 1.f : 0.f;
-      for (int r = j + 1; r < L; ++r) {
-        float acc = 0.f;
-        for (int m = j; m < r; ++m) acc = fmaf(Am[r * LC + m], Tm[m * LC + j], acc);
-        Tm[r * LC + j] = -acc;
-      }
-    }
-    __syncthreads();
-    // ---- X = Wr - Bh S and the inter-chunk part of the output, Qh S
-    constexpr int PER = (C * VS) / 256;  // outputs per thread
-    float o1[PER];
     {
-      const int r = tid / (VS / PER), j0 = (tid % (VS / PER)) * PER;
-      float xs[PER];
+      const int rb = tid >> 3, cb = tid & 7;
+      float acc[TRS][TNV];
 #pragma unroll
-      for (int jj = 0; jj < PER; ++jj) xs[jj] = o1[jj] = 0.f;
-      for (int c = 0; c < DK; ++c) {
-        const float bh = Bh[r * LDK + c], qh = Qh[r * LDK + c];
+      for (int i = 0; i < TRS; ++i)
 #pragma unroll
-        for (int jj = 0; jj < PER; ++jj) {
-          const float s = Ss[c * LV + j0 + jj];
-          xs[jj] = fmaf(bh, s, xs[jj]);
-          o1[jj] = fmaf(qh, s, o1[jj]);
-        }
+        for (int jv = 0; jv < TNV; ++jv) acc[i][jv] = Ss[(rb * TRS + i) * LV + cb * TNV + jv];
+      simt_tile_mm(acc, rb * TRS, cb * TNV, C, [&](int i, int r) { return Ac[r * LDK + i]; },
+                   [&](int r, int j) { return Xm[r * LV + j]; });
+#pragma unroll
+      for (int i = 0; i < TRS; ++i) {
+        const int ii = rb * TRS + i;
+        const float g = gL[ii];
+#pragma unroll
+        for (int jv = 0; jv < TNV; ++jv) Ss[ii * LV + cb * TNV + jv] = g * acc[i][jv];
       }
-#pragma unroll
-      for (int jj = 0; jj < PER; ++jj) Xm[r * LV + j0 + jj] = Wr[r * LV + j0 + jj] - xs[jj];
-    }
-    __syncthreads();
-    // ---- U = T X  (stored over Wr)
-    {
-      const int r = tid / (VS / PER), j0 = (tid % (VS / PER)) * PER;
-      float u[PER];
-#pragma unroll
-      for (int jj = 0; jj < PER; ++jj) u[jj] = 0.f;
-      for (int m = 0; m <= r; ++m) {
-        const float tv = Tm[r * LC + m];
-#pragma unroll
-        for (int jj = 0; jj < PER; ++jj) u[jj] = fmaf(tv, Xm[m * LV + j0 + jj], u[jj]);
-      }
-#pragma unroll
-      for (int jj = 0; jj < PER; ++jj) Wr[r * LV + j0 + jj] = u[jj];
-    }
-    __syncthreads();
-    // ---- K4: O = Qh S + P U
-    {
-      const int r = tid / (VS / PER), j0 = (tid % (VS / PER)) * PER;
-      for (int m = 0; m <= r; ++m) {
-        const float pv = Pm[r * LC + m];
-#pragma unroll
-        for (int jj = 0; jj < PER; ++jj) o1[jj] = fmaf(pv, Wr[m * LV + j0 + jj], o1[jj]);
-      }
-      if (r < L) {
-        const size_t th = (tok0 + t0 + r) * H + h;
-#pragma unroll
-        for (int jj = 0; jj < PER; ++jj) o[th * DV + v0 + j0 + jj] = from_f32<IO>(o1[jj]);
-      }
-    }
-    // ---- K3: S <- Diag(gamma_L) (S + Ac^T U)
-    for (int e = tid; e < DK * VS; e += blockDim.x) {
-      const int i = e / VS, j = e % VS;
-      float acc = Ss[i * LV + j];
-      for (int r = 0; r < L; ++r) acc = fmaf(Ac[r * LDK + i], Wr[r * LV + j], acc);
-      Ss[i * LV + j] = gL[i] * acc;
     }
   }
   __syncthreads();
