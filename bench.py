@@ -316,7 +316,7 @@ def run_backward(args, dr, p, x, dev, st, peaks, peaks_src):
     S0 = torch.zeros((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=dev)
     dST = torch.randn((p.B, p.H, p.dk, p.dv), generator=g).to(dev)
     chunk_path = p.io == "bf16" and p.dk == 128 and p.dv == 128
-    out = {"backward": True, "workload": p.name}
+    out = {"backward": True, "workload": p.name, "T": p.T}
     for variant in (["default", "sequential"] if chunk_path else ["default"]):
         run = lambda: dr.dr_diag_backward_variant(variant, x["q"], x["k"], x["v"], x["beta_k"], dout,
                                                   alpha=x["alpha"], beta_v=x["beta_v"], S0=S0, dS_T=dST, stream=st)
@@ -419,6 +419,9 @@ def main():
                     help="with --only-prefill / --backward: the workload to time (default: the headline one)")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (dr_backward) on the --config workload instead")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="with --only-prefill / --backward: override the workload's T (profiling a shorter case "
+                         "of the same shape; the line reports the T it ran)")
     ap.add_argument("--seqpar-cost", action="store_true",
                     help="time one rank's work of a sequence-parallel prefill of the --config workload split "
                          "over 2, 4 and 8 ranks (on this one GPU) beside the unsplit prefill")
@@ -441,14 +444,17 @@ def main():
 
     if args.only_decode:
         return run_decode_only(args, dr, dev, st, ws)
-    if args.backward:
+    def aid_problem():  # the workload of a profiling aid, with its T overridden if asked
         p = rank_problem(rank, args.config)
+        return p if args.seq_len is None else p.replace(T=args.seq_len)
+
+    if args.backward:
+        p = aid_problem()
         return run_backward(args, dr, p, to_dev(make_inputs(p), dev), dev, st, peaks, peaks_src)
     if args.seqpar_cost:
         return run_seqpar_cost(args, dr, rank_problem(rank, args.config), dev, st)
     if args.only_prefill:
-        line = time_prefill_workload(dr, rank_problem(rank, args.config), dev, st, args.steps, args.warmup, ws,
-                                     peaks, peaks_src)
+        line = time_prefill_workload(dr, aid_problem(), dev, st, args.steps, args.warmup, ws, peaks, peaks_src)
         if rank == 0:
             print(json.dumps({"only_prefill": True, "prefill_ms": line["ms"], **line}), flush=True)
         return 0
