@@ -53,7 +53,7 @@ __device__ __forceinline__ void simt_tile_mm(float (&acc)[TR][TN], int r0, int c
 }
 
 template <typename IO, int DK, int DV, int VS, int C>
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(256, 2)  // launched with 256 threads
 chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restrict__ k,
                       const IO *__restrict__ v, const float *__restrict__ alpha, int alpha_mode,
                       const float *__restrict__ beta_k, int beta_k_mode, const float *__restrict__ beta_v,
@@ -61,6 +61,7 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
                       const float *__restrict__ S0, IO *__restrict__ o, float *__restrict__ S_T,
                       uint32_t *__restrict__ status) {
   static_assert(VS == 32 && (C == 16 || C == 32 || C == 64) && (DK == 64 || DK == 128), "tile shapes");
+  constexpr int kNT = 256;  // the launch's block size
   using L_ = SimtSmem<DK, VS, C>;
   constexpr int LDK = L_::LDK, LC = L_::LC, LV = L_::LV;
   extern __shared__ float sm[];
@@ -89,7 +90,8 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
   }
   const size_t sbase = (static_cast<size_t>(b) * H + h) * DK * DV;
 
-  for (int e = tid; e < DK * VS; e += blockDim.x) {
+#pragma unroll
+  for (int e = tid; e < DK * VS; e += kNT) {
     const int i = e / VS, j = e % VS;
     Ss[i * LV + j] = S0 ? S0[sbase + static_cast<size_t>(i) * DV + v0 + j] : 0.f;
   }
@@ -103,7 +105,8 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
     __syncthreads();
     // ---- stage the chunk: q, k, the gates (coalesced, all threads) and the write vectors; rows past
     // the chunk's end read as identity transitions (alpha 1, beta 0, zero vectors)
-    for (int e = tid; e < C * DK; e += blockDim.x) {
+#pragma unroll
+    for (int e = tid; e < C * DK; e += kNT) {  // all of a thread's loads in flight together
       const int r = e / DK, c = e % DK;
       const bool valid = r < L;
       const size_t th = (tok0 + t0 + min(r, L - 1)) * H + h;
@@ -112,13 +115,14 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
       if (alpha_mode == MODE_CHANNEL) sAl[r * LDK + c] = valid ? __ldg(alpha + th * DK + c) : 1.f;
       if (beta_k_mode == MODE_CHANNEL) Ac[r * LDK + c] = valid ? __ldg(beta_k + th * DK + c) : 0.f;
     }
-    for (int r = tid; r < C; r += blockDim.x) {
+    for (int r = tid; r < C; r += kNT) {
       const bool valid = r < L;
       const size_t th = (tok0 + t0 + min(r, L - 1)) * H + h;
       sRow[r] = (valid && alpha_mode == MODE_SCALAR) ? __ldg(alpha + th) : 1.f;
       sRow[C + r] = (valid && beta_k_mode == MODE_SCALAR) ? __ldg(beta_k + th) : 0.f;
     }
-    for (int e = tid; e < C * VS; e += blockDim.x) {
+#pragma unroll
+    for (int e = tid; e < C * VS; e += kNT) {
       const int r = e / VS, j = e % VS;
       float w = 0.f;
       if (r < L) {
@@ -252,7 +256,7 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
   }
   __syncthreads();
   if (S_T) {
-    for (int e = tid; e < DK * VS; e += blockDim.x) {
+    for (int e = tid; e < DK * VS; e += kNT) {
       const int i = e / VS, j = e % VS;
       S_T[sbase + static_cast<size_t>(i) * DV + v0 + j] = Ss[i * LV + j];
     }

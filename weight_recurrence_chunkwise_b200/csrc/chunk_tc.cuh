@@ -135,7 +135,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t mma_bar, raw_bar;
   __shared__ uint32_t tmem_base_sh;
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t *tQKB = sm + OFF_QKB;
   uint8_t *tAC = sm + OFF_AC;
   uint8_t *tTP = sm + OFF_TP;

@@ -106,7 +106,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   __shared__ uint64_t bar_qk, bar_lmma, bar_cmma, bar_out, bar_v;
   __shared__ uint64_t bar_full[NSLOT], bar_free[NSLOT], bar_land[NSLOT];
   __shared__ uint32_t tmem_base_sh;
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase_addr = smem_u32(sm);
 
   const int H = p.H, DV = p.DV;

@@ -20,7 +20,7 @@ umma_selftest_kernel(const uint16_t *__restrict__ A, const uint16_t *__restrict_
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar;
   __shared__ uint32_t tmem_base;
-  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t *sA = base;
   uint8_t *sB = base + M * K * 2;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -90,7 +90,7 @@ constexpr size_t kTriSelftestSmem =
 __global__ void __launch_bounds__(128) tri_selftest_kernel(int variant, const float *__restrict__ A,
                                                            float *__restrict__ Tout) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   auto put = [&](int bi, int bj, const tri::Frag &F, int ln) {
     const int row = 16 * bi + (ln >> 2), col = 16 * bj + 2 * (ln & 3);
