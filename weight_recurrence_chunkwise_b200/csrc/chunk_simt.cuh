@@ -34,17 +34,19 @@ struct SimtSmem {
   static constexpr size_t bytes = floats * sizeof(float);
 };
 
-// acc[TR][TN] += sum_k a(r0 + i, k) b(k, c0 + j): a thread's register tile of a product of two
-// shared-memory operands (the k loop's loads are independent of the accumulation chains)
-template <int TR, int TN, typename FA, typename FB>
-__device__ __forceinline__ void simt_tile_mm(float (&acc)[TR][TN], int r0, int c0, int K, FA a, FB b) {
+// acc[TR][TN] += sum_k a[i * ai + k * ak] b[k * bk + j * bj]: a thread's register tile of a product of two
+// shared-memory operands, given as strided views from the tile's first row / column (the k loop's loads
+// are independent of the accumulation chains)
+template <int TR, int TN>
+__device__ __forceinline__ void simt_tile_mm(float (&acc)[TR][TN], int K, const float *a, int ai, int ak,
+                                             const float *b, int bk, int bj) {
 #pragma unroll 4
   for (int k = 0; k < K; ++k) {
     float av[TR], bv[TN];
 #pragma unroll
-    for (int i = 0; i < TR; ++i) av[i] = a(r0 + i, k);
+    for (int i = 0; i < TR; ++i) av[i] = a[i * ai + k * ak];
 #pragma unroll
-    for (int j = 0; j < TN; ++j) bv[j] = b(k, c0 + j);
+    for (int j = 0; j < TN; ++j) bv[j] = b[k * bk + j * bj];
 #pragma unroll
     for (int i = 0; i < TR; ++i)
 #pragma unroll
@@ -157,10 +159,11 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
     // ---- K2: [A; P] = [Bh; Qh] Ac^T (A strictly lower, P lower), and [X; Qh S] = [Wr; 0] - [Bh; -Qh] S
     {
       const int rb = tid >> 3, cb = tid & 7;
-      auto xq = [&](int r, int c) { return r < C ? Bh[r * LDK + c] : Qh[(r - C) * LDK + c]; };
+      // a thread's TR2 rows of [Bh; Qh] lie all in Bh or all in Qh (TR2 divides C)
+      const float *xq = rb * TR2 < C ? Bh + rb * TR2 * LDK : Qh + (rb * TR2 - C) * LDK;
       {
         float acc[TR2][TNA] = {};
-        simt_tile_mm(acc, rb * TR2, cb * TNA, DK, xq, [&](int c, int n) { return Ac[n * LDK + c]; });
+        simt_tile_mm(acc, DK, xq, LDK, 1, Ac + cb * TNA * LDK, 1, LDK);
 #pragma unroll
         for (int i = 0; i < TR2; ++i) {
           const int r = rb * TR2 + i;
@@ -174,7 +177,7 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
       }
       {
         float acc[TR2][TNV] = {};
-        simt_tile_mm(acc, rb * TR2, cb * TNV, DK, xq, [&](int c, int j) { return Ss[c * LV + j]; });
+        simt_tile_mm(acc, DK, xq, LDK, 1, Ss + cb * TNV, LV, 1);
 #pragma unroll
         for (int i = 0; i < TR2; ++i) {
           const int r = rb * TR2 + i;
@@ -224,8 +227,7 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
       for (int i = 0; i < TRO; ++i)
 #pragma unroll
         for (int jo = 0; jo < TNO; ++jo) acc[i][jo] = Om[(rb * TRO + i) * LV + cb * TNO + jo];
-      simt_tile_mm(acc, rb * TRO, cb * TNO, C, [&](int r, int m) { return Pm[r * LC + m]; },
-                   [&](int m, int j) { return Xm[m * LV + j]; });
+      simt_tile_mm(acc, C, Pm + rb * TRO * LC, LC, 1, Xm + cb * TNO, LV, 1);
 #pragma unroll
       for (int i = 0; i < TRO; ++i) {
         const int r = rb * TRO + i;
@@ -243,8 +245,7 @@ chunk_fwd_simt_kernel(int T, int H, const IO *__restrict__ q, const IO *__restri
       for (int i = 0; i < TRS; ++i)
 #pragma unroll
         for (int jv = 0; jv < TNV; ++jv) acc[i][jv] = Ss[(rb * TRS + i) * LV + cb * TNV + jv];
-      simt_tile_mm(acc, rb * TRS, cb * TNV, C, [&](int i, int r) { return Ac[r * LDK + i]; },
-                   [&](int r, int j) { return Xm[r * LV + j]; });
+      simt_tile_mm(acc, C, Ac + rb * TRS, 1, LDK, Xm + cb * TNV, LV, 1);
 #pragma unroll
       for (int i = 0; i < TRS; ++i) {
         const int ii = rb * TRS + i;
