@@ -69,12 +69,18 @@ def decode_bytes(B, H, dk, dv, io=2, alpha_ch=True, beta_ch=True):
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the ncu captures
 # summarised under profiles/, each valid only for the kernel sources it was taken on: the key is
 # a digest of the kernel's own source files under csrc/ (see csrc_digest), so any change to them
-# voids the number, and the workload it was taken on, so other workloads report none.
+# voids the number, and the workload it was taken on, so other workloads report none.  Captures on
+# a shorter sequence of the same workload (T noted in the profile) are scaled by T to a full launch.
 RING_SOURCES = ("chunk_tc3.cuh", "chunk_tc.cuh", "tri_inverse.cuh", "sm100.cuh", "common.cuh")
+BWD_CHUNK_SOURCES = ("backward_chunk.cuh",) + RING_SOURCES
 MEASURED_TRAFFIC = {
-    ("chunk_fwd_ring_kernel", "gdn_bf16"): ("f89185e36ba6", 250.54976e6, RING_SOURCES),
+    ("chunk_fwd_ring_kernel", "gdn_bf16"): ("c36b98adf557", 248.92e6, RING_SOURCES),
+    ("chunk_fwd_ring_kernel", "kda_bf16"): ("c36b98adf557", 531.82e6, RING_SOURCES),
+    ("chunk_fwd_ring_kernel", "fg2plus_bf16"): ("c36b98adf557", 4 * 664.91e6, RING_SOURCES),  # T = 8192 x 4
+    ("chunk_fwd_simt_kernel", "deltanet_f32"): ("31898eacf605", 0.4628e6, ("chunk_simt.cuh", "common.cuh")),
     ("decode_stream_kernel", "decode_bf16"): ("6cb82d40c1fd", 1031.005696e6, ("decode_stream.cuh", "common.cuh")),
     ("delta_rule_bwd_kernel", "gdn_bf16"): ("9a0d1d786d6e", 10536.615e6, ("backward.cuh", "common.cuh")),
+    ("chunk_bwd_kernel", "gdn_bf16"): ("590ac77db6be", 4 * 207.81e6, BWD_CHUNK_SOURCES),  # T = 1024 x 4
 }
 
 def decode_kernel_name(heads, sms=148):
@@ -340,6 +346,10 @@ def run_backward(args, dr, p, x, dev, st, peaks, peaks_src):
                                      "frac": gbs / peaks["hbm_gbs"], "peak_source": peaks_src,
                                      "traffic": None if chunked else measured_traffic("delta_rule_bwd_kernel", p.name),
                                      "algorithmic_bytes_per_launch": byts}}
+        if chunked:  # the two launches' own DRAM traffic (forward with chunk states, then the backward walk)
+            out[variant]["traffic_by_kernel"] = {
+                "chunk_fwd_ring_kernel": None,  # with states stored: not captured
+                "chunk_bwd_kernel": measured_traffic("chunk_bwd_kernel", p.name) if p.T == CONFIGS[p.name].T else None}
     print(json.dumps(out), flush=True)
     return 0
 
