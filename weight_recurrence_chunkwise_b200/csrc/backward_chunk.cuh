@@ -233,13 +233,6 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   // write scale of value columns col .. col + 3 of chunk row r (token index th): beta_v, or sqrt(beta_k)
   // when the write is symmetric (dk = dv)
-  auto wscale1 = [&](int r, size_t th, int col) -> float {
-    if (p.beta_v_mode == MODE_CHANNEL) return __ldg(g_beta_v + th * DV + col);
-    if (p.beta_v_mode == MODE_SCALAR) return __ldg(g_beta_v + th);
-    if (p.beta_k_mode == MODE_CHANNEL) return tc::sqrt_fast(__ldg(g_beta_k + th * DK + col));
-    if constexpr (kChanGates) return tc::sqrt_fast(__ldg(g_beta_k + th));
-    else return sRow[128 + r];
-  };
   auto wscale4 = [&](int r, size_t th, int col) -> float4 {
     if (p.beta_v_mode == MODE_CHANNEL) return __ldg(reinterpret_cast<const float4 *>(g_beta_v + th * DV + col));
     if (p.beta_v_mode == MODE_SCALAR) {
@@ -721,11 +714,23 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // one block ahead
       const int vc = srow, r0 = 32 * half;
       const bool row_sums = p.beta_v_mode == MODE_SCALAR || (p.beta_v_mode == MODE_ABSENT && p.beta_k_mode != MODE_CHANNEL);
+      // the block's raw write-scale sources, loaded one block ahead and transformed at use (a square
+      // root applied here would make the thread wait for the loads at once): beta_v (per channel or per
+      // row), or for a symmetric write beta_k (per channel or per row), or the scan's sqrt(beta_k)
+      const bool w_scan = !kChanGates && p.beta_v_mode == MODE_ABSENT;
+      const bool w_sqrt = kChanGates && p.beta_v_mode == MODE_ABSENT;
+      const float *w_src = p.beta_v_mode != MODE_ABSENT ? g_beta_v : g_beta_k;
+      const bool w_chan = p.beta_v_mode == MODE_CHANNEL || (p.beta_v_mode == MODE_ABSENT && p.beta_k_mode == MODE_CHANNEL);
       auto ld_w = [&](int jb, float (&w)[8]) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int r = r0 + jb + e;
-          w[e] = wscale1(r, (tok0 + min(r, L - 1)) * H + h, vc);
+          if (w_scan) {
+            w[e] = sRow[128 + r];
+          } else {
+            const size_t th = (tok0 + min(r, L - 1)) * H + h;
+            w[e] = __ldg(w_chan ? w_src + th * DV + vc : w_src + th);
+          }
         }
       };
       float cw[8];
@@ -735,23 +740,30 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int jb = 0; jb < 32; jb += 8) {
         float nw[8];
         if (jb < 24) ld_w(jb + 8, nw);
-        float x[8], xr[8];  // dV of the block's rows; v dV for a write strength that is scalar per row
+        float x[8], xr[8], vf[8];  // dV of the block's rows; raw v; v dV
         tmem_ld8(tmem_addr(tmem, quarter * 32, COL_U + r0 + jb), x);
+        // the block's raw v before any store of the block (the loads need not wait behind them)
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          vf[e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tDPA + sw128_off(r0 + jb + e, vc, 64)));
         tmem_ld_wait();
+        // global rows of the block: one 64-bit base, then 32-bit strides of H x DV floats
+        const size_t rbase = ((tok0 + r0 + jb) * H + h) * DV + vc;
+        const int rstride = H * DV;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int r = r0 + jb + e;
           *reinterpret_cast<__half *>(tDO + sw128_off(64 + r, vc, 128)) = __float2half_rn(-x[e]);
-          const float vf = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tDPA + sw128_off(r, vc, 64)));
-          xr[e] = vf * x[e];
+          xr[e] = vf[e] * x[e];
           if (r < L) {
-            const size_t th = (tok0 + r) * H + h;
-            g_dv[th * DV + vc] = cw[e] * x[e];
+            const float w = w_sqrt ? tc::sqrt_fast(cw[e]) : cw[e];
+            const size_t o = rbase + static_cast<size_t>(e * rstride);
+            g_dv[o] = w * x[e];
             if (p.beta_v_mode == MODE_CHANNEL) {
-              g_dbeta_v[th * DV + vc] = xr[e];
+              g_dbeta_v[o] = xr[e];
             } else if (p.beta_v_mode == MODE_ABSENT && p.beta_k_mode == MODE_CHANNEL) {
-              // symmetric channel write: d beta_k += 0.5 v dV / sqrt(beta_k), stored now, added to below
-              g_dbeta_k[th * DK + vc] = cw[e] > 0.f ? 0.5f * __fdividef(xr[e], cw[e]) : 0.f;
+              // symmetric channel write (dk = dv): d beta_k += 0.5 v dV / sqrt(beta_k), stored now, added to below
+              g_dbeta_k[o] = w > 0.f ? 0.5f * __fdividef(xr[e], w) : 0.f;
             }
           }
         }
@@ -898,14 +910,25 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tmem_ld8(tmem_addr(tmem, quarter * 32, COL_BS + r0 + jb), dq);
           tmem_ld8(tmem_addr(tmem, quarter * 32, COL_BS + 64 + r0 + jb), db);
           tmem_ld8(tmem_addr(tmem, quarter * 32, COL_U + r0 + jb), da);
+          // the block's shared-memory operands before any store of the block
+          float gmv[8], qvv[8], kvv[8], alv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            gmv[e] = sGam[(jb + e) * NT + tid];
+            alv[e] = sAl[(jb + e) * NT + tid];
+            qvv[e] = raw_at(tTP, r0 + jb + e);
+            kvv[e] = raw_at(tWY, r0 + jb + e);
+          }
           tmem_ld_wait();
+          const size_t obase = ((tok0 + r0 + jb) * H + h) * DK + i;  // row r0 + jb; rows H x DK floats apart
+          const int ostride = H * DK;
           float xg[8], xb[8];  // dgamma gamma and d beta_k per row, for gates that are scalar per row
 #pragma unroll
           for (int e = 7; e >= 0; --e) {
             const int j = jb + e, r = r0 + j;
             const bool valid = r < L;
-            const float gm = sGam[j * NT + tid], ginv = __fdividef(1.f, gm);
-            const float qv = raw_at(tTP, r), kv = raw_at(tWY, r);
+            const float gm = gmv[e], ginv = __fdividef(1.f, gm);
+            const float qv = qvv[e], kv = kvv[e];
             const float sbt = valid ? tc::sqrt_fast(cb[e]) : 0.f;
             const float scv = kScaled ? (valid ? cs[e] : 0.f) : 1.f;
             const float bv = sbt * kv, av = scv * bv, dav = da[e] * ginv;
@@ -918,12 +941,12 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const float dbk = sbt > 0.f ? 0.5f * kv * __fdividef(dbt, sbt) : 0.f;
             xb[e] = dbk;
             if (valid) {
-              const size_t o = ((tok0 + r) * H + h) * DK + i;
+              const size_t o = obase + static_cast<size_t>(e * ostride);
               g_dq[o] = gm * dq[e];
               g_dk[o] = sbt * dbt;
               if constexpr (kScaled) g_ds[o] = bv * dav;
               if (p.beta_k_mode == MODE_CHANNEL) g_dbeta_k[o] = cp[e] + dbk;
-              if (p.alpha_mode == MODE_CHANNEL && half == 1) g_dalpha[o] = acc / sAl[j * NT + tid];
+              if (p.alpha_mode == MODE_CHANNEL && half == 1) g_dalpha[o] = acc / alv[e];
             }
           }
           if (p.beta_k_mode != MODE_CHANNEL) {  // summed over channels: rows r0 + jb + (lane & 7)
@@ -970,14 +993,22 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tmem_ld8(tmem_addr(tmem, quarter * 32, COL_BS + r0 + jb), dq);
           tmem_ld8(tmem_addr(tmem, quarter * 32, COL_BS + 64 + r0 + jb), db);
           tmem_ld8(tmem_addr(tmem, quarter * 32, COL_U + r0 + jb), da);
+          float qvv[8], kvv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            qvv[e] = raw_at(tTP, r0 + jb + e);
+            kvv[e] = raw_at(tWY, r0 + jb + e);
+          }
           tmem_ld_wait();
+          const size_t obase = ((tok0 + r0 + jb) * H + h) * DK + i;  // row r0 + jb; rows H x DK floats apart
+          const int ostride = H * DK;
           float xg[8], xb[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int r = r0 + jb + e;
             const bool valid = r < L;
             const float gm = sRow[r], ginv = sRow[64 + r], sbt = sRow[128 + r];
-            const float qv = raw_at(tTP, r), kv = raw_at(tWY, r);
+            const float qv = qvv[e], kv = kvv[e];
             const float scv = kScaled ? (valid ? cs[e] : 0.f) : 1.f;
             const float bv = sbt * kv, av = scv * bv, dav = da[e] * ginv;
             float dg = qv * dq[e] + bv * db[e] - av * dav * ginv;
@@ -986,7 +1017,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const float dbt = gm * db[e] + scv * dav;
             xb[e] = sbt > 0.f ? 0.5f * kv * __fdividef(dbt, sbt) : 0.f;
             if (valid) {
-              const size_t o = ((tok0 + r) * H + h) * DK + i;
+              const size_t o = obase + static_cast<size_t>(e * ostride);
               g_dq[o] = gm * dq[e];
               g_dk[o] = sbt * dbt;
               if constexpr (kScaled) g_ds[o] = bv * dav;
