@@ -101,7 +101,8 @@ __device__ __forceinline__ bool mbar_test_cluster(uint64_t *bar, uint32_t parity
 template <typename IO, bool kChanGates, bool kScaled>
 __global__ void __launch_bounds__(NT, 1)
 chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
+                      const Params p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_qk, bar_lmma, bar_cmma, bar_out, bar_v;
   __shared__ uint64_t bar_full[NSLOT], bar_free[NSLOT], bar_land[NSLOT];
@@ -147,6 +148,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_a);
   }
   tc_fence_before();
   __syncthreads();
@@ -176,10 +178,17 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
     for (int i = 0; i < 4 * RGL; ++i) pal[i] = pbe[i] = 1.f;
 
+    // channel-wise decays arrive by TMA with q and k, into the slot's Ac and [T; P] tiles (free until
+    // K1 writes them): four 128-byte-swizzled boxes of 32 channels x 64 rows, fp32
+    const bool a_tma = kChanGates && p.alpha_mode == MODE_CHANNEL;
     auto issue_qk = [&](int c) {  // raw q and k of chunk c, in place into slot c % 3
       const int t0 = c * C;
       uint8_t *X = sm + slot_off(c % NSLOT);
-      mbar_arrive_expect_tx(&bar_qk, 4 * 64 * 128);
+      mbar_arrive_expect_tx(&bar_qk, 4 * 64 * 128 + (a_tma ? 4 * 64 * 128 : 0));
+      if (a_tma) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tma_load_4d(X + SAC + i * 64 * 128, &tm_a, &bar_qk, 32 * i, h, tt0 + t0, tb);
+      }
       tma_load_4d(X + 64 * 128, &tm_q, &bar_qk, 0, h, tt0 + t0, tb);
       tma_load_4d(X + SX_CB + 64 * 128, &tm_q, &bar_qk, 64, h, tt0 + t0, tb);
       tma_load_4d(X, &tm_k, &bar_qk, 0, h, tt0 + t0, tb);
@@ -210,7 +219,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // thread ltid: 128-byte line (ltid & 3) of row (ltid >> 2) of each channel-wise gate
         const size_t th = thb + static_cast<size_t>(min(ltid >> 2, L - 1)) * H;
         const size_t off = th * DK + (ltid & 3) * 32;
-        if (p.alpha_mode == MODE_CHANNEL) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.alpha + off));
+        // channel alpha: the TMA L2 prefetch two own chunks ahead covers it
         if (p.beta_k_mode == MODE_CHANNEL) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.beta_k + off));
       }
     };
@@ -221,11 +230,7 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       for (int j = 0; j < RGL; ++j) {  // 16-byte loads: four channels of a row per request
         const size_t th = thb + static_cast<size_t>(min(rgl * RGL + j, L - 1)) * H;
         if (p.alpha_mode == MODE_CHANNEL) {
-          const float4 a = __ldg(reinterpret_cast<const float4 *>(p.alpha + th * DK + c0));
-          pal[4 * j] = a.x;
-          pal[4 * j + 1] = a.y;
-          pal[4 * j + 2] = a.z;
-          pal[4 * j + 3] = a.w;
+          // by TMA (read in K1)
         } else if (p.alpha_mode == MODE_SCALAR) {
           pal[4 * j] = __ldg(p.alpha + th);
         }
@@ -290,6 +295,8 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tma_prefetch_l2_4d(&tm_q, x, h, tt0 + c * C, tb);
         tma_prefetch_l2_4d(&tm_k, x, h, tt0 + c * C, tb);
       }
+      if (a_tma)
+        for (int x = 0; x < DK; x += 32) tma_prefetch_l2_4d(&tm_a, x, h, tt0 + c * C, tb);
     };
     if (rank < nchunks) {
       if (ltid == kIo) {
@@ -370,6 +377,20 @@ chunk_fwd_ring_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (!(amax < kF16Max)) raise_status(p.status, STATUS_RANGE);
       } else {
         float *sPX = reinterpret_cast<float *>(tTP);  // row-group gate products, 8 x 128 fp32
+        if (a_tma) {  // my rows' decays from the TMA boxes (box c0 / 32, 16-byte chunk of 4 channels)
+          const uint8_t *abox = X + SAC + (c0 >> 5) * (64 * 128);
+          const uint32_t ach = static_cast<uint32_t>((c0 & 31) >> 2);
+#pragma unroll
+          for (int jj = 0; jj < RGL; ++jj) {
+            const int row = rgl * RGL + jj;
+            const float4 a = *reinterpret_cast<const float4 *>(abox + row * 128 + ((ach ^ static_cast<uint32_t>(row & 7)) << 4));
+            pal[4 * jj] = a.x;
+            pal[4 * jj + 1] = a.y;
+            pal[4 * jj + 2] = a.z;
+            pal[4 * jj + 3] = a.w;
+          }
+          bar_sync(BAR_LOCAL, NL);  // every thread has read its decays before sPX and Ac overwrite them
+        }
 #pragma unroll
         for (int jj = 0; jj < RGL; ++jj) {
           const bool valid = rgl * RGL + jj < L;

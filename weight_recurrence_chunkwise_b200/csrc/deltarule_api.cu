@@ -190,6 +190,11 @@ dr_status tc_ring_launch(const dr_problem *p, const int *cu, const void *q, cons
       !make_map(&mk, bf, 2, k, mB, p->T, p->H, p->dk, 64, tc::C, sw) ||
       !make_map(&mv, bf, 2, v, mB, p->T, p->H, p->dv, tc::VS, tc::C, sw))
     return DR_ERR_CUDA;
+  // channel-wise decays: 32-channel (128-byte) boxes of 64 rows; otherwise unused by the kernel
+  alignas(64) CUtensorMap ma = mq;
+  if (p->alpha_mode == DR_CHANNEL &&
+      !make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, alpha, mB, p->T, p->H, p->dk, 32, tc::C, sw))
+    return DR_ERR_CUDA;
   tc::Params prm{p->T, p->H, p->dv, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v, p->beta_v_mode,
                  S0, o, S_T, status, s_scale, cu, states};
   const bool chan_gates = p->alpha_mode == DR_CHANNEL || p->beta_k_mode != DR_SCALAR;
@@ -213,7 +218,7 @@ dr_status tc_ring_launch(const dr_problem *p, const int *cu, const void *q, cons
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, prm) != cudaSuccess) return DR_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ma, prm) != cudaSuccess) return DR_ERR_CUDA;
   return launch_status();
 }
 
