@@ -74,13 +74,13 @@ def decode_bytes(B, H, dk, dv, io=2, alpha_ch=True, beta_ch=True):
 RING_SOURCES = ("chunk_tc3.cuh", "chunk_tc.cuh", "tri_inverse.cuh", "sm100.cuh", "common.cuh")
 BWD_CHUNK_SOURCES = ("backward_chunk.cuh",) + RING_SOURCES
 MEASURED_TRAFFIC = {
-    ("chunk_fwd_ring_kernel", "gdn_bf16"): ("c36b98adf557", 248.92e6, RING_SOURCES),
-    ("chunk_fwd_ring_kernel", "kda_bf16"): ("c36b98adf557", 531.82e6, RING_SOURCES),
-    ("chunk_fwd_ring_kernel", "fg2plus_bf16"): ("c36b98adf557", 4 * 664.91e6, RING_SOURCES),  # T = 8192 x 4
+    ("chunk_fwd_ring_kernel", "gdn_bf16"): ("c4c8aa6942ac", 249.20e6, RING_SOURCES),
+    ("chunk_fwd_ring_kernel", "kda_bf16"): ("c4c8aa6942ac", 530.25e6, RING_SOURCES),
+    ("chunk_fwd_ring_kernel", "fg2plus_bf16"): ("c4c8aa6942ac", 4 * 663.67e6, RING_SOURCES),  # T = 8192 x 4
     ("chunk_fwd_simt_kernel", "deltanet_f32"): ("31898eacf605", 0.4628e6, ("chunk_simt.cuh", "common.cuh")),
     ("decode_stream_kernel", "decode_bf16"): ("6cb82d40c1fd", 1031.005696e6, ("decode_stream.cuh", "common.cuh")),
     ("delta_rule_bwd_kernel", "gdn_bf16"): ("9a0d1d786d6e", 10536.615e6, ("backward.cuh", "common.cuh")),
-    ("chunk_bwd_kernel", "gdn_bf16"): ("6264e935a60b", 4 * 207.73e6, BWD_CHUNK_SOURCES),  # T = 1024 x 4
+    ("chunk_bwd_kernel", "gdn_bf16"): ("c6645f4c852d", 4 * 207.79e6, BWD_CHUNK_SOURCES),  # T = 1024 x 4
 }
 
 def decode_kernel_name(heads, sms=148):
