@@ -840,6 +840,20 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       __syncwarp();
     }
+    // the per-channel stage's decays (channel i = srow, rows 32 half ..), requested while the products run
+    float s12a[kChanGates ? 32 : 1];
+    if constexpr (kChanGates) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int r = 32 * half + j;
+        const size_t th = (tok0 + min(r, L - 1)) * H + h;
+        s12a[j] = 1.f;
+        if (r < L) {
+          if (p.alpha_mode == MODE_CHANNEL) s12a[j] = __ldg(g_alpha + th * DK + srow);
+          else if (p.alpha_mode == MODE_SCALAR) s12a[j] = __ldg(g_alpha + th);
+        }
+      }
+    }
     if (!wait_mma()) { ok = false; break; }
 
     // ------------------------------------------------------------------ per key channel: gate gradients and outputs
@@ -860,21 +874,10 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // gamma of my rows: forward products (the lower half passes its product to the upper half)
         float prod = 1.f;
         {
-          float a[32];  // all loads in flight together
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const int r = r0 + j;
-            const size_t th = (tok0 + min(r, L - 1)) * H + h;
-            a[j] = 1.f;
-            if (r < L) {
-              if (p.alpha_mode == MODE_CHANNEL) a[j] = __ldg(g_alpha + th * DK + i);
-              else if (p.alpha_mode == MODE_SCALAR) a[j] = __ldg(g_alpha + th);
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            sAl[j * NT + tid] = a[j];
-            prod *= a[j];
+            sAl[j * NT + tid] = s12a[j];
+            prod *= s12a[j];
           }
         }
         if (half == 0) sXC[i] = prod;
@@ -946,7 +949,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               g_dk[o] = sbt * dbt;
               if constexpr (kScaled) g_ds[o] = bv * dav;
               if (p.beta_k_mode == MODE_CHANNEL) g_dbeta_k[o] = cp[e] + dbk;
-              if (p.alpha_mode == MODE_CHANNEL && half == 1) g_dalpha[o] = acc / alv[e];
+              if (p.alpha_mode == MODE_CHANNEL && half == 1) g_dalpha[o] = __fdividef(acc, alv[e]);
             }
           }
           if (p.beta_k_mode != MODE_CHANNEL) {  // summed over channels: rows r0 + jb + (lane & 7)
@@ -973,7 +976,7 @@ chunk_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           const float off = sXC[128 + i];
 #pragma unroll 4
           for (int j = 0; j < 32; ++j)
-            if (j < L) g_dalpha[((tok0 + j) * H + h) * DK + i] = (sSuf[j * NT + tid] + off) / sAl[j * NT + tid];
+            if (j < L) g_dalpha[((tok0 + j) * H + h) * DK + i] = __fdividef(sSuf[j * NT + tid] + off, sAl[j * NT + tid]);
         }
       } else {
         // gates scalar per row (the scan's gamma, 1/gamma, sqrt(beta_k) in shared memory); the per-row
