@@ -80,7 +80,7 @@ MEASURED_TRAFFIC = {
     ("chunk_fwd_simt_kernel", "deltanet_f32"): ("31898eacf605", 0.4628e6, ("chunk_simt.cuh", "common.cuh")),
     ("decode_stream_kernel", "decode_bf16"): ("6cb82d40c1fd", 1031.005696e6, ("decode_stream.cuh", "common.cuh")),
     ("delta_rule_bwd_kernel", "gdn_bf16"): ("9a0d1d786d6e", 10536.615e6, ("backward.cuh", "common.cuh")),
-    ("chunk_bwd_kernel", "gdn_bf16"): ("c6645f4c852d", 4 * 207.79e6, BWD_CHUNK_SOURCES),  # T = 1024 x 4
+    ("chunk_bwd_kernel", "gdn_bf16"): ("b945780a1cf8", 4 * 207.81e6, BWD_CHUNK_SOURCES),  # T = 1024 x 4
 }
 
 def decode_kernel_name(heads, sms=148):
