@@ -72,6 +72,7 @@ def decode_bytes(B, H, dk, dv, io=2, alpha_ch=True, beta_ch=True):
 # voids the number, and the workload it was taken on, so other workloads report none.  Captures on
 # a shorter sequence of the same workload (T noted in the profile) are scaled by T to a full launch.
 RING_SOURCES = ("chunk_tc3.cuh", "chunk_tc.cuh", "tri_inverse.cuh", "sm100.cuh", "common.cuh")
+QUAD_SOURCES = ("chunk_tc4.cuh", "chunk_tc.cuh", "tri_inverse.cuh", "sm100.cuh", "common.cuh")
 BWD_CHUNK_SOURCES = ("backward_chunk.cuh",) + RING_SOURCES
 MEASURED_TRAFFIC = {
     ("chunk_fwd_ring_kernel", "gdn_bf16"): ("c4c8aa6942ac", 249.20e6, RING_SOURCES),
@@ -89,10 +90,14 @@ def decode_kernel_name(heads, sms=148):
     return "decode_stream_kernel" if heads > sms else "decode_step_kernel"
 
 
-def prefill_kernel_name(p):
-    """The prefill kernel the library runs for a problem (the dispatch of dr_chunk_fwd)."""
+def prefill_kernel_name(p, ws_bytes=256):
+    """The prefill kernel the library runs for a problem (the dispatch of dr_chunk_fwd).  For the
+    cluster shapes, the library asks for factor staging in the workspace (dr_chunk_fwd_workspace
+    above the 256-byte status word) exactly when it runs the four-CTA kernel."""
     if p.io == "bf16" and p.dk == 128 and p.chunk == 64:
-        return "chunk_fwd_ring_kernel" if p.dv == 128 else "chunk_fwd_tc_kernel"
+        if p.dv != 128:
+            return "chunk_fwd_tc_kernel"
+        return "chunk_fwd_quad_kernel" if ws_bytes > 256 else "chunk_fwd_ring_kernel"
     return "chunk_fwd_simt_kernel"
 
 
@@ -355,13 +360,13 @@ def run_backward(args, dr, p, x, dev, st, peaks, peaks_src):
 
 
 # ----------------------------------------------------------------------------- our arm
-def prefill_roofline(p, ms, peaks, peaks_src, with_S0=False):
+def prefill_roofline(p, ms, peaks, peaks_src, with_S0=False, ws_bytes=256):
     """Roofline of one prefill launch: HBM-bound on algorithmic counts (SURVEY-style work model)."""
     byts = prefill_bytes(p, with_S0=with_S0)
     flops = p.token_heads * flops_per_token_head(p.dk, p.dv, p.chunk)
     gbs = byts / (ms / 1e3) / 1e9
     t_roof_ms = max(byts / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops_sustained"] * 1e12)) * 1e3
-    kern = prefill_kernel_name(p)
+    kern = prefill_kernel_name(p, ws_bytes)
     return {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
             "traffic": measured_traffic(kern, p.name), "peak_source": peaks_src, "kernel": kern,
             "algorithmic_bytes_per_launch": byts, "algorithmic_flops_per_launch": flops,
@@ -377,7 +382,8 @@ def time_prefill_workload(dr, p, dev, st, steps, warmup, ws, peaks, peaks_src):
     x = to_dev(make_inputs(p), dev)
     o = torch.empty_like(x["v"])
     S = torch.empty((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=dev)
-    wsb = torch.zeros(256, dtype=torch.uint8, device=dev)
+    need = dr.workspace_bytes(dr.make_problem(x["q"], x["v"], x["alpha"], x["beta_k"], x["beta_v"], p.chunk))
+    wsb = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
     in_bytes = sum(t.numel() * t.element_size() for t in x.values() if t is not None)
     flush = None if in_bytes > L2_BYTES else torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
     run = lambda: dr.dr_chunk_fwd(x["q"], x["k"], x["v"], x["beta_k"], alpha=x["alpha"], beta_v=x["beta_v"],
@@ -407,7 +413,7 @@ def time_prefill_workload(dr, p, dev, st, steps, warmup, ws, peaks, peaks_src):
             "io": p.io, "alpha": p.alpha, "beta_k": p.beta_k, "beta_v": p.beta_v, "S0": p.S0,
             "ms": ms, "value": p.token_heads * ws / (ms / 1e3) / 1e6, "unit": "Mtokens·heads/s", "launches": steps,
             "l2": "inputs larger than L2, no flush" if flush is None else "L2 flushed (256 MiB write) between launches",
-            "roofline": prefill_roofline(p, ms, peaks, peaks_src, with_S0=x["S0"] is not None)}
+            "roofline": prefill_roofline(p, ms, peaks, peaks_src, with_S0=x["S0"] is not None, ws_bytes=need)}
 
 
 def main():
@@ -544,7 +550,7 @@ def main():
     handoff_ms = max_over_ranks(statistics.mean(e[2].elapsed_time(e[3]) for e in ev), ws, dev)
     tok_heads = p.B * p.H * (p.T + 1)
     value = tok_heads * ws / (ms_step / 1e3) / 1e6
-    roofline = prefill_roofline(p, prefill_ms, peaks, peaks_src)
+    roofline = prefill_roofline(p, prefill_ms, peaks, peaks_src, ws_bytes=ws_buf.numel())
     workloads[WORKLOAD] = {"workload": p.name, "B": p.B, "H": p.H, "T": p.T, "dk": p.dk, "dv": p.dv,
                            "chunk": p.chunk, "ms": prefill_ms, "value": p.token_heads * ws / (prefill_ms / 1e3) / 1e6,
                            "unit": "Mtokens·heads/s", "launches": n, "l2": "inputs larger than L2, no flush",

@@ -96,7 +96,13 @@ typedef struct {
   dr_mode beta_v_mode;  /* DR_ABSENT, DR_SCALAR or DR_CHANNEL (per value channel) */
 } dr_problem;
 
-/* Bytes of device workspace dr_chunk_fwd needs for problem p (status word).  0 if p is invalid. */
+/*
+ * Bytes of device workspace dr_chunk_fwd needs for problem p: the status word
+ * (256 bytes), plus, when the library runs the four-CTA prefill (bf16, dk =
+ * dv = 128, chunk 64, and no more heads B*H than clusters of four CTAs the
+ * GPU holds at once), 266,240 bytes per (b, h) where it stages each chunk's
+ * factor block.  0 if p is invalid.
+ */
 DR_API size_t dr_chunk_fwd_workspace(const dr_problem *p);
 
 /*
@@ -239,9 +245,10 @@ DR_API dr_status dr_backward(const dr_problem *p,
  * takes the same inputs and outputs as dr_chunk_fwd but no workspace: the
  * scratch dr_chunk_fwd would keep in the workspace (its device status word)
  * lives in a file-scope device array of 4096 bytes inside the library, which
- * every GPU that loads the library holds until the process exits.  A problem
- * whose dr_chunk_fwd_workspace() exceeds 4096 bytes is rejected with
- * DR_ERR_WORKSPACE before anything is enqueued.  The call allocates nothing
+ * every GPU that loads the library holds until the process exits.  Where
+ * dr_chunk_fwd would pick the four-CTA prefill, whose factor staging does not
+ * fit in that array, this call runs the two-CTA prefill, which needs the
+ * status word only; the outputs are the same.  The call allocates nothing
  * (no cudaMalloc, no cudaFree, no allocating library routine).
  * Device and set-up: the GPU used is the current device, which must be the
  * device of `stream` and the device that holds q; a q on another device is

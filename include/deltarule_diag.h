@@ -34,10 +34,17 @@ extern "C" {
  *              library's choice for such shapes when dv != 128
  *   variant 2  the CUDA-core kernel (every supported shape; the library's
  *              choice for fp32 I/O and for chunk 16 and 32)
- * Arguments, layouts, ownership and errors are those of dr_chunk_fwd; a
- * variant that cannot take the problem returns DR_ERR_UNSUPPORTED before
- * anything is enqueued.  Every variant computes the same operation.
+ *   variant 3  the two-CTA cluster kernel (bf16 I/O, dk = dv = 128, chunk
+ *              64); the library's choice for such shapes with more heads
+ *              than resident four-CTA clusters
+ *   variant 4  the four-CTA cluster kernel (same shapes); the library's
+ *              choice for them otherwise
+ * Arguments, layouts, ownership and errors are those of dr_chunk_fwd, with
+ * a workspace of dr_diag_chunk_fwd_workspace(variant, p) bytes; a variant
+ * that cannot take the problem returns DR_ERR_UNSUPPORTED before anything
+ * is enqueued.  Every variant computes the same operation.
  */
+DR_API size_t dr_diag_chunk_fwd_workspace(int variant, const dr_problem *p);
 DR_API int dr_diag_chunk_fwd_variant(int variant, const dr_problem *p, const void *q, const void *k,
                                      const void *v, const float *alpha, const float *beta_k,
                                      const float *beta_v, const float *S0, void *o, float *S_T,

@@ -301,7 +301,8 @@ def test_extreme_decay_sets_range_status(dr):
     x = make_inputs(p)
     x["alpha"] = torch.full_like(x["alpha"], 1e-3)  # sum log alpha over a chunk ~ -442
     g = to_dev(x)
-    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    need = dr.workspace_bytes(dr.make_problem(g["q"], g["v"], g["alpha"], g["beta_k"], None, 64))
+    ws = torch.zeros(max(need, 256), dtype=torch.uint8, device="cuda")
     dr.dr_chunk_fwd(g["q"], g["k"], g["v"], g["beta_k"], alpha=g["alpha"], chunk=64, workspace=ws)
     assert dr.dr_workspace_status(ws) == dr.DR_ERR_RANGE
     # and a normal call afterwards clears it

@@ -2,8 +2,10 @@
 
 The library's choice (dr_chunk_fwd) and the other kernels, named through
 dr_diag_chunk_fwd_variant (include/deltarule_diag.h): the tensor-core kernel with one CTA per
-64-column value slice, and the CUDA-core kernel.  Cases cover ragged lengths, one to many chunks
-(the factor-slot ring wraps several times), scalar and channel gates, and the symmetric and
+64-column value slice, the CUDA-core kernel, and the two cluster kernels (two CTAs per head with a
+ring of factor slots; four CTAs per head with the factor blocks staged through global memory).
+Cases cover ragged lengths, one to many chunks (the factor slots and staging entries wrap several
+times), fewer chunks than CTAs in a cluster, scalar and channel gates, and the symmetric and
 separate write strengths; each result is checked against the float64 oracle.
 """
 import zlib
@@ -15,6 +17,7 @@ pytestmark = pytest.mark.gpu
 CASES = [
     # (T, alpha, beta_k, beta_v, S0)
     (1, "scalar", "scalar", "none", "zero"),
+    (129, "channel", "scalar", "none", "normal"),
     (63, "scalar", "scalar", "none", "normal"),
     (200, "scalar", "scalar", "scalar", "normal"),
     (453, "none", "scalar", "none", "zero"),
@@ -26,7 +29,7 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("variant", ["default", "single", "simt"])
+@pytest.mark.parametrize("variant", ["default", "single", "simt", "ring", "quad"])
 def test_prefill_kernel_variant(variant):
     import torch
 

@@ -3,10 +3,12 @@
 It serves callers that cannot allocate device memory -- runtimes that
 pre-plan all device memory and offer a kernel no workspace, or loops that
 cannot pay for cudaMalloc/cudaFree -- by keeping its scratch in a static
-device array inside the library.  It runs the same kernel as the allocating
-entry point dr_chunk_fwd on the same inputs, so its results must be the same
-bits, call after call: the shared array keeps the previous call's contents,
-so two different problems are run back to back.  Its device status word is
+device array inside the library.  For the cluster-kernel shapes it runs the
+two-CTA kernel (the four-CTA kernel's factor staging does not fit the array),
+so its results must be the bits of that kernel run through the allocating
+entry point (dr_diag_chunk_fwd_variant "ring"), call after call: the shared
+array keeps the previous call's contents, so two different problems are run
+back to back.  Its device status word is
 read back through dr_noalloc_status.  The file is named to be collected last.
 """
 import pytest
@@ -34,7 +36,7 @@ def test_noalloc_matches_allocating_entry_point_twice():
         x = _dev(make_inputs(p))
         args = (x["q"], x["k"], x["v"], x["beta_k"])
         kw = dict(alpha=x["alpha"], beta_v=x["beta_v"], S0=x["S0"], chunk=p.chunk)
-        o_ref, S_ref = dr.dr_chunk_fwd(*args, **kw)
+        o_ref, S_ref = dr.dr_diag_chunk_fwd_variant("ring", *args, **kw)
         o_new = torch.full_like(o_ref, float("nan"))
         S_new = torch.full_like(S_ref, float("nan"))
         dr.dr_chunk_fwd_noalloc(*args, **kw, o=o_new, S_T=S_new)

@@ -42,11 +42,12 @@ EXPORTS = ("dr_chunk_fwd_workspace", "dr_chunk_fwd", "dr_chunk_fwd_osdn", "dr_ch
            "dr_chunk_fwd_noalloc", "dr_decode_step",
            "dr_decode_step_osdn", "dr_state_map_apply", "dr_backward_workspace", "dr_backward",
            "dr_workspace_status", "dr_noalloc_status", "dr_status_string", "dr_version", "dr_diag_umma_selftest",
-           "dr_diag_tri_inverse", "dr_diag_wait_timeout", "dr_diag_chunk_fwd_variant", "dr_diag_decode_step_variant",
+           "dr_diag_tri_inverse", "dr_diag_wait_timeout", "dr_diag_chunk_fwd_workspace", "dr_diag_chunk_fwd_variant",
+           "dr_diag_decode_step_variant",
            "dr_diag_backward_workspace", "dr_diag_backward_variant")
 
 # kernels of dr_diag_chunk_fwd_variant / dr_diag_decode_step_variant (include/deltarule_diag.h)
-PREFILL_VARIANTS = {"default": 0, "single": 1, "simt": 2}
+PREFILL_VARIANTS = {"default": 0, "single": 1, "simt": 2, "ring": 3, "quad": 4}
 DECODE_VARIANTS = {"default": 0, "per_head": 1, "split4": 2, "stream": 3}
 BACKWARD_VARIANTS = {"default": 0, "sequential": 1, "chunk": 2}
 
@@ -93,6 +94,8 @@ def lib():
         L.dr_diag_tri_inverse.restype = ctypes.c_int
         L.dr_diag_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_ulonglong, vp, vp, vp]
         L.dr_diag_wait_timeout.restype = ctypes.c_int
+        L.dr_diag_chunk_fwd_workspace.argtypes = [ctypes.c_int, P]
+        L.dr_diag_chunk_fwd_workspace.restype = sz
         L.dr_diag_chunk_fwd_variant.argtypes = [ctypes.c_int, P] + [vp] * 9 + [vp, sz, vp]
         L.dr_diag_chunk_fwd_variant.restype = ctypes.c_int
         L.dr_diag_decode_step_variant.argtypes = [ctypes.c_int, P] + [vp] * 9 + [vp]
@@ -269,7 +272,7 @@ def _chunk_fwd(s, q, k, v, beta_k, alpha, beta_v, S0, chunk, o, S_T, workspace, 
                              ("beta_k", beta_k), ("beta_v", beta_v), ("s", s), ("S0", S0), ("S_T", S_T)])
     if s is not None and tuple(s.shape) != tuple(q.shape):
         raise ValueError("s must have the shape of q / k: [B, T, H, dk]")
-    need = workspace_bytes(p)
+    need = workspace_bytes(p) if variant is None else int(lib().dr_diag_chunk_fwd_workspace(int(variant), ctypes.byref(p)))
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     elif workspace.device != dev:

@@ -14,6 +14,7 @@
 #include "chunk_simt.cuh"
 #include "chunk_tc.cuh"
 #include "chunk_tc3.cuh"
+#include "chunk_tc4.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "decode_stream.cuh"
@@ -29,7 +30,7 @@ constexpr size_t kWorkspaceBytes = 256;  // status word, padded to an allocation
 
 // Prefill kernel variants (the library's choice is kDefault; the others are reachable only through
 // dr_diag_chunk_fwd_variant, for comparisons).
-enum PrefillVariant { kPrefillDefault = 0, kPrefillSingle = 1, kPrefillSimt = 2 };
+enum PrefillVariant { kPrefillDefault = 0, kPrefillSingle = 1, kPrefillSimt = 2, kPrefillRing = 3, kPrefillQuad = 4 };
 // Decode kernel variants, likewise (dr_diag_decode_step_variant).
 enum DecodeVariant { kDecodeDefault = 0, kDecodePerHead = 1, kDecodeSplit4 = 2, kDecodeStream = 3 };
 
@@ -175,6 +176,28 @@ dr_status tc_launch(const dr_problem *p, const void *q, const void *k, const voi
 
 // states: NULL, or [B, H, ceil(T/64), dk, dv] fp32 receiving the state at the start of every chunk
 // (dense batch only; the chunkwise backward's first pass, which passes o = NULL).
+// Tensor maps of the cluster prefills: q, k and v in 64-column boxes of one chunk's rows; the
+// channel-wise decays in 32-channel (128-byte) boxes (otherwise a copy of q's map, unused).
+struct RingMaps {
+  alignas(64) CUtensorMap q, k, v, a;
+};
+bool ring_maps(RingMaps &m, const dr_problem *p, const int *cu, const void *q, const void *k, const void *v,
+               const float *alpha) {
+  namespace tc = dr::tc;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  const int mB = cu ? 1 : p->B;  // a packed batch is one [1, Ttot, H, d] array
+  if (!make_map(&m.q, bf, 2, q, mB, p->T, p->H, p->dk, 64, tc::C, sw) ||
+      !make_map(&m.k, bf, 2, k, mB, p->T, p->H, p->dk, 64, tc::C, sw) ||
+      !make_map(&m.v, bf, 2, v, mB, p->T, p->H, p->dv, tc::VS, tc::C, sw))
+    return false;
+  m.a = m.q;
+  if (p->alpha_mode == DR_CHANNEL &&
+      !make_map(&m.a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, alpha, mB, p->T, p->H, p->dk, 32, tc::C, sw))
+    return false;
+  return true;
+}
+
 dr_status tc_ring_launch(const dr_problem *p, const int *cu, const void *q, const void *k, const void *v,
                          const float *alpha, const float *beta_k, const float *beta_v, const float *s_scale,
                          const float *S0, void *o, float *S_T, uint32_t *status, cudaStream_t st,
@@ -182,19 +205,8 @@ dr_status tc_ring_launch(const dr_problem *p, const int *cu, const void *q, cons
   using IO = __nv_bfloat16;
   namespace tc = dr::tc;
   namespace tc3 = dr::tc3;
-  alignas(64) CUtensorMap mq, mk, mv;
-  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
-  const int mB = cu ? 1 : p->B;  // a packed batch is one [1, Ttot, H, d] array
-  if (!make_map(&mq, bf, 2, q, mB, p->T, p->H, p->dk, 64, tc::C, sw) ||
-      !make_map(&mk, bf, 2, k, mB, p->T, p->H, p->dk, 64, tc::C, sw) ||
-      !make_map(&mv, bf, 2, v, mB, p->T, p->H, p->dv, tc::VS, tc::C, sw))
-    return DR_ERR_CUDA;
-  // channel-wise decays: 32-channel (128-byte) boxes of 64 rows; otherwise unused by the kernel
-  alignas(64) CUtensorMap ma = mq;
-  if (p->alpha_mode == DR_CHANNEL &&
-      !make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, alpha, mB, p->T, p->H, p->dk, 32, tc::C, sw))
-    return DR_ERR_CUDA;
+  RingMaps m;
+  if (!ring_maps(m, p, cu, q, k, v, alpha)) return DR_ERR_CUDA;
   tc::Params prm{p->T, p->H, p->dv, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v, p->beta_v_mode,
                  S0, o, S_T, status, s_scale, cu, states};
   const bool chan_gates = p->alpha_mode == DR_CHANNEL || p->beta_k_mode != DR_SCALAR;
@@ -218,7 +230,96 @@ dr_status tc_ring_launch(const dr_problem *p, const int *cu, const void *q, cons
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ma, prm) != cudaSuccess) return DR_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, m.q, m.k, m.v, m.a, prm) != cudaSuccess) return DR_ERR_CUDA;
+  return launch_status();
+}
+
+// The four-CTA prefill: one cluster of four CTAs per (b, h).
+template <bool kChan, bool kScaled>
+constexpr auto quad_kernel() {
+  return dr::tc4::chunk_fwd_quad_kernel<__nv_bfloat16, kChan, kScaled>;
+}
+using QuadKernel = decltype(quad_kernel<false, false>());
+QuadKernel pick_quad(bool chan, bool scaled) {
+  return scaled ? (chan ? quad_kernel<true, true>() : quad_kernel<false, true>())
+                : (chan ? quad_kernel<true, false>() : quad_kernel<false, false>());
+}
+cudaLaunchConfig_t quad_config(const dr_problem *p, cudaStream_t st, cudaLaunchAttribute *attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(dr::tc4::NCTA, p->H, p->B);
+  cfg.blockDim = dim3(dr::tc4::NT, 1, 1);
+  cfg.dynamicSmemBytes = dr::tc4::SMEM_BYTES;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = dr::tc4::NCTA;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+// Clusters of the four-CTA prefill that the current device holds at once (0: unknown or none);
+// computed once per device.
+int quad_resident_clusters() {
+  static std::mutex mu;
+  static int cached[64];
+  static bool known[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!known[dev]) {
+    int n = 0;
+    bool ok = true;
+    for (int v = 0; v < 4 && ok; ++v) {
+      ok = cudaFuncSetAttribute(pick_quad(v & 1, v & 2), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(dr::tc4::SMEM_BYTES)) == cudaSuccess;
+    }
+    if (ok) {
+      dr_problem one{};
+      one.B = 1;
+      one.H = 1;
+      cudaLaunchAttribute attr[1];
+      cudaLaunchConfig_t cfg = quad_config(&one, nullptr, attr);
+      if (cudaOccupancyMaxActiveClusters(&n, pick_quad(false, false), &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    cached[dev] = n;
+    known[dev] = true;
+  }
+  return cached[dev];
+}
+// Shapes the cluster prefills take: bf16 I/O, dk = dv = 128, chunk 64.
+bool ring_problem(const dr_problem *p) {
+  return p->io_dtype == DR_BF16 && p->dk == dr::tc::DK && p->chunk == dr::tc::C && p->dv == 2 * dr::tc::VS;
+}
+// The library's prefill choice for a problem the cluster kernels take: four CTAs per head when every
+// head's cluster is resident at once (a second wave would double the time), else two.
+bool quad_default(const dr_problem *p) {
+  const long long heads = static_cast<long long>(p->B) * p->H;
+  return heads <= quad_resident_clusters();
+}
+size_t quad_stage_bytes(const dr_problem *p) {
+  return static_cast<size_t>(p->B) * p->H * dr::tc4::STAGE_BYTES_PER_HEAD;
+}
+
+// stage: quad_stage_bytes(p) bytes of device memory, 16-byte aligned.
+dr_status tc_quad_launch(const dr_problem *p, const int *cu, const void *q, const void *k, const void *v,
+                         const float *alpha, const float *beta_k, const float *beta_v, const float *s_scale,
+                         const float *S0, void *o, float *S_T, uint32_t *status, uint8_t *stage, cudaStream_t st,
+                         float *states = nullptr) {
+  namespace tc = dr::tc;
+  RingMaps m;
+  if (!ring_maps(m, p, cu, q, k, v, alpha)) return DR_ERR_CUDA;
+  tc::Params prm{p->T, p->H, p->dv, alpha, p->alpha_mode, beta_k, p->beta_k_mode, beta_v, p->beta_v_mode,
+                 S0, o, S_T, status, s_scale, cu, states};
+  const bool chan_gates = p->alpha_mode == DR_CHANNEL || p->beta_k_mode != DR_SCALAR;
+  auto kern = pick_quad(chan_gates, s_scale != nullptr);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(dr::tc4::SMEM_BYTES)) != cudaSuccess)
+    return DR_ERR_CUDA;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = quad_config(p, st, attr);
+  if (cudaLaunchKernelEx(&cfg, kern, m.q, m.k, m.v, m.a, prm, stage) != cudaSuccess) return DR_ERR_CUDA;
   return launch_status();
 }
 
@@ -300,10 +401,14 @@ dr_status chunk_fwd_impl(const dr_problem *p, const int *cu, const void *q, cons
   uint32_t *status = static_cast<uint32_t *>(workspace);
   // a variant that cannot take the problem is refused before anything is enqueued
   const bool tc_shape = p->io_dtype == DR_BF16 && p->dk == dr::tc::DK && p->chunk == dr::tc::C;
-  const bool ring_shape = tc_shape && p->dv == 2 * dr::tc::VS;
+  const bool ring_shape = ring_problem(p);
   const bool plain = !s_scale && !cu;  // the one-CTA-per-slice kernel takes neither extension
   if (variant == kPrefillSingle && !(plain && tc_shape && p->dv % dr::tc::VS == 0)) return DR_ERR_UNSUPPORTED;
-  if (variant != kPrefillDefault && variant != kPrefillSingle && variant != kPrefillSimt) return DR_ERR_UNSUPPORTED;
+  if ((variant == kPrefillRing || variant == kPrefillQuad) && !ring_shape) return DR_ERR_UNSUPPORTED;
+  if (variant < kPrefillDefault || variant > kPrefillQuad) return DR_ERR_UNSUPPORTED;
+  // the four-CTA kernel stages its factor blocks in the workspace, after the status word
+  const bool quad = ring_shape && (variant == kPrefillQuad || (variant == kPrefillDefault && quad_default(p)));
+  if (quad && workspace_bytes < kWorkspaceBytes + quad_stage_bytes(p)) return DR_ERR_WORKSPACE;
   if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DR_ERR_CUDA;
   const size_t state_bytes = sizeof(float) * size_t(p->B) * p->H * p->dk * p->dv;
   if (p->T == 0) {  // nothing to scan: the final state is the initial state
@@ -317,7 +422,10 @@ dr_status chunk_fwd_impl(const dr_problem *p, const int *cu, const void *q, cons
     return simt_dispatch<float>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
   if (variant == kPrefillSimt)
     return simt_dispatch<__nv_bfloat16>(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
-  if (variant == kPrefillDefault && ring_shape)
+  if (quad)
+    return tc_quad_launch(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status,
+                          static_cast<uint8_t *>(workspace) + kWorkspaceBytes, st);
+  if ((variant == kPrefillDefault || variant == kPrefillRing) && ring_shape)
     return tc_ring_launch(p, cu, q, k, v, alpha, beta_k, beta_v, s_scale, S0, o, S_T, status, st);
   if (plain && tc_shape && p->dv % dr::tc::VS == 0)
     return tc_launch(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, status, st);
@@ -520,7 +628,8 @@ const char *dr_status_string(dr_status s) {
 }
 
 size_t dr_chunk_fwd_workspace(const dr_problem *p) {
-  return check_common(p, false) == DR_OK ? kWorkspaceBytes : 0;
+  if (check_common(p, false) != DR_OK) return 0;
+  return kWorkspaceBytes + (ring_problem(p) && quad_default(p) ? quad_stage_bytes(p) : 0);
 }
 
 dr_status dr_chunk_fwd(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
@@ -595,7 +704,6 @@ dr_status dr_chunk_fwd_noalloc(const dr_problem *p, const void *q, const void *k
                                void *o, float *S_T, void *stream) {
   const dr_status s = check_common(p, false);
   if (s != DR_OK) return s;
-  if (dr_chunk_fwd_workspace(p) > kStaticScratchBytes) return DR_ERR_WORKSPACE;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return DR_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return DR_ERR_UNSUPPORTED;
@@ -617,8 +725,12 @@ dr_status dr_chunk_fwd_noalloc(const dr_problem *p, const void *q, const void *k
     }
     scratch = g_static_addr[dev];
   }
-  // dr_chunk_fwd clears the status word at the start of the call, on `stream`.
-  return dr_chunk_fwd(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, scratch, kStaticScratchBytes, stream);
+  // The status word fits the array; the four-CTA prefill's staging does not, so such problems run
+  // the two-CTA prefill.  The call clears the status word at its start, on `stream`.
+  static_assert(kWorkspaceBytes <= kStaticScratchBytes, "status word");
+  const int variant = dr_chunk_fwd_workspace(p) > kStaticScratchBytes ? kPrefillRing : kPrefillDefault;
+  return chunk_fwd_impl(p, nullptr, q, k, v, alpha, beta_k, beta_v, nullptr, S0, o, S_T, scratch, kStaticScratchBytes,
+                        stream, variant);
 }
 
 dr_status dr_noalloc_status(void *stream) {
@@ -642,6 +754,12 @@ dr_status dr_workspace_status(const void *workspace, void *stream) {
   if (w & dr::STATUS_TIMEOUT) return DR_ERR_TIMEOUT;
   if (w & dr::STATUS_RANGE) return DR_ERR_RANGE;
   return DR_OK;
+}
+
+size_t dr_diag_chunk_fwd_workspace(int variant, const dr_problem *p) {
+  if (check_common(p, false) != DR_OK) return 0;
+  if (variant == kPrefillQuad) return ring_problem(p) ? kWorkspaceBytes + quad_stage_bytes(p) : 0;
+  return variant == kPrefillDefault ? dr_chunk_fwd_workspace(p) : kWorkspaceBytes;
 }
 
 int dr_diag_chunk_fwd_variant(int variant, const dr_problem *p, const void *q, const void *k, const void *v,
