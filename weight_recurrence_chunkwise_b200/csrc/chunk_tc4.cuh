@@ -27,8 +27,8 @@
 //             staging entry may be overwritten (one phase per chunk of that producer)
 //   full[j]   slot j of this CTA holds its chunk (bulk-load bytes)
 // Ordering of the staging memory: the producer's bulk store completes (wait_group 0) and is fenced
-// against the generic proxy before the release arrives; a consumer fences after its acquire before
-// its bulk load.
+// against the generic proxy, then one release fence precedes the (relaxed) arrives; a consumer
+// fences after its acquire before its bulk load.
 #pragma once
 #include "chunk_tc.cuh"
 
@@ -113,6 +113,9 @@ __device__ __forceinline__ void bulk_load_global(void *dst_smem, const void *src
 }
 // Orders this thread's async-proxy accesses (bulk copies) with its generic-proxy ones.
 __device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
+// Release-acquire fence at cluster scope: with it, the relaxed arrives that follow publish this
+// thread's earlier writes like release arrives, for one fence instead of one per arrive.
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 
 // kChanGates: the gates vary per key channel (alpha per channel, or beta_k per channel); else
 // they are one value per row (alpha absent or per token, beta_k per token).
@@ -630,11 +633,13 @@ chunk_fwd_quad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           bulk_store_global(dst + 32768, X + 32768, 32768);
           bulk_store_global(dst + 65536, X + 65536, FAC_BYTES - 65536);
           bulk_store_commit_wait();
+          if (c + NCTA < nchunks) issue_qk(c + NCTA);  // the store has read the working area
+          // the block is in global memory: one release fence orders it before all four arrives
           fence_proxy_async_all();
+          fence_acq_rel_cluster();
 #pragma unroll 1
           for (int r = 0; r < NCTA; ++r)
-            mbar_arrive_remote(mapa_shared(smem_u32(&bar_ready[rank]), static_cast<uint32_t>(r)));
-          if (c + NCTA < nchunks) issue_qk(c + NCTA);
+            mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&bar_ready[rank]), static_cast<uint32_t>(r)));
         } else {
           raise_status(p.status, STATUS_TIMEOUT);  // the next wait for raw q/k then fails for all
         }
@@ -870,7 +875,18 @@ chunk_fwd_quad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           __syncwarp();
         }
       }
-      if (c > 0) store_o(c - 1);  // overlaps the MMAs above
+      // the previous chunk's second MMA group (its outputs, and the last reads of its slot): waited
+      // for here, where the first group of this chunk runs, by the threads that store the outputs
+      // and by the one that requests blocks, which refills the slot with chunk c+1
+      bool ok_out = true;
+      if (c > 0) {
+        if (quarter >= 2 || ct == 128) ok_out = mbar_wait(&bar_out, ph_out & 1u, kWaitLimitNs);
+        ph_out ^= 1u;
+        tc_fence_after();
+        if (!ok_out) raise_status(p.status, STATUS_TIMEOUT);
+        if (ok_out && ct == 128) pump(c + 1);
+        if (ok_out) store_o(c - 1);  // overlaps the MMAs above
+      }
       if (!run) break;
       if (p.states) {  // this chunk's initial state, for the backward pass (dense batches only)
         float *dst = p.states + ((sbase / (static_cast<size_t>(DK) * DV)) * nchunks + c) * DK * DV +
@@ -881,8 +897,8 @@ chunk_fwd_quad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       }
       // MMA group 1 done
       {
-        bool ok = true;
-        if (ct == 0) ok = mbar_wait(&bar_cmma, ph_mma & 1u, kWaitLimitNs);
+        bool ok = ok_out;
+        if (ct == 0) ok = mbar_wait(&bar_cmma, ph_mma & 1u, kWaitLimitNs) && ok;
         ph_mma ^= 1u;
         const bool fail = bar_or(BAR_CHAIN, NT - NL, !ok);
         tc_fence_after();
@@ -931,7 +947,7 @@ chunk_fwd_quad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           umma_commit(&bar_cmma);  // the state update waits for Ac^T U alone
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) umma_f16(tmem + cD3, kstep(dTP, 128, kk), mstep(dU, kk), id_n, 1u);
-          umma_commit(&bar_out);   // the outputs and the slot's reuse wait for this
+          umma_commit(&bar_out);   // the outputs and the slot's reuse wait for this (next iteration)
         }
         __syncwarp();
       }
@@ -969,14 +985,6 @@ chunk_fwd_quad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         __syncwarp();
       }
-      // slot j is free once the outputs' MMAs are done: request chunk c+2 into it -- now if they are
-      // done already, else after E4
-      bool released = false;
-      if (ct == 128 && mbar_test_cluster(&bar_out, ph_out & 1u)) {
-        pump(c + 2);
-        released = true;
-      }
-
       // -------------------------------------------------------------- E4: S <- Diag(gamma_C) (S + Ac^T U)
       {
         float mx = 0.f;
@@ -993,21 +1001,8 @@ chunk_fwd_quad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       }
       fence_async_smem();
       tc_fence_before();
-      {
-        bool ok = true;
-        if (ct == 128 && !released) {
-          ok = mbar_wait(&bar_out, ph_out & 1u, kWaitLimitNs);
-          if (ok) pump(c + 2);
-        }
-        ph_out ^= 1u;
-        const bool fail = bar_or(BAR_CHAIN, NT - NL, !ok);
-        tc_fence_after();
-        if (fail) {
-          if (ct == 128) raise_status(p.status, STATUS_TIMEOUT);
-          aborted = true;
-          break;
-        }
-      }
+      bar_sync(BAR_CHAIN, NT - NL);  // S (fp16) complete for the next chunk's first MMA group
+      tc_fence_after();
     }
     if (!aborted && p.S_T) {
       float *dst = p.S_T + sbase + static_cast<size_t>(trow) * DV + v0 + hc;
