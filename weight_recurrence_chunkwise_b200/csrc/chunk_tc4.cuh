@@ -111,8 +111,8 @@ __device__ __forceinline__ void bulk_load_global(void *dst_smem, const void *src
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
-// Orders this thread's async-proxy accesses (bulk copies) with its generic-proxy ones.
-__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
+// Orders this thread's async-proxy accesses to global memory (bulk copies) with its generic-proxy ones.
+__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 // Release-acquire fence at cluster scope: with it, the relaxed arrives that follow publish this
 // thread's earlier writes like release arrives, for one fence instead of one per arrive.
 __device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
