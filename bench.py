@@ -18,6 +18,7 @@ With N > 1 launch under torch.distributed.run: every rank runs its own batch
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -78,6 +79,8 @@ MEASURED_TRAFFIC = {
     ("chunk_fwd_ring_kernel", "gdn_bf16"): ("c4c8aa6942ac", 249.20e6, RING_SOURCES),
     ("chunk_fwd_ring_kernel", "kda_bf16"): ("c4c8aa6942ac", 530.25e6, RING_SOURCES),
     ("chunk_fwd_ring_kernel", "fg2plus_bf16"): ("c4c8aa6942ac", 4 * 663.67e6, RING_SOURCES),  # T = 8192 x 4
+    ("chunk_fwd_quad_kernel", "kda_bf16"): ("1b1675a62aab", 537.56e6, QUAD_SOURCES),
+    ("chunk_fwd_quad_kernel", "fg2plus_bf16"): ("1b1675a62aab", 4 * 674.51e6, QUAD_SOURCES),  # T = 8192 x 4
     ("chunk_fwd_simt_kernel", "deltanet_f32"): ("31898eacf605", 0.4628e6, ("chunk_simt.cuh", "common.cuh")),
     ("decode_stream_kernel", "decode_bf16"): ("6cb82d40c1fd", 1031.005696e6, ("decode_stream.cuh", "common.cuh")),
     ("delta_rule_bwd_kernel", "gdn_bf16"): ("9a0d1d786d6e", 10536.615e6, ("backward.cuh", "common.cuh")),
@@ -360,13 +363,13 @@ def run_backward(args, dr, p, x, dev, st, peaks, peaks_src):
 
 
 # ----------------------------------------------------------------------------- our arm
-def prefill_roofline(p, ms, peaks, peaks_src, with_S0=False, ws_bytes=256):
+def prefill_roofline(p, ms, peaks, peaks_src, with_S0=False, ws_bytes=256, variant="default"):
     """Roofline of one prefill launch: HBM-bound on algorithmic counts (SURVEY-style work model)."""
     byts = prefill_bytes(p, with_S0=with_S0)
     flops = p.token_heads * flops_per_token_head(p.dk, p.dv, p.chunk)
     gbs = byts / (ms / 1e3) / 1e9
     t_roof_ms = max(byts / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops_sustained"] * 1e12)) * 1e3
-    kern = prefill_kernel_name(p, ws_bytes)
+    kern = {"ring": "chunk_fwd_ring_kernel", "quad": "chunk_fwd_quad_kernel"}.get(variant) or prefill_kernel_name(p, ws_bytes)
     return {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
             "traffic": measured_traffic(kern, p.name), "peak_source": peaks_src, "kernel": kern,
             "algorithmic_bytes_per_launch": byts, "algorithmic_flops_per_launch": flops,
@@ -374,20 +377,30 @@ def prefill_roofline(p, ms, peaks, peaks_src, with_S0=False, ws_bytes=256):
             "frac_of_max_roofline": t_roof_ms / ms}
 
 
-def time_prefill_workload(dr, p, dev, st, steps, warmup, ws, peaks, peaks_src):
+def time_prefill_workload(dr, p, dev, st, steps, warmup, ws, peaks, peaks_src, variant="default"):
     """Prefill alone on one workload: mean CUDA-event duration of each launch, max over ranks.
 
     Inputs larger than L2 need no flush; a smaller workload gets an L2 flush (a 256 MiB write)
-    between launches, outside the per-launch events."""
+    between launches, outside the per-launch events.  `variant` names a kernel of
+    dr_diag_chunk_fwd_variant instead of the library's choice (a profiling aid)."""
     x = to_dev(make_inputs(p), dev)
     o = torch.empty_like(x["v"])
     S = torch.empty((p.B, p.H, p.dk, p.dv), dtype=torch.float32, device=dev)
-    need = dr.workspace_bytes(dr.make_problem(x["q"], x["v"], x["alpha"], x["beta_k"], x["beta_v"], p.chunk))
+    prob = dr.make_problem(x["q"], x["v"], x["alpha"], x["beta_k"], x["beta_v"], p.chunk)
+    if variant == "default":
+        need = dr.workspace_bytes(prob)
+    else:
+        need = int(dr.lib().dr_diag_chunk_fwd_workspace(dr.PREFILL_VARIANTS[variant], ctypes.byref(prob)))
     wsb = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
     in_bytes = sum(t.numel() * t.element_size() for t in x.values() if t is not None)
     flush = None if in_bytes > L2_BYTES else torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
-    run = lambda: dr.dr_chunk_fwd(x["q"], x["k"], x["v"], x["beta_k"], alpha=x["alpha"], beta_v=x["beta_v"],
-                                  S0=x["S0"], chunk=p.chunk, o=o, S_T=S, workspace=wsb, stream=st)
+    if variant == "default":
+        run = lambda: dr.dr_chunk_fwd(x["q"], x["k"], x["v"], x["beta_k"], alpha=x["alpha"], beta_v=x["beta_v"],
+                                      S0=x["S0"], chunk=p.chunk, o=o, S_T=S, workspace=wsb, stream=st)
+    else:
+        run = lambda: dr.dr_diag_chunk_fwd_variant(variant, x["q"], x["k"], x["v"], x["beta_k"], alpha=x["alpha"],
+                                                   beta_v=x["beta_v"], S0=x["S0"], chunk=p.chunk, o=o, S_T=S,
+                                                   workspace=wsb, stream=st)
     for _ in range(warmup):
         run()
     torch.cuda.synchronize()
@@ -413,7 +426,8 @@ def time_prefill_workload(dr, p, dev, st, steps, warmup, ws, peaks, peaks_src):
             "io": p.io, "alpha": p.alpha, "beta_k": p.beta_k, "beta_v": p.beta_v, "S0": p.S0,
             "ms": ms, "value": p.token_heads * ws / (ms / 1e3) / 1e6, "unit": "Mtokens·heads/s", "launches": steps,
             "l2": "inputs larger than L2, no flush" if flush is None else "L2 flushed (256 MiB write) between launches",
-            "roofline": prefill_roofline(p, ms, peaks, peaks_src, with_S0=x["S0"] is not None, ws_bytes=need)}
+            "roofline": prefill_roofline(p, ms, peaks, peaks_src, with_S0=x["S0"] is not None, ws_bytes=need,
+                                         variant=variant)}
 
 
 def main():
@@ -435,6 +449,8 @@ def main():
                     help="with --only-prefill / --backward: the workload to time (default: the headline one)")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (dr_backward) on the --config workload instead")
+    ap.add_argument("--prefill-variant", default="default", choices=["default", "ring", "quad"],
+                    help="with --only-prefill: time the named cluster kernel instead of the library's choice")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="with --only-prefill / --backward: override the workload's T (profiling a shorter case "
                          "of the same shape; the line reports the T it ran)")
@@ -470,7 +486,8 @@ def main():
     if args.seqpar_cost:
         return run_seqpar_cost(args, dr, rank_problem(rank, args.config), dev, st)
     if args.only_prefill:
-        line = time_prefill_workload(dr, aid_problem(), dev, st, args.steps, args.warmup, ws, peaks, peaks_src)
+        line = time_prefill_workload(dr, aid_problem(), dev, st, args.steps, args.warmup, ws, peaks, peaks_src,
+                                     variant=args.prefill_variant)
         if rank == 0:
             print(json.dumps({"only_prefill": True, "prefill_ms": line["ms"], **line}), flush=True)
         return 0
