@@ -76,7 +76,7 @@ typedef enum {
   DR_ERR_INVALID_ARG = 1,   /* NULL required pointer, negative size, mode/shape mismatch */
   DR_ERR_UNSUPPORTED = 2,   /* valid but not implemented: sizes outside the lists above */
   DR_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned */
-  DR_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than dr_chunk_fwd_workspace() */
+  DR_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than the entry point needs (see its comment) */
   DR_ERR_RANGE = 5,         /* device: cumulative decay inside a chunk below the factorised range */
   DR_ERR_TIMEOUT = 6,       /* device: a bounded wait expired; outputs are invalid */
   DR_ERR_CUDA = 7           /* a CUDA runtime call or kernel launch failed */
@@ -114,7 +114,9 @@ DR_API size_t dr_chunk_fwd_workspace(const dr_problem *p);
  * step 7; FG2-GDN page, section 2, DPLR/WY remark).
  * workspace: device memory of at least dr_chunk_fwd_workspace(p) bytes,
  * reused across calls on the same stream; its status word is reset at the
- * start of every call.
+ * start of every call.  A workspace that holds the status word but not the
+ * four-CTA prefill's staging runs the two-CTA prefill instead (the same
+ * operation; slower on batches with few heads).
  */
 DR_API dr_status dr_chunk_fwd(const dr_problem *p,
                        const void *q, const void *k, const void *v,
@@ -248,7 +250,7 @@ DR_API dr_status dr_backward(const dr_problem *p,
  * every GPU that loads the library holds until the process exits.  Where
  * dr_chunk_fwd would pick the four-CTA prefill, whose factor staging does not
  * fit in that array, this call runs the two-CTA prefill, which needs the
- * status word only; the outputs are the same.  The call allocates nothing
+ * status word only; it computes the same operation.  The call allocates nothing
  * (no cudaMalloc, no cudaFree, no allocating library routine).
  * Device and set-up: the GPU used is the current device, which must be the
  * device of `stream` and the device that holds q; a q on another device is

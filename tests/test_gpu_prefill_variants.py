@@ -65,3 +65,29 @@ def test_unsupported_variant_is_refused():
     with pytest.raises(dr.DeltaRuleError) as e:
         dr.dr_diag_chunk_fwd_variant("single", g["q"], g["k"], g["v"], g["beta_k"], alpha=g["alpha"], chunk=64)
     assert e.value.code == dr.DR_ERR_UNSUPPORTED
+
+
+def test_workspace_size_selects_the_cluster_kernel():
+    """The library's choice with a workspace that holds only the status word is the two-CTA kernel's
+    result, bit for bit; with dr_chunk_fwd_workspace bytes it is the four-CTA kernel's."""
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import weight_recurrence_chunkwise_b200 as dr
+    from synth import make_inputs, problem
+
+    p = problem("kda_bf16", B=1, H=2, T=300, dk=128, dv=128, chunk=64, io="bf16", alpha="channel",
+                beta_k="channel", beta_v="none", S0="normal", seed=11)
+    g = {n: (None if t is None else t.cuda()) for n, t in make_inputs(p).items()}
+    args = (g["q"], g["k"], g["v"], g["beta_k"])
+    kw = dict(alpha=g["alpha"], beta_v=g["beta_v"], S0=g["S0"], chunk=64)
+    need = dr.workspace_bytes(dr.make_problem(g["q"], g["v"], g["alpha"], g["beta_k"], g["beta_v"], 64))
+    assert need > 256  # two heads: the four-CTA kernel's clusters are resident
+    o_small, S_small = dr.dr_chunk_fwd(*args, **kw, workspace=torch.zeros(256, dtype=torch.uint8, device="cuda"))
+    o_ring, S_ring = dr.dr_diag_chunk_fwd_variant("ring", *args, **kw)
+    o_full, S_full = dr.dr_chunk_fwd(*args, **kw)
+    o_quad, S_quad = dr.dr_diag_chunk_fwd_variant("quad", *args, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(o_small, o_ring) and torch.equal(S_small, S_ring)
+    assert torch.equal(o_full, o_quad) and torch.equal(S_full, S_quad)

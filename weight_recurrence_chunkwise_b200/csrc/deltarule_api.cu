@@ -406,9 +406,12 @@ dr_status chunk_fwd_impl(const dr_problem *p, const int *cu, const void *q, cons
   if (variant == kPrefillSingle && !(plain && tc_shape && p->dv % dr::tc::VS == 0)) return DR_ERR_UNSUPPORTED;
   if ((variant == kPrefillRing || variant == kPrefillQuad) && !ring_shape) return DR_ERR_UNSUPPORTED;
   if (variant < kPrefillDefault || variant > kPrefillQuad) return DR_ERR_UNSUPPORTED;
-  // the four-CTA kernel stages its factor blocks in the workspace, after the status word
-  const bool quad = ring_shape && (variant == kPrefillQuad || (variant == kPrefillDefault && quad_default(p)));
-  if (quad && workspace_bytes < kWorkspaceBytes + quad_stage_bytes(p)) return DR_ERR_WORKSPACE;
+  // The four-CTA kernel stages its factor blocks in the workspace, after the status word.  The
+  // library's choice takes it only when the workspace holds that staging (dr_chunk_fwd_workspace
+  // asks for it); a workspace with the status word alone runs the two-CTA kernel.
+  const bool quad_fits = workspace_bytes >= kWorkspaceBytes + quad_stage_bytes(p);
+  if (variant == kPrefillQuad && ring_shape && !quad_fits) return DR_ERR_WORKSPACE;
+  const bool quad = ring_shape && (variant == kPrefillQuad || (variant == kPrefillDefault && quad_fits && quad_default(p)));
   if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DR_ERR_CUDA;
   const size_t state_bytes = sizeof(float) * size_t(p->B) * p->H * p->dk * p->dv;
   if (p->T == 0) {  // nothing to scan: the final state is the initial state
@@ -726,11 +729,10 @@ dr_status dr_chunk_fwd_noalloc(const dr_problem *p, const void *q, const void *k
     scratch = g_static_addr[dev];
   }
   // The status word fits the array; the four-CTA prefill's staging does not, so such problems run
-  // the two-CTA prefill.  The call clears the status word at its start, on `stream`.
+  // the two-CTA prefill (the library's choice for a workspace of that size).  The call clears the
+  // status word at its start, on `stream`.
   static_assert(kWorkspaceBytes <= kStaticScratchBytes, "status word");
-  const int variant = dr_chunk_fwd_workspace(p) > kStaticScratchBytes ? kPrefillRing : kPrefillDefault;
-  return chunk_fwd_impl(p, nullptr, q, k, v, alpha, beta_k, beta_v, nullptr, S0, o, S_T, scratch, kStaticScratchBytes,
-                        stream, variant);
+  return dr_chunk_fwd(p, q, k, v, alpha, beta_k, beta_v, S0, o, S_T, scratch, kStaticScratchBytes, stream);
 }
 
 dr_status dr_noalloc_status(void *stream) {
