@@ -224,7 +224,9 @@ DR_API dr_status dr_state_map_apply(int n, int dk, int dv, const float *M, const
  *            dS0 [B,H,dk,dv] or NULL (not wanted).  A gate's gradient at beta = 0
  *            is reported as 0 (the square root has no derivative there).
  *   workspace >= dr_backward_workspace(p) bytes, 16-byte aligned, device memory
- *            (fp32 state checkpoints and per-head recomputation scratch).
+ *            (fp32 state checkpoints and per-head recomputation scratch; for
+ *            the chunkwise kernel, also the four-CTA prefill's factor staging
+ *            when its first pass runs on that kernel).
  * dk, dv in {64, 128}; fp32 or bf16 I/O.  Asynchronous on `stream`.  Errors as
  * dr_chunk_fwd, plus DR_ERR_INVALID_ARG for a missing or extra gradient buffer.
  */

@@ -484,9 +484,19 @@ enum BackwardVariant { kBwdDefault = 0, kBwdSequential = 1, kBwdChunk = 2 };
 
 bool bwd_chunk_shape(const dr_problem *p) { return p->io_dtype == DR_BF16 && p->dk == 128 && p->dv == 128; }
 
-size_t bwd_chunk_workspace_bytes(const dr_problem *p) {
+// The chunkwise backward's workspace: the status word, the chunk-start states, and (when its
+// first pass runs on the four-CTA prefill) that kernel's factor staging.
+size_t bwd_chunk_states_bytes(const dr_problem *p) {
   const size_t nc = (static_cast<size_t>(p->T) + dr::tc::C - 1) / dr::tc::C;
-  return kWorkspaceBytes + sizeof(float) * static_cast<size_t>(p->B) * p->H * nc * p->dk * p->dv;
+  return sizeof(float) * static_cast<size_t>(p->B) * p->H * nc * p->dk * p->dv;
+}
+bool bwd_first_pass_quad(const dr_problem *p) {
+  dr_problem pf = *p;
+  pf.chunk = dr::tc::C;
+  return ring_problem(&pf) && quad_default(&pf);
+}
+size_t bwd_chunk_workspace_bytes(const dr_problem *p) {
+  return kWorkspaceBytes + bwd_chunk_states_bytes(p) + (bwd_first_pass_quad(p) ? quad_stage_bytes(p) : 0);
 }
 
 int resolve_bwd_variant(const dr_problem *p, int variant) {
@@ -501,15 +511,24 @@ size_t bwd_variant_workspace_bytes(const dr_problem *p, int variant) {
 dr_status bwd_chunk_launch(const dr_problem *p, const void *q, const void *k, const void *v, const float *alpha,
                            const float *beta_k, const float *beta_v, const float *s, const float *S0,
                            const void *dout, const float *dS_T, float *dq, float *dk, float *dv, float *dalpha,
-                           float *dbeta_k, float *dbeta_v, float *ds, float *dS0, void *workspace, cudaStream_t st) {
+                           float *dbeta_k, float *dbeta_v, float *ds, float *dS0, void *workspace,
+                           size_t workspace_bytes, cudaStream_t st) {
   namespace bwc = dr::bwc;
   uint32_t *status = static_cast<uint32_t *>(workspace);
-  float *states = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kWorkspaceBytes);
+  uint8_t *ws8 = static_cast<uint8_t *>(workspace);
+  float *states = reinterpret_cast<float *>(ws8 + kWorkspaceBytes);
+  uint8_t *stage = ws8 + kWorkspaceBytes + bwd_chunk_states_bytes(p);
   if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DR_ERR_CUDA;
   dr_problem pf = *p;
   pf.chunk = dr::tc::C;
-  dr_status r = tc_ring_launch(&pf, nullptr, q, k, v, alpha, beta_k, beta_v, s, S0, nullptr, nullptr, status, st,
-                               states);
+  // first pass: the prefill with every chunk's initial state stored (no outputs), on the kernel the
+  // forward would use when the workspace holds its staging
+  const bool quad = bwd_first_pass_quad(p) &&
+                    workspace_bytes >= kWorkspaceBytes + bwd_chunk_states_bytes(p) + quad_stage_bytes(p);
+  dr_status r = quad ? tc_quad_launch(&pf, nullptr, q, k, v, alpha, beta_k, beta_v, s, S0, nullptr, nullptr, status,
+                                      stage, st, states)
+                     : tc_ring_launch(&pf, nullptr, q, k, v, alpha, beta_k, beta_v, s, S0, nullptr, nullptr, status,
+                                      st, states);
   if (r != DR_OK) return r;
   alignas(64) CUtensorMap mq, mk, mv, mdo;
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -585,7 +604,7 @@ static dr_status backward_impl(int variant, const dr_problem *p, const void *q, 
   if (!workspace || workspace_bytes < bwd_variant_workspace_bytes(p, variant)) return DR_ERR_WORKSPACE;
   if (resolve_bwd_variant(p, variant) == kBwdChunk)
     return bwd_chunk_launch(p, q, k, v, alpha, beta_k, beta_v, s, S0, dout, dS_T, dq, dk, dv, dalpha, dbeta_k,
-                            dbeta_v, ds, dS0, workspace, cs);
+                            dbeta_v, ds, dS0, workspace, workspace_bytes, cs);
   float *ws = static_cast<float *>(workspace);
   {  // the per-key-channel gradients are sums over value-column slices, accumulated in place
     const size_t tok = static_cast<size_t>(p->B) * p->T * p->H;
