@@ -41,3 +41,18 @@ def test_backward_bytes():
     per_out = 4 * (2 * 128 + 128) + 4 + 4                           # fp32 dq, dk, dv, gate gradients
     state = p.B * p.H * 128 * 128 * 4                               # S0, dS_T read; dS0 written
     assert bench.backward_bytes(p) == p.token_heads * (per_in + per_out) + 3 * state
+
+
+def test_prefill_kernel_names_follow_the_dispatch():
+    """The bench names the kernel the library runs: for the cluster shapes, the four-CTA kernel
+    exactly when dr_chunk_fwd_workspace asks for more than the 256-byte status word (its factor
+    staging), else the two-CTA ring; other shapes their own kernels."""
+    fg2 = problem("fg2plus_bf16")
+    assert bench.prefill_kernel_name(fg2, 256) == "chunk_fwd_ring_kernel"
+    assert bench.prefill_kernel_name(fg2, 256 + fg2.B * fg2.H * 266240) == "chunk_fwd_quad_kernel"
+    assert bench.prefill_kernel_name(problem("gdn_bf16", dv=64), 256) == "chunk_fwd_tc_kernel"
+    assert bench.prefill_kernel_name(problem("deltanet_f32"), 256) == "chunk_fwd_simt_kernel"
+    # traffic is keyed per (kernel, workload) and tied to the kernel's sources
+    for kern, wl in (("chunk_fwd_quad_kernel", "fg2plus_bf16"), ("chunk_fwd_quad_kernel", "kda_bf16"),
+                     ("chunk_fwd_ring_kernel", "gdn_bf16")):
+        assert (kern, wl) in bench.MEASURED_TRAFFIC
